@@ -1,0 +1,301 @@
+/*
+ * attention_oracle.c -- TEST INFRASTRUCTURE, NOT PART OF THE PRODUCT PATH.
+ *
+ * A plain, slow, obviously correct CPU implementation of the exact attention forward
+ *
+ *     O = softmax(scale * Q K^T  [+ causal mask]) V ,   LSE_i = ln sum_j exp(S_ij)
+ *
+ * in IEEE fp64, written straight from the definition.  Only the test suite, the
+ * smoke check and the benchmark's CPU-baseline leg may load it.  It shares no code,
+ * header, table or helper with the CUDA library; the two only see the same seeded
+ * bf16 inputs.
+ *
+ * Where each step comes from:
+ *  - the formula softmax(Q K^T / sqrt(d_k)) V and its three-step listing (scores,
+ *    softmax, weighted sum), with S and P materialised as full N x N matrices:
+ *    hwcomputing.csdn.net article on FlashAttention in CANN ops-transformer, section
+ *    "where the memory black hole of standard attention comes from";
+ *  - the softmax definition softmax(x_i) = e^{x_i} / sum_j e^{x_j}: same article,
+ *    section "online softmax: keeping block-wise computation exact";
+ *  - causal mask ("only see content before the current position") and no mask:
+ *    same article, "performance tuning" item 3 (mask modes);
+ *  - GQA: query head h uses KV head floor(h / n_rep), n_rep = Hq / Hkv, i.e. the
+ *    repeat_interleave(n_rep, dim=1) expansion of K and V: "Transformer efficient
+ *    attention: Flash Attention vs GQA" (yunthe.com), section "GQA principle and
+ *    implementation";
+ *  - tensor layout [batch, seq, heads, head_dim]: same yunthe.com page, the
+ *    flash_attn_func call in section "Flash Attention IO optimisation".
+ *
+ * Readings where the pages are silent (each also listed in the design notes):
+ *  - the causal mask keeps the diagonal (key j visible to query i iff j <= i) and,
+ *    for Nq != Nk, is aligned to the bottom-right: j <= i + (Nk - Nq);
+ *  - a row with no visible key (only possible when Nq > Nk under the causal mask,
+ *    or Nk == 0) has O = 0 and LSE = -inf, the limit of an empty sum;
+ *  - LSE is the natural-log log-sum-exp of the scaled, masked logits;
+ *  - inputs are bf16 bit patterns, widened exactly to fp64; nothing is rounded
+ *    in between.
+ *
+ * Softmax is taken in two passes over the materialised row (row max M_i first,
+ * then exp(S_ij - M_i)), the textbook way to keep exp() in range.
+ *
+ * Compile-time ORACLE_PLANT_* macros build deliberately wrong variants; the test
+ * suite uses them to show that its pins catch each kind of mistake.  A normal build
+ * defines none of them.
+ */
+#include <math.h>
+#include <pthread.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#define ORACLE_OK 0
+#define ORACLE_EINVAL -1
+#define ORACLE_ENOMEM -2
+#define ORACLE_ETHREAD -3
+
+static double bf16_bits_to_double(uint16_t bits) {
+    uint32_t u = (uint32_t)bits << 16;
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return (double)f;
+}
+
+typedef struct {
+    const uint16_t *q, *k, *v;
+    int B, Hq, Hkv, Nq, Nk, d;
+    double scale;
+    int causal;
+} problem_t;
+
+static int kv_head_of(const problem_t *p, int hq) {
+#ifdef ORACLE_PLANT_GQA_MODULO
+    return hq % p->Hkv;
+#else
+    return hq / (p->Hq / p->Hkv);
+#endif
+}
+
+static int key_visible(const problem_t *p, int i, int j) {
+    if (!p->causal) return 1;
+#ifdef ORACLE_PLANT_CAUSAL_STRICT
+    return (long)j < (long)i + (long)(p->Nk - p->Nq);
+#else
+    return (long)j <= (long)i + (long)(p->Nk - p->Nq);
+#endif
+}
+
+static double q_at(const problem_t *p, int b, int i, int h, int c) {
+    return bf16_bits_to_double(p->q[(((size_t)b * p->Nq + i) * p->Hq + h) * p->d + c]);
+}
+static double k_at(const problem_t *p, int b, int j, int g, int c) {
+    return bf16_bits_to_double(p->k[(((size_t)b * p->Nk + j) * p->Hkv + g) * p->d + c]);
+}
+static double v_at(const problem_t *p, int b, int j, int g, int c) {
+#ifdef ORACLE_PLANT_TRANSPOSE_V
+    c = p->d - 1 - c;
+#endif
+    return bf16_bits_to_double(p->v[(((size_t)b * p->Nk + j) * p->Hkv + g) * p->d + c]);
+}
+
+/*
+ * One query row of one (b, hq): fills srow[0..Nk) with S_i. (scores, then masked),
+ * turns it into the probability row P_i. in place, and writes O_i. (d values) and
+ * LSE_i.  Step numbers follow the three-step standard listing.
+ */
+static void attention_row(const problem_t *p, int b, int hq, int i, double *srow,
+                          double *o_row, double *lse_out) {
+    const int g = kv_head_of(p, hq);
+    const int Nk = p->Nk, d = p->d;
+
+    /* step 1: scores S_ij = scale * sum_c Q[i,c] K[j,c]; masked entries -> -inf */
+    for (int j = 0; j < Nk; ++j) {
+        if (!key_visible(p, i, j)) { srow[j] = -INFINITY; continue; }
+        double acc = 0.0;
+        for (int c = 0; c < d; ++c) acc += q_at(p, b, i, hq, c) * k_at(p, b, j, g, c);
+#ifdef ORACLE_PLANT_NO_SCALE
+        srow[j] = acc;
+#else
+        srow[j] = p->scale * acc;
+#endif
+    }
+
+    /* step 2: softmax over the row, two passes: M = max_j S_ij, Z = sum_j exp(S_ij - M) */
+    double M = -INFINITY;
+    for (int j = 0; j < Nk; ++j) if (srow[j] > M) M = srow[j];
+    if (M == -INFINITY) {               /* no visible key: empty sum */
+        for (int c = 0; c < d; ++c) o_row[c] = 0.0;
+        for (int j = 0; j < Nk; ++j) srow[j] = 0.0;
+        *lse_out = -INFINITY;
+        return;
+    }
+    double Z = 0.0;
+    for (int j = 0; j < Nk; ++j) {
+        srow[j] = exp(srow[j] - M);     /* exp(-inf) = 0 for masked keys */
+        Z += srow[j];
+    }
+#ifndef ORACLE_PLANT_NO_NORMALIZE
+    for (int j = 0; j < Nk; ++j) srow[j] /= Z;
+#endif
+#ifdef ORACLE_PLANT_LSE_NO_MAX
+    *lse_out = log(Z);
+#else
+    *lse_out = M + log(Z);
+#endif
+
+    /* step 3: weighted sum O_i. = sum_j P_ij V_j. */
+    for (int c = 0; c < d; ++c) o_row[c] = 0.0;
+    for (int j = 0; j < Nk; ++j) {
+        const double pij = srow[j];
+        if (pij == 0.0) continue;
+        for (int c = 0; c < d; ++c) o_row[c] += pij * v_at(p, b, j, g, c);
+    }
+}
+
+/* ---- full forward: S and P materialised per (b, hq), rows split across threads ---- */
+
+typedef struct {
+    const problem_t *p;
+    int b, hq, i0, i1;
+    double *S;          /* Nq x Nk for this (b, hq), shared; each thread owns its rows */
+    double *out, *lse;  /* whole outputs */
+    double *probs;      /* optional [B,Hq,Nq,Nk] copy of P */
+} head_job_t;
+
+static void *head_rows_worker(void *arg) {
+    head_job_t *jb = (head_job_t *)arg;
+    const problem_t *p = jb->p;
+    for (int i = jb->i0; i < jb->i1; ++i) {
+        double *srow = jb->S + (size_t)i * p->Nk;
+        double *o_row = jb->out + (((size_t)jb->b * p->Nq + i) * p->Hq + jb->hq) * p->d;
+        double *l = jb->lse + ((size_t)jb->b * p->Hq + jb->hq) * p->Nq + i;
+        attention_row(p, jb->b, jb->hq, i, srow, o_row, l);
+        if (jb->probs) {
+            double *dst = jb->probs + (((size_t)jb->b * p->Hq + jb->hq) * p->Nq + i) * p->Nk;
+            memcpy(dst, srow, sizeof(double) * (size_t)p->Nk);
+        }
+    }
+    return NULL;
+}
+
+static int check_problem(const problem_t *p) {
+    if (p->B < 0 || p->Hq <= 0 || p->Hkv <= 0 || p->Nq < 0 || p->Nk < 0 || p->d <= 0) return 0;
+    if (p->Hq % p->Hkv != 0) return 0;
+    if (!isfinite(p->scale)) return 0;
+    return 1;
+}
+
+static int run_full(const problem_t *p, double *out, double *lse, double *probs, int nthreads) {
+    if (!check_problem(p)) return ORACLE_EINVAL;
+    if (nthreads < 1) nthreads = 1;
+    if (p->B == 0 || p->Nq == 0) return ORACLE_OK;
+    const size_t nk_alloc = p->Nk > 0 ? (size_t)p->Nk : 1;
+    double *S = (double *)malloc(sizeof(double) * (size_t)p->Nq * nk_alloc);
+    if (!S) return ORACLE_ENOMEM;
+    pthread_t *tid = (pthread_t *)malloc(sizeof(pthread_t) * (size_t)nthreads);
+    head_job_t *jobs = (head_job_t *)malloc(sizeof(head_job_t) * (size_t)nthreads);
+    if (!tid || !jobs) { free(S); free(tid); free(jobs); return ORACLE_ENOMEM; }
+    int rc = ORACLE_OK;
+    for (int b = 0; b < p->B && rc == ORACLE_OK; ++b) {
+        for (int hq = 0; hq < p->Hq && rc == ORACLE_OK; ++hq) {
+            int nt = nthreads < p->Nq ? nthreads : p->Nq;
+            int started = 0;
+            for (int t = 0; t < nt; ++t) {
+                jobs[t] = (head_job_t){p, b, hq, (int)((long)p->Nq * t / nt),
+                                       (int)((long)p->Nq * (t + 1) / nt), S, out, lse, probs};
+                if (nt == 1) { head_rows_worker(&jobs[t]); continue; }
+                if (pthread_create(&tid[t], NULL, head_rows_worker, &jobs[t]) != 0) {
+                    rc = ORACLE_ETHREAD;
+                    break;
+                }
+                ++started;
+            }
+            for (int t = 0; t < started; ++t) pthread_join(tid[t], NULL);
+        }
+    }
+    free(S);
+    free(tid);
+    free(jobs);
+    return rc;
+}
+
+/*
+ * oracle_attention_fwd: the whole forward.
+ *   q [B,Nq,Hq,d], k/v [B,Nk,Hkv,d]: bf16 bit patterns (host memory).
+ *   out [B,Nq,Hq,d] fp64, lse [B,Hq,Nq] fp64 (natural log).
+ * Returns 0, or a negative code (bad sizes, no memory, thread failure).
+ */
+int oracle_attention_fwd(const uint16_t *q, const uint16_t *k, const uint16_t *v,
+                         double *out, double *lse, int B, int Hq, int Hkv, int Nq, int Nk,
+                         int d, double scale, int causal, int nthreads) {
+    problem_t p = {q, k, v, B, Hq, Hkv, Nq, Nk, d, scale, causal ? 1 : 0};
+    return run_full(&p, out, lse, NULL, nthreads);
+}
+
+/*
+ * oracle_attention_probs: as oracle_attention_fwd, and also copies the
+ * probability matrix P into probs [B,Hq,Nq,Nk] (tiny problems only).
+ */
+int oracle_attention_probs(const uint16_t *q, const uint16_t *k, const uint16_t *v,
+                           double *out, double *lse, double *probs, int B, int Hq, int Hkv,
+                           int Nq, int Nk, int d, double scale, int causal) {
+    problem_t p = {q, k, v, B, Hq, Hkv, Nq, Nk, d, scale, causal ? 1 : 0};
+    return run_full(&p, out, lse, probs, 1);
+}
+
+/* ---- selected rows: the same definition evaluated only for listed (b, hq, i) ---- */
+
+typedef struct {
+    const problem_t *p;
+    const int32_t *rows;   /* triples (b, hq, i) */
+    long r0, r1;
+    double *out_rows;      /* [nrows, d] */
+    double *lse_rows;      /* [nrows] */
+    int rc;
+} rows_job_t;
+
+static void *rows_worker(void *arg) {
+    rows_job_t *jb = (rows_job_t *)arg;
+    const problem_t *p = jb->p;
+    double *srow = (double *)malloc(sizeof(double) * (size_t)(p->Nk > 0 ? p->Nk : 1));
+    if (!srow) { jb->rc = ORACLE_ENOMEM; return NULL; }
+    for (long r = jb->r0; r < jb->r1; ++r) {
+        int b = jb->rows[3 * r], hq = jb->rows[3 * r + 1], i = jb->rows[3 * r + 2];
+        attention_row(p, b, hq, i, srow, jb->out_rows + r * p->d, jb->lse_rows + r);
+    }
+    free(srow);
+    return NULL;
+}
+
+/*
+ * oracle_attention_rows: O and LSE of the listed rows only.
+ *   rows: nrows triples (b, hq, i), each in range; out_rows [nrows, d]; lse_rows [nrows].
+ */
+int oracle_attention_rows(const uint16_t *q, const uint16_t *k, const uint16_t *v,
+                          const int32_t *rows, long nrows, double *out_rows, double *lse_rows,
+                          int B, int Hq, int Hkv, int Nq, int Nk, int d, double scale,
+                          int causal, int nthreads) {
+    problem_t p = {q, k, v, B, Hq, Hkv, Nq, Nk, d, scale, causal ? 1 : 0};
+    if (!check_problem(&p) || nrows < 0) return ORACLE_EINVAL;
+    for (long r = 0; r < nrows; ++r) {
+        int b = rows[3 * r], hq = rows[3 * r + 1], i = rows[3 * r + 2];
+        if (b < 0 || b >= B || hq < 0 || hq >= Hq || i < 0 || i >= Nq) return ORACLE_EINVAL;
+    }
+    if (nthreads < 1) nthreads = 1;
+    if (nrows == 0) return ORACLE_OK;
+    int nt = (long)nthreads < nrows ? nthreads : (int)nrows;
+    pthread_t *tid = (pthread_t *)malloc(sizeof(pthread_t) * (size_t)nt);
+    rows_job_t *jobs = (rows_job_t *)malloc(sizeof(rows_job_t) * (size_t)nt);
+    if (!tid || !jobs) { free(tid); free(jobs); return ORACLE_ENOMEM; }
+    int started = 0, rc = ORACLE_OK;
+    for (int t = 0; t < nt; ++t) {
+        jobs[t] = (rows_job_t){&p, rows, nrows * t / nt, nrows * (t + 1) / nt, out_rows, lse_rows, 0};
+        if (nt == 1) { rows_worker(&jobs[t]); continue; }
+        if (pthread_create(&tid[t], NULL, rows_worker, &jobs[t]) != 0) { rc = ORACLE_ETHREAD; break; }
+        ++started;
+    }
+    for (int t = 0; t < started; ++t) pthread_join(tid[t], NULL);
+    for (int t = 0; t < nt && rc == ORACLE_OK; ++t) if (jobs[t].rc) rc = jobs[t].rc;
+    free(tid);
+    free(jobs);
+    return rc;
+}

@@ -1,0 +1,292 @@
+"""Independent checks ("pins") of the CPU oracle.  None of them calls back into the
+oracle's own arithmetic; each states a fact the pages or plain mathematics fix:
+
+* brute force in 40-digit decimal arithmetic, straight from softmax(x_i) = e^{x_i} /
+  sum_j e^{x_j} (no max subtraction needed at that precision);
+* closed forms of special cases (one key, constant V, zero Q, causal row 0);
+* invariants (P rows sum to one, GQA equals MHA with K/V repeated per the
+  repeat_interleave expansion, key permutation invariance, causal = non-causal on
+  the visible prefix);
+* a second statement of the method: the block-wise online-softmax recurrence of the
+  hwcomputing.csdn.net FlashAttention article (section "online softmax"), with the
+  scale applied, run in fp64 at several block sizes.
+
+Each pin is a function taking an oracle object and raising AssertionError on a
+mismatch, so the mutation test can run every pin against deliberately broken builds.
+"""
+from __future__ import annotations
+
+import math
+from decimal import Decimal, getcontext
+
+import numpy as np
+
+import synth
+
+TOL = 1e-12
+
+
+def bits_f64(bits):
+    return synth.bf16_bits_to_f32(bits).astype(np.float64)
+
+
+def tiny_inputs(B, Hq, Hkv, Nq, Nk, d, seed, q_mult=1.0):
+    w = synth.Workload("tiny", 1000 + seed, B, Hq, Hkv, Nq, Nk, d, False, q_mult=q_mult, seed=seed)
+    return synth.make_inputs(w)
+
+
+def visible(i, j, Nq, Nk, causal):
+    """Causal reading: keep the diagonal, align bottom-right (j <= i + Nk - Nq)."""
+    return (not causal) or j <= i + (Nk - Nq)
+
+
+# ---------------------------------------------------------------- brute force
+
+def brute_force_decimal(x, scale, causal, prec=40):
+    """O and LSE by the definition in `prec`-digit decimal arithmetic (tiny inputs)."""
+    getcontext().prec = prec
+    q, k, v = (bits_f64(x[n]) for n in ("q", "k", "v"))
+    B, Nq, Hq, d = q.shape
+    _, Nk, Hkv, _ = k.shape
+    rep = Hq // Hkv
+    D = Decimal
+    sc = D(float(scale))
+    O = np.zeros((B, Nq, Hq, d))
+    L = np.zeros((B, Hq, Nq))
+    kd = [[[[D(float(k[b, j, g, c])) for c in range(d)] for g in range(Hkv)] for j in range(Nk)] for b in range(B)]
+    vd = [[[[D(float(v[b, j, g, c])) for c in range(d)] for g in range(Hkv)] for j in range(Nk)] for b in range(B)]
+    for b in range(B):
+        for h in range(Hq):
+            g = h // rep
+            for i in range(Nq):
+                qi = [D(float(q[b, i, h, c])) for c in range(d)]
+                num = [D(0)] * d
+                Z = D(0)
+                for j in range(Nk):
+                    if not visible(i, j, Nq, Nk, causal):
+                        continue
+                    s = sc * sum(qi[c] * kd[b][j][g][c] for c in range(d))
+                    e = s.exp()
+                    Z += e
+                    for c in range(d):
+                        num[c] += e * vd[b][j][g][c]
+                if Z == 0:
+                    O[b, i, h, :] = 0.0
+                    L[b, h, i] = -math.inf
+                else:
+                    O[b, i, h, :] = [float(n / Z) for n in num]
+                    L[b, h, i] = float(Z.ln())
+    return O, L
+
+
+# ---------------------------------------------------------------- second statement
+
+def online_softmax_blocks(x, scale, causal, block):
+    """The block-wise recurrence: running row max m, running sum l, output rescaled by
+    exp(m_old - m_new) at every block, divided by l at the end (fp64)."""
+    q, k, v = (bits_f64(x[n]) for n in ("q", "k", "v"))
+    B, Nq, Hq, d = q.shape
+    _, Nk, Hkv, _ = k.shape
+    rep = Hq // Hkv
+    O = np.zeros((B, Nq, Hq, d))
+    L = np.zeros((B, Hq, Nq))
+    ii = np.arange(Nq)[:, None]
+    for b in range(B):
+        for h in range(Hq):
+            g = h // rep
+            Q = q[b, :, h, :]
+            m = np.full(Nq, -np.inf)
+            l = np.zeros(Nq)
+            acc = np.zeros((Nq, d))
+            for j0 in range(0, Nk, block):
+                Kb = k[b, j0:j0 + block, g, :]
+                Vb = v[b, j0:j0 + block, g, :]
+                s = scale * (Q @ Kb.T)
+                if causal:
+                    jj = np.arange(j0, j0 + Kb.shape[0])[None, :]
+                    s = np.where(jj <= ii + (Nk - Nq), s, -np.inf)
+                m_new = np.maximum(m, s.max(axis=1))
+                safe = np.where(np.isfinite(m_new), m_new, 0.0)
+                corr = np.where(np.isfinite(m), np.exp(m - safe), 0.0)
+                p = np.exp(s - safe[:, None])
+                acc = acc * corr[:, None] + p @ Vb
+                l = l * corr + p.sum(axis=1)
+                m = m_new
+            nz = l > 0
+            O[b, :, h, :] = np.where(nz[:, None], acc / np.where(nz, l, 1.0)[:, None], 0.0)
+            L[b, h, :] = np.where(nz, m + np.log(np.where(nz, l, 1.0)), -np.inf)
+    return O, L
+
+
+def assert_close(a, b, tol=TOL, what=""):
+    a, b = np.asarray(a), np.asarray(b)
+    assert a.shape == b.shape, (what, a.shape, b.shape)
+    fin = np.isfinite(b)
+    assert np.array_equal(np.isfinite(a), fin), f"{what}: finiteness differs"
+    assert np.array_equal(a[~fin], b[~fin]), f"{what}: infinities differ"
+    if fin.any():
+        err = np.abs(a[fin] - b[fin]) / np.maximum(1.0, np.abs(b[fin]))
+        assert err.max() <= tol, f"{what}: max rel err {err.max():.3e} > {tol}"
+
+
+# ---------------------------------------------------------------- the pins
+
+BRUTE_CASES = [
+    # B, Hq, Hkv, Nq, Nk, d, causal, seed
+    (1, 1, 1, 5, 7, 32, False, 1),
+    (1, 2, 1, 6, 6, 64, True, 2),
+    (2, 4, 2, 9, 9, 16, True, 3),
+    (1, 4, 1, 11, 5, 80, True, 4),     # Nq > Nk: first rows see no key
+    (1, 2, 2, 4, 13, 96, True, 5),     # Nq < Nk: bottom-right alignment
+    (1, 1, 1, 3, 4, 128, False, 6),
+    (1, 3, 3, 3, 3, 192, False, 7),
+    (1, 1, 1, 2, 3, 256, True, 8),
+]
+
+
+def pin_brute_force(orc):
+    for (B, Hq, Hkv, Nq, Nk, d, causal, seed) in BRUTE_CASES:
+        x = tiny_inputs(B, Hq, Hkv, Nq, Nk, d, seed)
+        scale = 1.0 / math.sqrt(d)
+        O, L = orc.forward(x["q"], x["k"], x["v"], scale, causal)
+        Ob, Lb = brute_force_decimal(x, scale, causal)
+        assert_close(O, Ob, what=f"O brute {B,Hq,Hkv,Nq,Nk,d,causal}")
+        assert_close(L, Lb, what=f"LSE brute {B,Hq,Hkv,Nq,Nk,d,causal}")
+
+
+def pin_large_logits(orc):
+    """Q x 8 (exact in bf16): logits of size ~8-30; must neither overflow nor drift."""
+    x = tiny_inputs(1, 2, 1, 7, 9, 64, seed=11, q_mult=8.0)
+    scale = 1.0 / 8.0
+    for causal in (False, True):
+        O, L = orc.forward(x["q"], x["k"], x["v"], scale, causal)
+        Ob, Lb = brute_force_decimal(x, scale, causal)
+        assert np.isfinite(O).all()
+        assert_close(O, Ob, what="O qx8")
+        assert_close(L, Lb, what="LSE qx8")
+
+
+def pin_probs_rows_sum_to_one(orc):
+    x = tiny_inputs(1, 2, 2, 9, 12, 32, seed=12)
+    for causal in (False, True):
+        _, _, P = orc.probs(x["q"], x["k"], x["v"], 0.3, causal)
+        assert (P >= 0).all()
+        assert np.abs(P.sum(axis=-1) - 1.0).max() < TOL
+        if causal:
+            i = np.arange(9)[:, None]
+            j = np.arange(12)[None, :]
+            hidden = j > i + 3          # Nk - Nq = 3
+            assert (P[..., hidden] == 0).all()
+
+
+def pin_one_key(orc):
+    """Nk = 1: every row attends to its single key: O = v_0, LSE = scale * q . k_0."""
+    x = tiny_inputs(2, 4, 2, 5, 1, 64, seed=13)
+    scale = 0.125
+    O, L = orc.forward(x["q"], x["k"], x["v"], scale, False)
+    q, k, v = (bits_f64(x[n]) for n in ("q", "k", "v"))
+    for b in range(2):
+        for h in range(4):
+            g = h // 2
+            assert_close(O[b, :, h, :], np.broadcast_to(v[b, 0, g, :], (5, 64)), what="O one key")
+            assert_close(L[b, h, :], scale * (q[b, :, h, :] @ k[b, 0, g, :]), what="LSE one key")
+
+
+def pin_constant_v(orc):
+    """Every key carries the same value row -> every output row equals it."""
+    x = tiny_inputs(1, 2, 2, 8, 10, 32, seed=14)
+    v = x["v"].copy()
+    v[:] = v[:, :1]
+    for causal in (False, True):
+        O, _ = orc.forward(x["q"], x["k"], v, 0.2, causal)
+        vf = bits_f64(v)
+        for h in range(2):
+            assert_close(O[0, :, h, :], np.broadcast_to(vf[0, 0, h, :], (8, 32)), what="O const V")
+
+
+def pin_zero_q(orc):
+    """Q = 0: all logits equal -> O = mean of the visible V rows, LSE = ln(#visible)."""
+    x = tiny_inputs(1, 2, 1, 6, 6, 32, seed=15)
+    q = np.zeros_like(x["q"])
+    vf = bits_f64(x["v"])
+    for causal in (False, True):
+        O, L = orc.forward(q, x["k"], x["v"], 0.5, causal)
+        for i in range(6):
+            n = i + 1 if causal else 6
+            for h in range(2):
+                assert_close(O[0, i, h, :], vf[0, :n, 0, :].mean(axis=0), what="O zero Q")
+                assert_close(L[0, h, i], math.log(n), what="LSE zero Q")
+
+
+def pin_causal_row0(orc):
+    """Causal, Nq = Nk: row 0 sees only key 0 -> O_0 = v_0, LSE_0 = s_00."""
+    x = tiny_inputs(1, 2, 2, 7, 7, 64, seed=16)
+    scale = 0.125
+    O, L = orc.forward(x["q"], x["k"], x["v"], scale, True)
+    q, k, v = (bits_f64(x[n]) for n in ("q", "k", "v"))
+    for h in range(2):
+        assert_close(O[0, 0, h, :], v[0, 0, h, :], what="O causal row 0")
+        assert_close(L[0, h, 0], scale * float(q[0, 0, h, :] @ k[0, 0, h, :]), what="LSE causal row 0")
+
+
+def pin_gqa_equals_repeated_mha(orc):
+    """GQA result == MHA with K/V repeated n_rep times per head (repeat_interleave)."""
+    x = tiny_inputs(2, 8, 2, 6, 9, 32, seed=17)
+    kr = np.repeat(x["k"], 4, axis=2)
+    vr = np.repeat(x["v"], 4, axis=2)
+    for causal in (False, True):
+        O1, L1 = orc.forward(x["q"], x["k"], x["v"], 0.3, causal)
+        O2, L2 = orc.forward(x["q"], kr, vr, 0.3, causal)
+        assert_close(O1, O2, what="GQA vs MHA O")
+        assert_close(L1, L2, what="GQA vs MHA LSE")
+
+
+def pin_key_permutation(orc):
+    """Without a mask the result does not depend on the order of the (key, value) pairs."""
+    x = tiny_inputs(1, 2, 2, 5, 11, 32, seed=18)
+    perm = np.random.default_rng(0).permutation(11)
+    O1, L1 = orc.forward(x["q"], x["k"], x["v"], 0.3, False)
+    O2, L2 = orc.forward(x["q"], x["k"][:, perm], x["v"][:, perm], 0.3, False)
+    assert_close(O1, O2, what="perm O")
+    assert_close(L1, L2, what="perm LSE")
+
+
+def pin_causal_prefix(orc):
+    """Causal row i equals unmasked attention of query i over keys 0..i."""
+    x = tiny_inputs(1, 1, 1, 9, 9, 32, seed=19)
+    O, L = orc.forward(x["q"], x["k"], x["v"], 0.3, True)
+    for i in (0, 3, 8):
+        Oi, Li = orc.forward(x["q"][:, i:i + 1], x["k"][:, :i + 1], x["v"][:, :i + 1], 0.3, False)
+        assert_close(O[0, i, 0], Oi[0, 0, 0], what="prefix O")
+        assert_close(L[0, 0, i], Li[0, 0, 0], what="prefix LSE")
+
+
+def pin_online_recurrence(orc):
+    """The block-wise online-softmax recurrence reaches the oracle's result at every block size."""
+    for (B, Hq, Hkv, Nq, Nk, d, causal) in [(1, 2, 1, 37, 37, 32, True), (2, 2, 2, 20, 45, 64, False),
+                                             (1, 2, 2, 30, 17, 16, True)]:
+        x = tiny_inputs(B, Hq, Hkv, Nq, Nk, d, seed=20 + Nq)
+        O, L = orc.forward(x["q"], x["k"], x["v"], 0.2, causal)
+        for block in (1, 5, 16, 64, 128):
+            Ob, Lb = online_softmax_blocks(x, 0.2, causal, block)
+            assert_close(O, Ob, what=f"online O block {block}")
+            assert_close(L, Lb, what=f"online LSE block {block}")
+
+
+def pin_rows_match_full(orc):
+    """The selected-rows entry point gives the full forward's rows."""
+    x = tiny_inputs(2, 4, 2, 13, 10, 32, seed=21)
+    rows = [(0, 0, 0), (1, 3, 12), (0, 2, 5), (1, 1, 2)]
+    for causal in (False, True):
+        O, L = orc.forward(x["q"], x["k"], x["v"], 0.3, causal)
+        Or, Lr = orc.rows(x["q"], x["k"], x["v"], rows, 0.3, causal)
+        for r, (b, h, i) in enumerate(rows):
+            assert np.array_equal(Or[r], O[b, i, h])
+            assert Lr[r] == L[b, h, i] or (np.isinf(Lr[r]) and np.isinf(L[b, h, i]))
+
+
+ALL_PINS = [
+    pin_brute_force, pin_large_logits, pin_probs_rows_sum_to_one, pin_one_key, pin_constant_v,
+    pin_zero_q, pin_causal_row0, pin_gqa_equals_repeated_mha, pin_key_permutation,
+    pin_causal_prefix, pin_online_recurrence, pin_rows_match_full,
+]
