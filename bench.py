@@ -1,0 +1,347 @@
+#!/usr/bin/env python3
+"""Throughput benchmark of the exact attention forward (fa_fwd) on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+One step = one fa_fwd call over the whole workload (every row of the hot path: tile
+schedule, TMA loads, QK^T, online softmax, PV, epilogue).  Default workload: the
+d=128, N=4096 point of the sequence-length sweep (B=8, H=32), inputs larger than L2.
+For N > 1 (launched under torchrun) every rank runs its own replica on its own seeded
+batch (weak scaling: no data-path collective exists in the forward pass); the time is
+the max over ranks of CUDA-event time.
+
+Prints ONE JSON line (rank 0).  TFLOP/s counts 4*B*Hq*Nq*Nk*d per call (half for causal).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import re
+import statistics
+import subprocess
+import sys
+import threading
+import time
+from pathlib import Path
+
+import numpy as np
+
+ROOT = Path(__file__).resolve().parent
+sys.path.insert(0, str(ROOT))
+
+import synth  # noqa: E402
+
+METRIC = "attention fwd TFLOP/s and % of B200 bf16 tensor peak vs seq len (1 GPU)"
+FALLBACK_PEAKS = {"bf16_tflops": 1590.0, "hbm_gbs": 6650.0, "source": "fallback"}
+KERNEL_NAME = "fa_fwd_kernel"
+
+
+def peaks():
+    p = ROOT / "MEASURED_PEAKS.json"
+    if p.exists():
+        d = json.loads(p.read_text())
+        return {"bf16_tflops": float(d["bf16_tflops"]), "bf16_tflops_sustained": float(d.get("bf16_tflops_sustained", 0)),
+                "hbm_gbs": float(d["hbm_gbs"]), "source": "measured"}
+    return dict(FALLBACK_PEAKS)
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for f in sorted((ROOT / "exact_attention_146_b200" / "csrc").glob("*")):
+        h.update(f.read_bytes())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(workload: str):
+    """DRAM bytes per launch of the kernel from the committed ncu summary, if that
+    summary was taken on the current kernel source (else None)."""
+    f = ROOT / "profiles" / f"{KERNEL_NAME}_{workload}.md"
+    if not f.exists():
+        return None
+    text = f.read_text()
+    m_hash = re.search(r"kernel_source_hash:\s*([0-9a-f]+)", text)
+    m_bytes = re.search(r"dram_bytes_per_launch:\s*([0-9.eE+]+)", text)
+    if not m_hash or not m_bytes or m_hash.group(1) != kernel_source_hash():
+        return None
+    return float(m_bytes.group(1))
+
+
+class ClockSampler:
+    """nvidia-smi clocks / throttle reasons sampled while the timed region runs."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int, period_ms: int = 50):
+        self.rows = []
+        self.proc = None
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={gpu_index}", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
+                 f"-lms={period_ms}"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.th = threading.Thread(target=self._read, daemon=True)
+            self.th.start()
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) >= 9:
+                self.rows.append((time.time(), parts))
+
+    def window(self, t0, t1):
+        return [r for (t, r) in self.rows if t0 <= t <= t1]
+
+    def stop(self):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    @staticmethod
+    def summarize(rows):
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower().startswith("active")})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+def dist_setup(n_gpus):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != n_gpus and world > 1:
+        raise SystemExit(f"--gpus {n_gpus} but WORLD_SIZE={world}")
+    return world, rank, local
+
+
+def oracle_sample_tflops(w: synth.Workload, target_s: float, heads_cap: int | None = None):
+    """Time the CPU oracle on a bounded sample of the workload: whole (b, hq) heads of
+    batch element 0, as many as fit in ~target_s.  Returns (TFLOP/s, sample text, cores)."""
+    import oracle
+    orc = oracle.default()
+    cores = os.cpu_count() or 1
+    one = w.with_(B=1)
+    x = synth.make_inputs(one)
+    per_head = w.flops / (w.B * w.Hq)
+    done_flop, t_used, heads = 0.0, 0.0, 0
+    n_rep = w.Hq // w.Hkv
+    h = 0
+    while t_used < target_s and h < w.Hq and (heads_cap is None or heads < heads_cap):
+        g = h // n_rep
+        q = np.ascontiguousarray(x["q"][:, :, h:h + 1])
+        k = np.ascontiguousarray(x["k"][:, :, g:g + 1])
+        v = np.ascontiguousarray(x["v"][:, :, g:g + 1])
+        t0 = time.perf_counter()
+        orc.forward(q, k, v, w.scale, w.causal, threads=cores)
+        t_used += time.perf_counter() - t0
+        done_flop += per_head
+        heads += 1
+        h += 1
+    tf = done_flop / t_used / 1e12
+    return tf, f"{heads} of {w.B * w.Hq} (b, head) slices of {w.name} (batch element 0), {t_used:.1f} s", cores, t_used
+
+
+def run_reference(args, w, world, rank):
+    """The CPU fp64 oracle as the reference arm, timed on this host's cores."""
+    if rank != 0:
+        return 0
+    import oracle
+    orc = oracle.default()
+    cores = os.cpu_count() or 1
+    x = synth.make_inputs(w.with_(B=1))
+    per_head = w.flops / (w.B * w.Hq)
+    times = []
+    for step in range(args.warmup + args.steps):
+        h = step % w.Hq
+        g = h // (w.Hq // w.Hkv)
+        q = np.ascontiguousarray(x["q"][:, :, h:h + 1])
+        k = np.ascontiguousarray(x["k"][:, :, g:g + 1])
+        v = np.ascontiguousarray(x["v"][:, :, g:g + 1])
+        t0 = time.perf_counter()
+        orc.forward(q, k, v, w.scale, w.causal, threads=cores)
+        dt = time.perf_counter() - t0
+        if step >= args.warmup:
+            times.append(dt)
+    ms = 1e3 * sum(times) / len(times)
+    value = per_head / (ms * 1e-3) / 1e12
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "Nq": w.Nq, "Nk": w.Nk, "d": w.d,
+                   "causal": w.causal, "step": "one (b, head) slice of the workload per step"},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+                         "sample": f"one (b, head) slice of {w.name} per step"},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_ours(args, w, world, rank, local):
+    import torch
+    import exact_attention_146_b200 as fa
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    pg = None
+    if world > 1:
+        import torch.distributed as dist
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
+        pg = dist
+    stream = torch.cuda.current_stream()
+
+    # per-rank replica of the workload on its own seeded data (weak scaling)
+    wr = w.with_(seed=w.seed + rank)
+    x = synth.make_inputs(wr)
+    host = {n: torch.from_numpy(x[n].view(np.int16)).view(torch.bfloat16).pin_memory() for n in ("q", "k", "v")}
+    q, k, v = (host[n].to(dev, non_blocking=True) for n in ("q", "k", "v"))
+    out = torch.empty_like(q)
+    lse = torch.empty((w.B, w.Hq, w.Nq), dtype=torch.float32, device=dev)
+    torch.cuda.synchronize()
+
+    def step():
+        fa.fa_fwd(q, k, v, causal=w.causal, scale=w.scale, out=out, lse=lse)
+
+    for _ in range(args.warmup):
+        step()
+    st, word = fa.device_status()
+    if st != fa.FA_OK:
+        raise SystemExit(f"device status after warm-up: {st} ({word:#x})")
+
+    sampler = ClockSampler(local) if not args.no_clocks else None
+    if sampler:
+        time.sleep(0.3)
+    if pg:
+        pg.barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t_wall0 = time.time()
+    e0.record(stream)
+    for _ in range(args.steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    t_wall1 = time.time()
+    if pg:
+        pg.barrier()
+    ms = e0.elapsed_time(e1) / args.steps
+    st, word = fa.device_status()
+    if st != fa.FA_OK:
+        raise SystemExit(f"device status after timed steps: {st} ({word:#x})")
+    clocks = None
+    if sampler:
+        time.sleep(0.15)
+        sampler.stop()
+        clocks = ClockSampler.summarize(sampler.window(t_wall0, t_wall1 + 0.1))
+    ms_max = ms
+    if pg:
+        t = torch.tensor([ms], device=dev, dtype=torch.float64)
+        pg.all_reduce(t, op=pg.ReduceOp.MAX)
+        ms_max = float(t.item())
+
+    value = world * w.flops / (ms_max * 1e-3) / 1e12
+    pk = peaks()
+    achieved = w.flops / (ms * 1e-3) / 1e12           # per launch on this rank
+    roofline = {"bound": "tensor", "achieved": achieved, "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
+                "frac": achieved / pk["bf16_tflops"], "traffic": profiled_traffic(w.name),
+                "peak_source": f"{pk['source']} bf16 dense (burst)",
+                "algorithmic_bytes": w.io_bytes,
+                "hbm_gbs": w.io_bytes / (ms * 1e-3) / 1e9}
+
+    # end to end through the public API: pinned host inputs in, O and LSE back to host
+    e2e = None
+    if not args.no_e2e:
+        out_h = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+        lse_h = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
+        n_e2e = max(1, min(args.steps, args.e2e_steps))
+
+        def e2e_step():
+            q.copy_(host["q"], non_blocking=True)
+            k.copy_(host["k"], non_blocking=True)
+            v.copy_(host["v"], non_blocking=True)
+            fa.fa_fwd(q, k, v, causal=w.causal, scale=w.scale, out=out, lse=lse)
+            out_h.copy_(out, non_blocking=True)
+            lse_h.copy_(lse, non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize()
+        if pg:
+            pg.barrier()
+        f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        f0.record(stream)
+        for _ in range(n_e2e):
+            e2e_step()
+        f1.record(stream)
+        torch.cuda.synchronize()
+        ms_e2e = f0.elapsed_time(f1) / n_e2e
+        if pg:
+            t = torch.tensor([ms_e2e], device=dev, dtype=torch.float64)
+            pg.all_reduce(t, op=pg.ReduceOp.MAX)
+            ms_e2e = float(t.item())
+        h2d = sum(host[n].numel() * 2 for n in ("q", "k", "v"))
+        d2h = out.numel() * 2 + lse.numel() * 4
+        e2e = {"value": world * w.flops / (ms_e2e * 1e-3) / 1e12, "unit": "TFLOP/s", "ms_per_step": ms_e2e,
+               "steps": n_e2e, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        tf, sample, cores, secs = oracle_sample_tflops(w, args.cpu_seconds)
+        cpu = {"value": tf, "unit": "TFLOP/s", "cores": cores, "kind": "oracle", "sample": sample}
+
+    if pg:
+        pg.barrier()
+        pg.destroy_process_group()
+    if rank != 0:
+        return 0
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_max, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "Nq": w.Nq, "Nk": w.Nk, "d": w.d,
+                   "causal": w.causal, "global_batch": w.B * world, "seq_len": w.Nq,
+                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                   "l2": "inputs larger than L2 (no flush)" if w.io_bytes > 3 * 126e6 else "inputs fit L2: warm-L2 number",
+                   "pct_of_peak": 100.0 * achieved / pk["bf16_tflops"]},
+        "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": args.steps, "clocks": clocks,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--workload", default=synth.HEADLINE, choices=sorted(synth.WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--e2e-steps", type=int, default=5)
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-clocks", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    w = synth.WORKLOADS[args.workload]
+    world, rank, local = dist_setup(args.gpus)
+    if args.impl == "reference":
+        return run_reference(args, w, world, rank)
+    return run_ours(args, w, world, rank, local)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

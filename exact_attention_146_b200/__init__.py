@@ -1,0 +1,126 @@
+"""B200-native exact attention forward: Python binding of libfa.so.
+
+This module only marshals arguments (torch tensors -> device pointers, sizes and the
+current CUDA stream) into the C ABI declared in ``include/fa.h``; every step of the
+computation runs in the CUDA kernels of ``csrc/``.  There is no fallback: if the
+library is missing or the device is not sm_100 the calls raise.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+from pathlib import Path
+
+__all__ = ["fa_fwd", "device_status", "tile_config", "status_string", "FaError", "lib",
+           "SUPPORTED_HEAD_DIMS", "LIB_PATH"]
+
+LIB_PATH = Path(__file__).resolve().parent / "libfa.so"
+SUPPORTED_HEAD_DIMS = (32, 64, 80, 96, 128, 192, 256)
+
+FA_OK = 0
+FA_ERR_INVALID_ARG = 1
+FA_ERR_UNSUPPORTED_HEAD_DIM = 2
+FA_ERR_MISALIGNED = 3
+FA_ERR_UNSUPPORTED_DEVICE = 4
+FA_ERR_CUDA = 5
+FA_ERR_DEVICE_TIMEOUT = 6
+FA_ERR_NOT_DEVICE_MEMORY = 7
+FA_ERR_OVERLAP = 8
+
+EXPORTED = ("fa_fwd", "fa_status_string", "fa_device_status", "fa_tile_config", "fa_version")
+
+
+class FaError(RuntimeError):
+    def __init__(self, code: int, what: str = "fa_fwd"):
+        self.code = code
+        super().__init__(f"{what}: status {code}: {status_string(code)}")
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded libfa.so (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not LIB_PATH.exists():
+            raise RuntimeError(f"{LIB_PATH} is missing: build it with `python -m exact_attention_146_b200.build`")
+        L = ctypes.CDLL(str(LIB_PATH))
+        vp, ci, cf = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
+        L.fa_fwd.argtypes = [vp, vp, vp, vp, vp, ci, ci, ci, ci, ci, ci, cf, ci, vp]
+        L.fa_fwd.restype = ci
+        L.fa_status_string.argtypes = [ci]
+        L.fa_status_string.restype = ctypes.c_char_p
+        L.fa_device_status.argtypes = [vp, ctypes.POINTER(ci)]
+        L.fa_device_status.restype = ci
+        L.fa_tile_config.argtypes = [ci] + [ctypes.POINTER(ci)] * 4
+        L.fa_tile_config.restype = ci
+        L.fa_version.argtypes = []
+        L.fa_version.restype = ci
+        _lib = L
+    return _lib
+
+
+def status_string(code: int) -> str:
+    return lib().fa_status_string(int(code)).decode()
+
+
+def tile_config(d: int) -> dict:
+    """Tiling fa_fwd uses for head dim d: block_q, block_k, q_tiles_per_unit, kv_slots."""
+    vals = [ctypes.c_int(0) for _ in range(4)]
+    rc = lib().fa_tile_config(int(d), *[ctypes.byref(x) for x in vals])
+    if rc != FA_OK:
+        raise FaError(rc, "fa_tile_config")
+    return dict(zip(("block_q", "block_k", "q_tiles_per_unit", "kv_slots"), (x.value for x in vals)))
+
+
+def _stream_handle(stream) -> int:
+    import torch
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return int(stream.cuda_stream) if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def fa_fwd_raw(q_ptr, k_ptr, v_ptr, out_ptr, lse_ptr, B, Hq, Hkv, Nq, Nk, d, scale, causal, stream_ptr) -> int:
+    """Direct C-ABI call with integer pointers; returns the status code."""
+    return lib().fa_fwd(q_ptr, k_ptr, v_ptr, out_ptr, lse_ptr, int(B), int(Hq), int(Hkv), int(Nq), int(Nk),
+                        int(d), float(scale), int(causal), stream_ptr)
+
+
+def fa_fwd(q, k, v, *, causal: bool = False, scale: float | None = None, out=None, lse=None,
+           return_lse: bool = True, stream=None):
+    """Exact attention forward on [B, N, H, d] bf16 CUDA tensors.
+
+    q: [B, Nq, Hq, d]; k, v: [B, Nk, Hkv, d] with Hq % Hkv == 0 (GQA: query head h
+    uses KV head h // (Hq // Hkv)).  Returns (out [B, Nq, Hq, d] bf16, lse [B, Hq, Nq]
+    fp32 natural-log log-sum-exp, or None if return_lse is False).  scale defaults to
+    1/sqrt(d).  Runs asynchronously on `stream` (default: torch's current stream)."""
+    import torch
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        if t.dtype != torch.bfloat16 or not t.is_cuda or not t.is_contiguous() or t.dim() != 4:
+            raise ValueError(f"{name} must be a contiguous 4-D bf16 CUDA tensor, got {t.dtype} {tuple(t.shape)}")
+    B, Nq, Hq, d = q.shape
+    Bk, Nk, Hkv, dk = k.shape
+    if v.shape != k.shape or Bk != B or dk != d:
+        raise ValueError(f"shape mismatch q{tuple(q.shape)} k{tuple(k.shape)} v{tuple(v.shape)}")
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if out is None:
+        out = torch.empty_like(q)
+    if return_lse and lse is None:
+        lse = torch.empty((B, Hq, Nq), dtype=torch.float32, device=q.device)
+    if not return_lse:
+        lse = None
+    rc = fa_fwd_raw(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                    lse.data_ptr() if lse is not None else None, B, Hq, Hkv, Nq, Nk, d, scale,
+                    1 if causal else 0, _stream_handle(stream))
+    if rc != FA_OK:
+        raise FaError(rc)
+    return out, lse
+
+
+def device_status(stream=None) -> tuple[int, int]:
+    """Synchronise `stream`, return (status, raw word) of the device status word, and clear it."""
+    detail = ctypes.c_int(0)
+    rc = lib().fa_device_status(_stream_handle(stream), ctypes.byref(detail))
+    return rc, detail.value

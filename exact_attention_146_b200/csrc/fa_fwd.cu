@@ -1,0 +1,321 @@
+// fa_fwd.cu -- the C ABI of libfa.so (declared in include/fa.h): argument validation,
+// device and pointer checks, TMA tensor-map encoding, per-head-dim dispatch, launch,
+// and the device status word.  One tuned kernel instantiation per head dimension, the
+// per-hdim specialisation the datacanvas.csdn.net head-dim article describes (section
+// "technical roots of the head-dim limit"), as C++ template instances.
+#include <algorithm>
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "fa.h"
+#include "fa_kernel.cuh"
+
+namespace {
+
+using namespace fa;
+
+// Tiling per head dim: TileCfg<d, key rows per tile, query tiles per unit, K/V slots>.
+using Cfg32 = TileCfg<32, 128, 2, 8>;
+using Cfg64 = TileCfg<64, 128, 2, 8>;
+using Cfg80 = TileCfg<80, 128, 2, 4>;
+using Cfg96 = TileCfg<96, 128, 2, 4>;
+using Cfg128 = TileCfg<128, 128, 2, 4>;
+using Cfg192 = TileCfg<192, 64, 2, 4>;
+using Cfg256 = TileCfg<256, 64, 1, 4>;
+
+__device__ int g_fa_status;   // per-device kernel status word (0 = OK)
+
+constexpr int kMaxDevices = 64;
+
+struct DeviceState {
+    bool probed = false;
+    bool supported = false;
+    int num_sms = 0;
+    int *status_ptr = nullptr;
+    bool smem_attr_set[8] = {};
+};
+DeviceState g_devices[kMaxDevices];
+std::mutex g_mutex;
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                   const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                   const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+using AddressRangeFn = CUresult (*)(CUdeviceptr *, size_t *, CUdeviceptr);
+
+void *driver_fn(const char *name) {
+    void *fn = nullptr;
+    cudaDriverEntryPointQueryResult q{};
+    if (cudaGetDriverEntryPoint(name, &fn, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+        return nullptr;
+    return fn;
+}
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = reinterpret_cast<EncodeTiledFn>(driver_fn("cuTensorMapEncodeTiled"));
+    return fn;
+}
+
+AddressRangeFn address_range_fn() {
+    static AddressRangeFn fn = reinterpret_cast<AddressRangeFn>(driver_fn("cuMemGetAddressRange"));
+    return fn;
+}
+
+// Current device, probed once: sm_100 (compute capability 10.0) or not.
+int current_device(DeviceState **out, int *dev_out) {
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+        cudaGetLastError();
+        return FA_ERR_UNSUPPORTED_DEVICE;
+    }
+    std::lock_guard<std::mutex> lock(g_mutex);
+    DeviceState &st = g_devices[dev];
+    if (!st.probed) {
+        int major = 0, minor = 0, sms = 0;
+        if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+            cudaGetLastError();
+            return FA_ERR_UNSUPPORTED_DEVICE;
+        }
+        st.supported = (major == 10 && minor == 0);
+        st.num_sms = sms;
+        if (st.supported) {
+            void *p = nullptr;
+            if (cudaGetSymbolAddress(&p, g_fa_status) != cudaSuccess) {
+                cudaGetLastError();
+                return FA_ERR_CUDA;
+            }
+            st.status_ptr = static_cast<int *>(p);
+        }
+        st.probed = true;
+    }
+    if (!st.supported) return FA_ERR_UNSUPPORTED_DEVICE;
+    *out = &st;
+    *dev_out = dev;
+    return FA_OK;
+}
+
+// `bytes` starting at `p` must be device (or managed) memory of device `dev`, inside one
+// allocation.
+int check_device_range(const void *p, size_t bytes, int dev) {
+    cudaPointerAttributes a{};
+    if (cudaPointerGetAttributes(&a, p) != cudaSuccess) {
+        cudaGetLastError();
+        return FA_ERR_NOT_DEVICE_MEMORY;
+    }
+    if (!(a.type == cudaMemoryTypeDevice || a.type == cudaMemoryTypeManaged) || a.device != dev)
+        return FA_ERR_NOT_DEVICE_MEMORY;
+    if (AddressRangeFn fn = address_range_fn()) {
+        CUdeviceptr base = 0;
+        size_t size = 0;
+        if (fn(&base, &size, reinterpret_cast<CUdeviceptr>(p)) != CUDA_SUCCESS)
+            return FA_ERR_NOT_DEVICE_MEMORY;
+        const uintptr_t lo = reinterpret_cast<uintptr_t>(p);
+        if (lo + bytes > uintptr_t(base) + size) return FA_ERR_NOT_DEVICE_MEMORY;
+    }
+    return FA_OK;
+}
+
+bool overlaps(const void *a, size_t na, const void *b, size_t nb) {
+    if (a == nullptr || b == nullptr || na == 0 || nb == 0) return false;
+    const uintptr_t a0 = reinterpret_cast<uintptr_t>(a), b0 = reinterpret_cast<uintptr_t>(b);
+    return a0 < b0 + nb && b0 < a0 + na;
+}
+
+// 4-D view (d, H, N, B) of a [B, N, H, d] bf16 tensor, box (CW, 1, rows, 1).
+int encode_bnhd(CUtensorMap *m, const void *base, int d, int H, int N, int B, int cw, int rows) {
+    EncodeTiledFn fn = encode_fn();
+    if (fn == nullptr) return FA_ERR_CUDA;
+    const cuuint64_t dims[4] = {cuuint64_t(d), cuuint64_t(H), cuuint64_t(N), cuuint64_t(B)};
+    const cuuint64_t strides[3] = {cuuint64_t(d) * 2, cuuint64_t(H) * d * 2, cuuint64_t(N) * H * d * 2};
+    const cuuint32_t box[4] = {cuuint32_t(cw), 1, cuuint32_t(rows), 1};
+    const cuuint32_t estr[4] = {1, 1, 1, 1};
+    const CUtensorMapSwizzle sw = (cw * 2 == 128) ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
+    const CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(base), dims, strides,
+                          box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? FA_OK : FA_ERR_CUDA;
+}
+
+struct Problem {
+    const void *q, *k, *v;
+    void *out;
+    float *lse;
+    int B, Hq, Hkv, Nq, Nk, d;
+    float scale;
+    int causal;
+};
+
+template <class C>
+int launch(const Problem &pr, DeviceState &dev, int cfg_slot, cudaStream_t stream) {
+    auto kern = fa_fwd_kernel<C>;
+    if (!dev.smem_attr_set[cfg_slot]) {
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) !=
+            cudaSuccess) {
+            cudaGetLastError();
+            return FA_ERR_CUDA;
+        }
+        dev.smem_attr_set[cfg_slot] = true;
+    }
+    CUtensorMap mq, mk, mv;
+    int rc;
+    if ((rc = encode_bnhd(&mq, pr.q, C::D, pr.Hq, pr.Nq, pr.B, C::CW, kBlockQ)) != FA_OK) return rc;
+    if ((rc = encode_bnhd(&mk, pr.k, C::D, pr.Hkv, pr.Nk, pr.B, C::CW, C::BC)) != FA_OK) return rc;
+    if ((rc = encode_bnhd(&mv, pr.v, C::D, pr.Hkv, pr.Nk, pr.B, C::CW, C::BC)) != FA_OK) return rc;
+
+    FwdParams p{};
+    p.out = static_cast<__nv_bfloat16 *>(pr.out);
+    p.lse = pr.lse;
+    p.status = dev.status_ptr;
+    p.B = pr.B;
+    p.Hq = pr.Hq;
+    p.Hkv = pr.Hkv;
+    p.Nq = pr.Nq;
+    p.Nk = pr.Nk;
+    p.n_rep = pr.Hq / pr.Hkv;
+    p.causal = pr.causal;
+    p.nqb = (pr.Nq + C::NQT * kBlockQ - 1) / (C::NQT * kBlockQ);
+    const long long units = (long long)pr.B * pr.Hq * p.nqb;
+    if (units > 0x7fffffffLL) return FA_ERR_INVALID_ARG;
+    p.num_units = int(units);
+    p.scale_log2 = pr.scale * 1.4426950408889634f;
+
+    const int grid = int(units < dev.num_sms ? units : dev.num_sms);
+    fa_fwd_kernel<C><<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(mq, mk, mv, p);
+    if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
+    return FA_OK;
+}
+
+int tile_config(int d, int *bq, int *bk, int *nqt, int *ns) {
+    int BC, NQT, NS;
+    switch (d) {
+        case 32: BC = Cfg32::BC; NQT = Cfg32::NQT; NS = Cfg32::NS; break;
+        case 64: BC = Cfg64::BC; NQT = Cfg64::NQT; NS = Cfg64::NS; break;
+        case 80: BC = Cfg80::BC; NQT = Cfg80::NQT; NS = Cfg80::NS; break;
+        case 96: BC = Cfg96::BC; NQT = Cfg96::NQT; NS = Cfg96::NS; break;
+        case 128: BC = Cfg128::BC; NQT = Cfg128::NQT; NS = Cfg128::NS; break;
+        case 192: BC = Cfg192::BC; NQT = Cfg192::NQT; NS = Cfg192::NS; break;
+        case 256: BC = Cfg256::BC; NQT = Cfg256::NQT; NS = Cfg256::NS; break;
+        default: return FA_ERR_UNSUPPORTED_HEAD_DIM;
+    }
+    if (bq) *bq = kBlockQ;
+    if (bk) *bk = BC;
+    if (nqt) *nqt = NQT;
+    if (ns) *ns = NS;
+    return FA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int fa_version(void) { return 100; }
+
+const char *fa_status_string(int status) {
+    switch (status) {
+        case FA_OK: return "ok";
+        case FA_ERR_INVALID_ARG:
+            return "invalid argument (null pointer, negative size, Hq not a multiple of Hkv, scale not "
+                   "finite and positive, causal not 0/1, or sizes beyond 32-bit indexing)";
+        case FA_ERR_UNSUPPORTED_HEAD_DIM:
+            return "unsupported head dimension: fa_fwd supports head dimensions 32, 64, 80, 96, 128, 192, 256";
+        case FA_ERR_MISALIGNED: return "misaligned pointer: q/k/v/out need 16-byte, lse 4-byte alignment";
+        case FA_ERR_UNSUPPORTED_DEVICE: return "no CUDA device, or the current device is not sm_100 (B200)";
+        case FA_ERR_CUDA: return "a CUDA runtime or driver call failed";
+        case FA_ERR_DEVICE_TIMEOUT: return "a kernel pipeline wait timed out; outputs are undefined";
+        case FA_ERR_NOT_DEVICE_MEMORY:
+            return "a tensor is not device memory of the current device, or runs past its allocation";
+        case FA_ERR_OVERLAP: return "out or lse overlaps an input or each other";
+        default: return "unknown status";
+    }
+}
+
+int fa_tile_config(int d, int *block_q, int *block_k, int *q_tiles_per_unit, int *kv_slots) {
+    return tile_config(d, block_q, block_k, q_tiles_per_unit, kv_slots);
+}
+
+int fa_fwd(const void *q, const void *k, const void *v, void *out, float *lse, int B, int Hq, int Hkv,
+           int Nq, int Nk, int d, float scale, int causal, void *stream) {
+    // ---- host-only validation (no CUDA call before this block passes)
+    if (B < 0 || Hq <= 0 || Hkv <= 0 || Nq < 0 || Nk < 0) return FA_ERR_INVALID_ARG;
+    if (Hq % Hkv != 0) return FA_ERR_INVALID_ARG;
+    if (causal != 0 && causal != 1) return FA_ERR_INVALID_ARG;
+    if (!std::isfinite(scale) || !(scale > 0.f)) return FA_ERR_INVALID_ARG;
+    if (tile_config(d, nullptr, nullptr, nullptr, nullptr) != FA_OK) return FA_ERR_UNSUPPORTED_HEAD_DIM;
+    const size_t q_bytes = size_t(B) * size_t(Nq) * size_t(Hq) * size_t(d) * 2;
+    const size_t kv_bytes = size_t(B) * size_t(Nk) * size_t(Hkv) * size_t(d) * 2;
+    const size_t lse_bytes = size_t(B) * size_t(Hq) * size_t(Nq) * 4;
+    if (q_bytes == 0) return FA_OK;   // B == 0 or Nq == 0: no output rows
+    if (q == nullptr || out == nullptr) return FA_ERR_INVALID_ARG;
+    if (kv_bytes > 0 && (k == nullptr || v == nullptr)) return FA_ERR_INVALID_ARG;
+    auto mis = [](const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) != 0; };
+    if (mis(q, 16) || mis(out, 16) || (kv_bytes > 0 && (mis(k, 16) || mis(v, 16))) || (lse && mis(lse, 4)))
+        return FA_ERR_MISALIGNED;
+    if (overlaps(out, q_bytes, q, q_bytes) || overlaps(out, q_bytes, k, kv_bytes) ||
+        overlaps(out, q_bytes, v, kv_bytes) || overlaps(lse, lse_bytes, q, q_bytes) ||
+        overlaps(lse, lse_bytes, k, kv_bytes) || overlaps(lse, lse_bytes, v, kv_bytes) ||
+        overlaps(lse, lse_bytes, out, q_bytes))
+        return FA_ERR_OVERLAP;
+
+    // ---- device checks
+    DeviceState *dev = nullptr;
+    int dev_id = -1;
+    int rc = current_device(&dev, &dev_id);
+    if (rc != FA_OK) return rc;
+    if ((rc = check_device_range(q, q_bytes, dev_id)) != FA_OK) return rc;
+    if ((rc = check_device_range(out, q_bytes, dev_id)) != FA_OK) return rc;
+    if (kv_bytes > 0) {
+        if ((rc = check_device_range(k, kv_bytes, dev_id)) != FA_OK) return rc;
+        if ((rc = check_device_range(v, kv_bytes, dev_id)) != FA_OK) return rc;
+    }
+    if (lse && (rc = check_device_range(lse, lse_bytes, dev_id)) != FA_OK) return rc;
+
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (Nk == 0) {
+        const size_t n16 = q_bytes / 16;
+        const int grid = int(std::min<size_t>((n16 + 255) / 256, size_t(dev->num_sms) * 8));
+        fa_no_keys_kernel<<<grid > 0 ? grid : 1, 256, 0, st>>>(static_cast<uint4 *>(out), n16, lse,
+                                                             lse ? size_t(B) * Hq * Nq : 0);
+        return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+    }
+
+    const Problem pr{q, k, v, out, lse, B, Hq, Hkv, Nq, Nk, d, scale, causal};
+    switch (d) {
+        case 32: return launch<Cfg32>(pr, *dev, 0, st);
+        case 64: return launch<Cfg64>(pr, *dev, 1, st);
+        case 80: return launch<Cfg80>(pr, *dev, 2, st);
+        case 96: return launch<Cfg96>(pr, *dev, 3, st);
+        case 128: return launch<Cfg128>(pr, *dev, 4, st);
+        case 192: return launch<Cfg192>(pr, *dev, 5, st);
+        case 256: return launch<Cfg256>(pr, *dev, 6, st);
+        default: return FA_ERR_UNSUPPORTED_HEAD_DIM;
+    }
+}
+
+int fa_device_status(void *stream, int *detail) {
+    DeviceState *dev = nullptr;
+    int dev_id = -1;
+    int rc = current_device(&dev, &dev_id);
+    if (rc != FA_OK) return rc;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    int word = 0;
+    const int zero = 0;
+    if (cudaStreamSynchronize(st) != cudaSuccess ||
+        cudaMemcpyFromSymbolAsync(&word, g_fa_status, sizeof(int), 0, cudaMemcpyDeviceToHost, st) != cudaSuccess ||
+        cudaMemcpyToSymbolAsync(g_fa_status, &zero, sizeof(int), 0, cudaMemcpyHostToDevice, st) != cudaSuccess ||
+        cudaStreamSynchronize(st) != cudaSuccess) {
+        cudaGetLastError();
+        return FA_ERR_CUDA;
+    }
+    if (detail) *detail = word;
+    return (word & 0xFF) == 0 ? FA_OK : (word & 0xFF);
+}
+
+}  // extern "C"

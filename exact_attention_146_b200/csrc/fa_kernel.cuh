@@ -1,0 +1,563 @@
+// fa_kernel.cuh -- persistent sm_100a kernel for the exact attention forward.
+//
+// The method is the tiled FlashAttention forward described on the hwcomputing.csdn.net
+// article "FlashAttention in CANN ops-transformer": Q is cut into row blocks, K/V into
+// column blocks; for each Q block the K/V blocks stream through on-chip memory while a
+// running row max m and running sum l keep the softmax exact (section "online
+// softmax"), scale and mask are fused into the same pass (section "fusion"), the next
+// block is fetched while the current one is computed (section "double buffering"), and
+// the output is divided by l once at the end.
+//
+// How it maps onto a B200 SM (one CTA per SM, persistent over work units):
+//   * work unit = (batch b, query head hq, block of NQT x 128 query rows);
+//   * TMA warp (one thread): Q tiles once per unit, then K_j, V_j into an NS-slot
+//     shared-memory ring guarded by full/empty mbarriers;
+//   * MMA warp (one thread): S_t = Q_t K_j^T with tcgen05.mma into TMEM (fp32), and
+//     O_t += P_t V_j with P read straight from TMEM (it overwrites S_t as bf16);
+//     the two query tiles are interleaved so that one tile's softmax runs while the
+//     tensor core works on the other tile;
+//   * softmax warpgroup t (128 threads, thread r owns row r of tile t, which is TMEM
+//     lane r): loads its row of S_t, masks, takes the row max, p = 2^(s*scale*log2e - m)
+//     with one FFMA + ex2 per element, writes P back as bf16, keeps m and l in
+//     registers, rescales its O row in TMEM only when the max grew by more than
+//     2^8 (the final O / l is unchanged by the reference max used), and at the end
+//     writes O / l as bf16 and LSE = (m + log2 l) ln 2.
+// Every pipeline wait is bounded: after a time limit the kernel records
+// FA_ERR_DEVICE_TIMEOUT in a device status word, unwinds every role, waits for its own
+// in-flight copies and MMAs, frees TMEM and returns.
+#pragma once
+
+#include <cstdint>
+#include <cuda_bf16.h>
+
+#include "sm100.cuh"
+
+namespace fa {
+
+constexpr int kBlockQ = 128;                          // query rows per tile = TMEM lanes = MMA M
+constexpr uint64_t kWaitLimitNs = 1000000000ull;      // 1 s per wait
+constexpr float kRescaleLog2 = 8.0f;                  // lazy-rescale threshold (log2 units)
+constexpr int kStatusTimeout = 6;                     // = FA_ERR_DEVICE_TIMEOUT
+
+// Which wait gave up (bits 8..15 of the status word).
+enum WaitSite : int {
+    kSiteQEmpty = 1, kSiteKvEmpty = 2, kSiteKvFull = 3, kSiteQFull = 4, kSitePFull = 5,
+    kSiteOEmpty = 6, kSiteSFull = 7, kSiteODone = 8, kSiteDrain = 9, kSiteProducerDrain = 10
+};
+
+struct FwdParams {
+    __nv_bfloat16 *out;   // [B, Nq, Hq, d]
+    float *lse;           // [B, Hq, Nq] or nullptr
+    int *status;          // device status word
+    int B, Hq, Hkv, Nq, Nk;
+    int n_rep;            // Hq / Hkv
+    int causal;
+    int nqb;              // query blocks of NQT*128 rows per (b, hq)
+    int num_units;        // B * Hq * nqb
+    float scale_log2;     // scale * log2(e)
+};
+
+// Compile-time tiling for one head dimension.
+template <int D_, int BC_, int NQT_, int NS_>
+struct TileCfg {
+    static constexpr int D = D_;        // head dim
+    static constexpr int BC = BC_;      // key/value rows per tile
+    static constexpr int NQT = NQT_;    // query tiles per unit (1 or 2)
+    static constexpr int NS = NS_;      // K/V slots in the ring
+    static constexpr int CW = (D == 32) ? 32 : 64;       // elements per swizzled smem row
+    static constexpr int RB = CW * 2;                     // bytes per swizzled row (64 or 128)
+    static constexpr int NCH = (D + CW - 1) / CW;         // column chunks of a tile
+    static constexpr int Q_CHUNK = kBlockQ * RB;
+    static constexpr int KV_CHUNK = BC * RB;
+    static constexpr int Q_TILE = NCH * Q_CHUNK;
+    static constexpr int KV_TILE = NCH * KV_CHUNK;
+    static constexpr uint32_t LAYOUT = (RB == 128) ? 2u : 4u;   // UMMA 128B / 64B swizzle
+    static constexpr int SBO = 8 * RB;                          // 8-row swizzle atom
+    // TMEM columns: S_t at t*BC (P_t reuses its first BC/2 columns), O_t after all S.
+    static constexpr int OST = (D == 256) ? 256 : ((D + 63) / 64) * 64;
+    static constexpr int O_COL0 = NQT * BC;
+    static constexpr int TMEM_COLS = 512;
+    static constexpr int O_CHUNKS = (D + 31) / 32;
+    // shared memory (offsets from a 1024-byte aligned base)
+    static constexpr int SMEM_Q = 0;
+    static constexpr int SMEM_KV = NQT * Q_TILE;
+    static constexpr int SMEM_BAR = SMEM_KV + NS * KV_TILE;
+    static constexpr int NUM_BARS = 2 * NS + 6 * NQT + 1;
+    static constexpr int SMEM_MISC = SMEM_BAR + NUM_BARS * 8;
+    // Each CTA holds all 512 TMEM columns, so ask for enough shared memory that a
+    // second CTA can never be resident on the same SM (it would only wait in alloc).
+    static constexpr int SMEM_NEEDED = SMEM_MISC + 16 + 1024;
+    static constexpr int SMEM_BYTES = SMEM_NEEDED > 120 * 1024 ? SMEM_NEEDED : 120 * 1024;
+    // warps: 4 per query tile (softmax), then the TMA warp and the MMA warp
+    static constexpr int SOFTMAX_WARPS = 4 * NQT;
+    static constexpr int TMA_WARP = SOFTMAX_WARPS;
+    static constexpr int MMA_WARP = SOFTMAX_WARPS + 1;
+    static constexpr int THREADS = 32 * (SOFTMAX_WARPS + 2);
+    static constexpr uint32_t IDESC_S = sm100::idesc_bf16_f32(kBlockQ, BC, 0, 0);
+    static constexpr uint32_t IDESC_O = sm100::idesc_bf16_f32(kBlockQ, D, 0, 1);
+
+    static_assert(NQT == 1 || NQT == 2, "one or two query tiles per unit");
+    static_assert(D % 16 == 0 && D >= 32 && D <= 256, "MMA N and K granularity");
+    static_assert(BC % 64 == 0 && BC <= 256, "key tile: whole 32-column TMEM chunks of P");
+    static_assert(O_COL0 + NQT * OST <= TMEM_COLS, "TMEM budget");
+    static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+    // barrier indices
+    static constexpr int B_FULL = 0, B_EMPTY = NS, B_QFULL = 2 * NS, B_QEMPTY = 2 * NS + NQT,
+                         B_SFULL = 2 * NS + 2 * NQT, B_PFULL = 2 * NS + 3 * NQT,
+                         B_ODONE = 2 * NS + 4 * NQT, B_OEMPTY = 2 * NS + 5 * NQT,
+                         B_DRAIN = 2 * NS + 6 * NQT;
+};
+
+struct UnitInfo {
+    int b, hq, kvh, q0;
+    int nk[2];     // key tiles each query tile visits
+    int nk_max;
+};
+
+// Static schedule shared by all roles.  Causal: longest query blocks first, heads of
+// one KV group adjacent.  Non-causal: the query blocks of one head adjacent, so the
+// CTAs running at the same time share K/V through L2.
+template <class C>
+__device__ __forceinline__ UnitInfo decode_unit(int u, const FwdParams &p) {
+    UnitInfo w;
+    const int bh = p.B * p.Hq;
+    int qb, r;
+    if (p.causal) {
+        const int outer = u / bh;
+        qb = p.nqb - 1 - outer;
+        r = u - outer * bh;
+    } else {
+        r = u / p.nqb;
+        qb = u - r * p.nqb;
+    }
+    w.b = r / p.Hq;
+    w.hq = r - w.b * p.Hq;
+    w.kvh = w.hq / p.n_rep;
+    w.q0 = qb * (C::NQT * kBlockQ);
+    const int nkv = (p.Nk + C::BC - 1) / C::BC;
+    w.nk_max = 0;
+#pragma unroll
+    for (int t = 0; t < 2; ++t) {
+        int n = 0;
+        const int q_lo = w.q0 + t * kBlockQ;
+        if (t < C::NQT && q_lo < p.Nq) {
+            if (!p.causal) {
+                n = nkv;
+            } else {
+                const int q_hi = min(q_lo + kBlockQ - 1, p.Nq - 1);
+                const int lim = q_hi + (p.Nk - p.Nq);   // last visible key of the tile's last row
+                n = lim < 0 ? 0 : min(nkv, lim / C::BC + 1);
+            }
+        }
+        w.nk[t] = n;
+        w.nk_max = max(w.nk_max, n);
+    }
+    return w;
+}
+
+struct Ctl {
+    volatile int *abort_flag;
+    int *status;
+};
+
+// Poll `bar` until the phase of parity `parity` completes.  Gives up when another role
+// has raised the abort flag (unless `drain`: unwinding waits for the hardware's own
+// copies/MMAs regardless) or after `limit_ns`, recording the timeout in the status word.
+__device__ __noinline__ bool wait_slow(uint32_t bar, uint32_t parity, Ctl ctl, int site,
+                                       uint64_t limit_ns, bool drain = false) {
+    const uint64_t t0 = sm100::global_timer_ns();
+    while (true) {
+#pragma unroll 1
+        for (int i = 0; i < 64; ++i)
+            if (sm100::mbar_try_wait(bar, parity)) return true;
+        if (!drain && *ctl.abort_flag) return false;
+        if (sm100::global_timer_ns() - t0 > limit_ns) {
+            *ctl.abort_flag = 1;
+            atomicCAS(ctl.status, 0, kStatusTimeout | (site << 8) | (min(int(blockIdx.x), 0xFFFF) << 16));
+            return false;
+        }
+    }
+}
+
+__device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, const Ctl &ctl, int site,
+                                         uint64_t limit_ns = kWaitLimitNs) {
+    if (sm100::mbar_try_wait(bar, parity)) return true;
+    return wait_slow(bar, parity, ctl, site, limit_ns);
+}
+
+// Warp-uniform wait: every lane polls, the warp proceeds only if all lanes saw it.
+__device__ __forceinline__ bool warp_wait_bar(uint32_t bar, uint32_t parity, const Ctl &ctl, int site) {
+    const bool ok = wait_bar(bar, parity, ctl, site);
+    const bool all = __all_sync(0xffffffffu, ok);
+    if (!all) *ctl.abort_flag = 1;
+    return all;
+}
+
+// ------------------------------------------------------------------ TMA producer
+
+template <class C>
+__device__ void producer_role(const CUtensorMap *tm_q, const CUtensorMap *tm_k, const CUtensorMap *tm_v,
+                              const FwdParams &p, uint32_t sbase, const Ctl &ctl) {
+    auto bar = [&](int i) { return sbase + C::SMEM_BAR + 8u * uint32_t(i); };
+    sm100::prefetch_tensormap(tm_q);
+    sm100::prefetch_tensormap(tm_k);
+    sm100::prefetch_tensormap(tm_v);
+    uint32_t kv_cnt = 0;
+    uint32_t qcnt[2] = {0, 0};
+    bool ok = true;
+    for (int u = blockIdx.x; ok && u < p.num_units; u += gridDim.x) {
+        const UnitInfo w = decode_unit<C>(u, p);
+        if (w.nk_max == 0) continue;
+#pragma unroll
+        for (int t = 0; t < C::NQT; ++t) {
+            if (!ok || w.nk[t] == 0) continue;
+            if (!wait_bar(bar(C::B_QEMPTY + t), (qcnt[t] & 1u) ^ 1u, ctl, kSiteQEmpty)) { ok = false; break; }
+            ++qcnt[t];
+            const uint32_t fb = bar(C::B_QFULL + t);
+            sm100::mbar_arrive_expect_tx(fb, C::Q_TILE);
+            const uint32_t dst = sbase + C::SMEM_Q + t * C::Q_TILE;
+#pragma unroll
+            for (int c = 0; c < C::NCH; ++c)
+                sm100::tma_load_4d(dst + c * C::Q_CHUNK, tm_q, fb, c * C::CW, w.hq, w.q0 + t * kBlockQ, w.b);
+        }
+        for (int j = 0; ok && j < w.nk_max; ++j) {
+#pragma unroll
+            for (int which = 0; which < 2; ++which) {
+                const int s = int(kv_cnt % C::NS);
+                if (!wait_bar(bar(C::B_EMPTY + s), ((kv_cnt / C::NS) & 1u) ^ 1u, ctl, kSiteKvEmpty)) { ok = false; break; }
+                const uint32_t fb = bar(C::B_FULL + s);
+                sm100::mbar_arrive_expect_tx(fb, C::KV_TILE);
+                const uint32_t dst = sbase + C::SMEM_KV + s * C::KV_TILE;
+                const CUtensorMap *m = which ? tm_v : tm_k;
+#pragma unroll
+                for (int c = 0; c < C::NCH; ++c)
+                    sm100::tma_load_4d(dst + c * C::KV_CHUNK, m, fb, c * C::CW, w.kvh, j * C::BC, w.b);
+                ++kv_cnt;
+            }
+        }
+    }
+    if (!ok) {
+        // Unwinding after a timeout: let this thread's copies still in flight land
+        // before the CTA exits (the last load issued into each slot, and each Q tile).
+        const uint32_t first = kv_cnt > uint32_t(C::NS) ? kv_cnt - C::NS : 0u;
+        for (uint32_t n = first; n < kv_cnt; ++n)
+            wait_slow(bar(C::B_FULL + int(n % C::NS)), (n / C::NS) & 1u, ctl, kSiteProducerDrain,
+                      kWaitLimitNs / 10, true);
+#pragma unroll
+        for (int t = 0; t < C::NQT; ++t)
+            if (qcnt[t] > 0)
+                wait_slow(bar(C::B_QFULL + t), (qcnt[t] - 1) & 1u, ctl, kSiteProducerDrain, kWaitLimitNs / 10, true);
+    }
+}
+
+// ------------------------------------------------------------------ MMA issuer
+
+template <class C>
+__device__ __forceinline__ void issue_qk(uint32_t sbase, uint32_t tmem, int t, int slot) {
+    const uint32_t qa = sbase + C::SMEM_Q + t * C::Q_TILE;
+    const uint32_t kb = sbase + C::SMEM_KV + slot * C::KV_TILE;
+#pragma unroll
+    for (int kk = 0; kk < C::D / 16; ++kk) {
+        const int ch = (kk * 16) / C::CW;
+        const uint32_t off = uint32_t((kk * 16) % C::CW) * 2u;
+        const uint64_t a = sm100::smem_desc(qa + ch * C::Q_CHUNK + off, 16, C::SBO, C::LAYOUT);
+        const uint64_t b = sm100::smem_desc(kb + ch * C::KV_CHUNK + off, 16, C::SBO, C::LAYOUT);
+        sm100::mma_bf16_ss(tmem + uint32_t(t * C::BC), a, b, C::IDESC_S, kk > 0 ? 1u : 0u);
+    }
+}
+
+template <class C>
+__device__ __forceinline__ void issue_pv(uint32_t sbase, uint32_t tmem, int t, int slot, bool accumulate) {
+    const uint32_t vb = sbase + C::SMEM_KV + slot * C::KV_TILE;
+#pragma unroll
+    for (int kk = 0; kk < C::BC / 16; ++kk) {
+        // V tile is [BC rows x d] row-major: MN-major B operand; 16 key rows per MMA,
+        // 64-element column chunks C::KV_CHUNK bytes apart (leading byte offset).
+        const uint64_t b = sm100::smem_desc(vb + uint32_t(kk * 16 * C::RB), C::KV_CHUNK, C::SBO, C::LAYOUT);
+        const uint32_t a_tmem = tmem + uint32_t(t * C::BC + kk * 8);   // 16 bf16 = 8 columns
+        sm100::mma_bf16_ts(tmem + uint32_t(C::O_COL0 + t * C::OST), a_tmem, b, C::IDESC_O,
+                           (accumulate || kk > 0) ? 1u : 0u);
+    }
+}
+
+template <class C>
+__device__ void mma_role(const FwdParams &p, uint32_t sbase, uint32_t tmem, const Ctl &ctl) {
+    auto bar = [&](int i) { return sbase + C::SMEM_BAR + 8u * uint32_t(i); };
+    uint32_t kv_cnt = 0;
+    uint32_t qcnt[2] = {0, 0}, pcnt[2] = {0, 0};
+    uint32_t u_local = 0;
+    bool ok = true;
+    for (int u = blockIdx.x; ok && u < p.num_units; u += gridDim.x, ++u_local) {
+        const UnitInfo w = decode_unit<C>(u, p);
+        if (w.nk_max == 0) continue;
+        // prologue: S_t,0 for every tile that has work
+        const int s_k0 = int(kv_cnt % C::NS);
+        if (!wait_bar(bar(C::B_FULL + s_k0), (kv_cnt / C::NS) & 1u, ctl, kSiteKvFull)) { ok = false; break; }
+        ++kv_cnt;
+#pragma unroll
+        for (int t = 0; t < C::NQT; ++t) {
+            if (!ok || w.nk[t] == 0) continue;
+            if (!wait_bar(bar(C::B_QFULL + t), qcnt[t] & 1u, ctl, kSiteQFull)) { ok = false; break; }
+            ++qcnt[t];
+            sm100::tc_fence_after_sync();
+            issue_qk<C>(sbase, tmem, t, s_k0);
+            sm100::tc_commit(bar(C::B_SFULL + t));
+            if (w.nk[t] == 1) sm100::tc_commit(bar(C::B_QEMPTY + t));
+        }
+        if (!ok) break;
+        sm100::tc_commit(bar(C::B_EMPTY + s_k0));
+        for (int j = 0; ok && j < w.nk_max; ++j) {
+            const int s_v = int(kv_cnt % C::NS);
+            if (!wait_bar(bar(C::B_FULL + s_v), (kv_cnt / C::NS) & 1u, ctl, kSiteKvFull)) { ok = false; break; }
+            ++kv_cnt;
+            const bool has_next = j + 1 < w.nk_max;
+            int s_k = 0;
+            if (has_next) {
+                s_k = int(kv_cnt % C::NS);
+                if (!wait_bar(bar(C::B_FULL + s_k), (kv_cnt / C::NS) & 1u, ctl, kSiteKvFull)) { ok = false; break; }
+                ++kv_cnt;
+            }
+#pragma unroll
+            for (int t = 0; t < C::NQT; ++t) {
+                if (!ok) break;
+                if (j < w.nk[t]) {
+                    if (!wait_bar(bar(C::B_PFULL + t), pcnt[t] & 1u, ctl, kSitePFull)) { ok = false; break; }
+                    ++pcnt[t];
+                    if (j == 0 && u_local > 0 &&
+                        !wait_bar(bar(C::B_OEMPTY + t), (u_local - 1) & 1u, ctl, kSiteOEmpty)) { ok = false; break; }
+                    sm100::tc_fence_after_sync();
+                    issue_pv<C>(sbase, tmem, t, s_v, j > 0);
+                    sm100::tc_commit(bar(C::B_ODONE + t));
+                }
+                if (j + 1 < w.nk[t]) {
+                    issue_qk<C>(sbase, tmem, t, s_k);
+                    sm100::tc_commit(bar(C::B_SFULL + t));
+                    if (j + 2 == w.nk[t]) sm100::tc_commit(bar(C::B_QEMPTY + t));
+                }
+            }
+            if (!ok) break;
+            sm100::tc_commit(bar(C::B_EMPTY + s_v));
+            if (has_next) sm100::tc_commit(bar(C::B_EMPTY + s_k));
+        }
+    }
+    // Every MMA this thread issued is complete before the CTA may free TMEM.
+    sm100::tc_commit(bar(C::B_DRAIN));
+    wait_slow(bar(C::B_DRAIN), 0u, ctl, kSiteDrain, kWaitLimitNs, true);
+}
+
+// ------------------------------------------------------------------ softmax / epilogue
+
+template <class C>
+__device__ void softmax_role(const FwdParams &p, uint32_t sbase, uint32_t tmem, const Ctl &ctl,
+                             int warp, int lane) {
+    constexpr int BC = C::BC;
+    auto bar = [&](int i) { return sbase + C::SMEM_BAR + 8u * uint32_t(i); };
+    const int t = warp / 4;
+    const int quarter = warp % 4;                  // TMEM lanes 32*quarter .. +31
+    const int row_in_tile = quarter * 32 + lane;
+    const uint32_t lane_off = uint32_t(quarter * 32) << 16;
+    const uint32_t s_taddr = tmem + lane_off + uint32_t(t * BC);
+    const uint32_t o_taddr = tmem + lane_off + uint32_t(C::O_COL0 + t * C::OST);
+    const float c_log2 = p.scale_log2;
+    uint32_t scnt = 0, ocnt = 0;
+
+    for (int u = blockIdx.x; u < p.num_units; u += gridDim.x) {
+        const UnitInfo w = decode_unit<C>(u, p);
+        const int nk = w.nk[t];
+        const int q_lo = w.q0 + t * kBlockQ;
+        const int row = q_lo + row_in_tile;
+        const int diag = p.Nk - p.Nq;              // causal: key j visible to row i iff j <= i + diag
+        const int row_lim = p.causal ? row + diag : 0x7fffffff;
+        float m_ref = -INFINITY;                   // reference max, log2 units (scaled)
+        float l = 0.f;                             // running sum of 2^(s*c - m_ref)
+
+        for (int j = 0; j < nk; ++j) {
+            if (!warp_wait_bar(bar(C::B_SFULL + t), scnt & 1u, ctl, kSiteSFull)) goto unwind;
+            ++scnt;
+            sm100::tc_fence_after_sync();
+            uint32_t s[BC / 32][32];
+#pragma unroll
+            for (int c = 0; c < BC / 32; ++c) sm100::tmem_ld32_sync(s_taddr + uint32_t(32 * c), s[c]);
+
+            const int k_lo = j * BC;
+            const bool need_mask = (k_lo + BC > p.Nk) || (p.causal && k_lo + BC - 1 > q_lo + diag);
+            if (need_mask) {
+#pragma unroll
+                for (int c = 0; c < BC / 32; ++c)
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) {
+                        const int key = k_lo + 32 * c + i;
+                        if (key > row_lim || key >= p.Nk) s[c][i] = __float_as_uint(-INFINITY);
+                    }
+            }
+            float mx0 = -INFINITY, mx1 = -INFINITY, mx2 = -INFINITY, mx3 = -INFINITY;
+#pragma unroll
+            for (int c = 0; c < BC / 32; ++c)
+#pragma unroll
+                for (int i = 0; i < 32; i += 4) {
+                    mx0 = fmaxf(mx0, __uint_as_float(s[c][i]));
+                    mx1 = fmaxf(mx1, __uint_as_float(s[c][i + 1]));
+                    mx2 = fmaxf(mx2, __uint_as_float(s[c][i + 2]));
+                    mx3 = fmaxf(mx3, __uint_as_float(s[c][i + 3]));
+                }
+            const float mx_s = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * c_log2;
+            float alpha = 1.f;
+            bool need_rescale = false;
+            if (j == 0) {
+                m_ref = mx_s;
+            } else if (mx_s > m_ref + kRescaleLog2) {
+                alpha = sm100::ex2_approx(m_ref - mx_s);
+                m_ref = mx_s;
+                need_rescale = true;
+            }
+            const float neg_m = (m_ref == -INFINITY) ? 0.f : -m_ref;
+            float sum0 = 0.f, sum1 = 0.f, sum2 = 0.f, sum3 = 0.f;
+#pragma unroll
+            for (int c = 0; c < BC / 64; ++c) {
+                uint32_t pk[32];
+#pragma unroll
+                for (int i = 0; i < 32; i += 2) {
+                    const int e = 64 * c + 2 * i;          // element index of this pair
+                    const float p0 = sm100::ex2_approx(fmaf(__uint_as_float(s[e / 32][e % 32]), c_log2, neg_m));
+                    const float p1 = sm100::ex2_approx(fmaf(__uint_as_float(s[e / 32][e % 32 + 1]), c_log2, neg_m));
+                    const float p2 = sm100::ex2_approx(fmaf(__uint_as_float(s[e / 32][e % 32 + 2]), c_log2, neg_m));
+                    const float p3 = sm100::ex2_approx(fmaf(__uint_as_float(s[e / 32][e % 32 + 3]), c_log2, neg_m));
+                    sum0 += p0; sum1 += p1; sum2 += p2; sum3 += p3;
+                    pk[i] = sm100::pack_bf16x2(p0, p1);
+                    pk[i + 1] = sm100::pack_bf16x2(p2, p3);
+                }
+                sm100::tmem_st32(s_taddr + uint32_t(32 * c), pk);
+            }
+            l = l * alpha + ((sum0 + sum1) + (sum2 + sum3));
+
+            if (__any_sync(0xffffffffu, need_rescale)) {
+                // O_t holds the sum up to block j-1 at the old reference; wait for that
+                // MMA, then scale this warp's rows by alpha (1 where the max held).
+                if (!warp_wait_bar(bar(C::B_ODONE + t), (ocnt + uint32_t(j) - 1u) & 1u, ctl, kSiteODone)) goto unwind;
+                sm100::tc_fence_after_sync();
+#pragma unroll
+                for (int c = 0; c < C::O_CHUNKS; ++c) {
+                    uint32_t o[32];
+                    sm100::tmem_ld32_sync(o_taddr + uint32_t(32 * c), o);
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+                    sm100::tmem_st32(o_taddr + uint32_t(32 * c), o);
+                }
+            }
+            sm100::tmem_st_wait();
+            sm100::tc_fence_before_sync();
+            sm100::mbar_arrive(bar(C::B_PFULL + t));
+        }
+
+        // epilogue: O / l -> bf16 -> out, LSE -> lse
+        if (nk > 0) {
+            if (!warp_wait_bar(bar(C::B_ODONE + t), (ocnt + uint32_t(nk) - 1u) & 1u, ctl, kSiteODone)) goto unwind;
+            sm100::tc_fence_after_sync();
+        }
+        ocnt += uint32_t(nk);
+        {
+            const float inv_l = l > 0.f ? 1.f / l : 0.f;
+            const bool store = row < p.Nq;
+            __nv_bfloat16 *orow = p.out + ((size_t(w.b) * p.Nq + size_t(row)) * p.Hq + w.hq) * C::D;
+#pragma unroll
+            for (int c = 0; c < C::O_CHUNKS; ++c) {
+                uint32_t o[32];
+                if (nk > 0) {
+                    sm100::tmem_ld32_sync(o_taddr + uint32_t(32 * c), o);
+                } else {
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) o[i] = 0u;
+                }
+                uint32_t pk[16];
+#pragma unroll
+                for (int i = 0; i < 16; ++i)
+                    pk[i] = sm100::pack_bf16x2(__uint_as_float(o[2 * i]) * inv_l, __uint_as_float(o[2 * i + 1]) * inv_l);
+                if (store) {
+#pragma unroll
+                    for (int v4 = 0; v4 < 4; ++v4) {
+                        const int col = 32 * c + 8 * v4;
+                        if (col < C::D)
+                            *reinterpret_cast<uint4 *>(orow + col) =
+                                make_uint4(pk[4 * v4], pk[4 * v4 + 1], pk[4 * v4 + 2], pk[4 * v4 + 3]);
+                    }
+                }
+            }
+            sm100::tc_fence_before_sync();
+            sm100::mbar_arrive(bar(C::B_OEMPTY + t));
+            if (p.lse != nullptr && store)
+                p.lse[(size_t(w.b) * p.Hq + w.hq) * p.Nq + row] =
+                    l > 0.f ? (m_ref + log2f(l)) * 0.6931471805599453f : -INFINITY;
+        }
+    }
+unwind:
+    sm100::tmem_st_wait();
+}
+
+// ------------------------------------------------------------------ kernel
+
+template <class C>
+__global__ void __launch_bounds__(C::THREADS, 1)
+fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+              const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ FwdParams p) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const uint32_t sbase = sm100::smem_u32(smem);
+    const int warp = int(threadIdx.x) / 32;
+    const int lane = int(threadIdx.x) % 32;
+    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(smem + C::SMEM_MISC);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + C::SMEM_MISC + 4);
+    const Ctl ctl{abort_flag, p.status};
+
+    if (threadIdx.x == 0) {
+        auto bar = [&](int i) { return sbase + C::SMEM_BAR + 8u * uint32_t(i); };
+        for (int s = 0; s < C::NS; ++s) {
+            sm100::mbar_init(bar(C::B_FULL + s), 1);
+            sm100::mbar_init(bar(C::B_EMPTY + s), 1);
+        }
+        for (int t = 0; t < C::NQT; ++t) {
+            sm100::mbar_init(bar(C::B_QFULL + t), 1);
+            sm100::mbar_init(bar(C::B_QEMPTY + t), 1);
+            sm100::mbar_init(bar(C::B_SFULL + t), 1);
+            sm100::mbar_init(bar(C::B_PFULL + t), 128);
+            sm100::mbar_init(bar(C::B_ODONE + t), 1);
+            sm100::mbar_init(bar(C::B_OEMPTY + t), 128);
+        }
+        sm100::mbar_init(bar(C::B_DRAIN), 1);
+        *abort_flag = 0;
+        sm100::fence_mbar_init();
+    }
+    if (warp == 0) {
+        sm100::tmem_alloc(sm100::smem_u32(tmem_holder), C::TMEM_COLS);
+        sm100::tmem_relinquish();
+    }
+    sm100::tc_fence_before_sync();
+    __syncthreads();
+    sm100::tc_fence_after_sync();
+    const uint32_t tmem = *tmem_holder;
+
+    if (warp < C::SOFTMAX_WARPS) {
+        softmax_role<C>(p, sbase, tmem, ctl, warp, lane);
+    } else if (warp == C::TMA_WARP) {
+        if (lane == 0) producer_role<C>(&tm_q, &tm_k, &tm_v, p, sbase, ctl);
+    } else if (warp == C::MMA_WARP) {
+        if (lane == 0) mma_role<C>(p, sbase, tmem, ctl);
+    }
+    __syncwarp();
+
+    sm100::tc_fence_before_sync();
+    __syncthreads();
+    sm100::tc_fence_after_sync();
+    if (warp == 0) sm100::tmem_dealloc(tmem, C::TMEM_COLS);
+}
+
+// Nk == 0: no key at all, so every output row is 0 and every LSE is -inf.
+__global__ void fa_no_keys_kernel(uint4 *out, size_t n_vec16, float *lse, size_t n_lse) {
+    const size_t stride = size_t(gridDim.x) * blockDim.x;
+    for (size_t i = size_t(blockIdx.x) * blockDim.x + threadIdx.x; i < n_vec16; i += stride)
+        out[i] = make_uint4(0u, 0u, 0u, 0u);
+    if (lse != nullptr)
+        for (size_t i = size_t(blockIdx.x) * blockDim.x + threadIdx.x; i < n_lse; i += stride)
+            lse[i] = -INFINITY;
+}
+
+}  // namespace fa

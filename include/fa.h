@@ -1,0 +1,103 @@
+/*
+ * fa.h -- C ABI of the B200 (sm_100a) exact attention forward library (libfa.so).
+ *
+ * The operation (exact attention, forward):
+ *
+ *     S = scale * Q K^T               (per batch b and query head h)
+ *     S_ij = -inf where masked        (causal: key j hidden from query i iff j > i + Nk - Nq)
+ *     P = softmax(S) row by row,      O = P V
+ *     LSE_i = ln sum_j exp(S_ij)      (natural log; -inf for a row with no visible key)
+ *
+ * is the formula softmax(Q K^T / sqrt(d_k)) V with its optional causal mask, as stated
+ * on the hwcomputing.csdn.net article "FlashAttention in CANN ops-transformer"
+ * (sections "where the memory black hole of standard attention comes from" and
+ * "performance tuning", item 3 mask modes).  It is computed tile by tile with the
+ * online softmax of the same article (section "online softmax": running row max m,
+ * running sum l, rescale by exp(m_old - m_new), final O /= l), so S and P never
+ * reach device memory.  Query head h reads key/value head h / (Hq / Hkv): the
+ * repeat_interleave expansion of grouped-query attention ("Transformer efficient
+ * attention: Flash Attention vs GQA", yunthe.com, section "GQA principle").
+ * The head dimensions are those listed on the datacanvas.csdn.net head-dim article
+ * (32, 64, 96, 128, 192, 256, plus 80 added by the custom-compile workaround).
+ *
+ * Conventions for every entry point:
+ *  - All tensors are dense, row-major (C-contiguous), owned by the caller; the library
+ *    allocates no device memory per call and keeps no pointer after it returns.
+ *  - Pointers to tensors are DEVICE pointers on the calling thread's current CUDA device.
+ *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
+ *  - Work is enqueued asynchronously on `stream`; no host synchronisation happens,
+ *    except in fa_device_status.
+ *  - A non-zero return means nothing was launched.
+ */
+#ifndef EXACT_ATTENTION_FA_H
+#define EXACT_ATTENTION_FA_H
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Status codes returned by the entry points. */
+enum fa_status_code {
+    FA_OK = 0,
+    FA_ERR_INVALID_ARG = 1,          /* null pointer, negative size, Hq % Hkv != 0, scale <= 0 or
+                                        not finite, causal not 0/1, sizes beyond 32-bit indexing */
+    FA_ERR_UNSUPPORTED_HEAD_DIM = 2, /* d not in {32, 64, 80, 96, 128, 192, 256} */
+    FA_ERR_MISALIGNED = 3,           /* q/k/v/out not 16-byte aligned, or lse not 4-byte aligned */
+    FA_ERR_UNSUPPORTED_DEVICE = 4,   /* no CUDA device, or the current device is not sm_100 */
+    FA_ERR_CUDA = 5,                 /* a CUDA runtime/driver call failed (launch, tensor-map encode) */
+    FA_ERR_DEVICE_TIMEOUT = 6,       /* reported by fa_device_status: a pipeline wait in the kernel
+                                        gave up after its time limit; outputs are undefined */
+    FA_ERR_NOT_DEVICE_MEMORY = 7,    /* a tensor pointer is not device memory of the current device,
+                                        or its extent runs past the end of its allocation */
+    FA_ERR_OVERLAP = 8               /* out or lse overlaps an input or each other */
+};
+
+/*
+ * fa_fwd -- exact attention forward.
+ *
+ *   q    [B, Nq, Hq,  d] bf16, read only
+ *   k    [B, Nk, Hkv, d] bf16, read only
+ *   v    [B, Nk, Hkv, d] bf16, read only
+ *   out  [B, Nq, Hq,  d] bf16, written (O, rounded to nearest-even from fp32)
+ *   lse  [B, Hq, Nq]     fp32, written, or NULL to skip it
+ *   B >= 0, Hq >= 1, Hkv >= 1 with Hq % Hkv == 0, Nq >= 0, Nk >= 0
+ *   d in {32, 64, 80, 96, 128, 192, 256}
+ *   scale > 0 and finite (the usual choice is 1/sqrt(d)); applied to Q K^T as given
+ *   causal in {0, 1}
+ *
+ * B == 0 or Nq == 0: nothing to do, returns FA_OK.  Nk == 0: every row has no key,
+ * so out is zero and lse is -inf.  Pointers of empty tensors may be NULL.
+ * Errors are returned synchronously (see fa_status_code); a device-side pipeline
+ * timeout is reported later by fa_device_status.
+ */
+int fa_fwd(const void *q, const void *k, const void *v, void *out, float *lse,
+           int B, int Hq, int Hkv, int Nq, int Nk, int d, float scale, int causal,
+           void *stream);
+
+/* Human-readable text of a status code (static storage; never NULL). */
+const char *fa_status_string(int status);
+
+/*
+ * fa_device_status -- synchronises `stream`, then returns and clears the current
+ * device's kernel status word: FA_OK, or FA_ERR_DEVICE_TIMEOUT if a pipeline wait in
+ * an fa_fwd kernel ran out of time.  FA_ERR_CUDA if the synchronisation itself failed.
+ * If `detail` is not NULL it receives the raw status word (bits 8.. name the wait).
+ */
+int fa_device_status(void *stream, int *detail);
+
+/*
+ * fa_tile_config -- the tiling fa_fwd uses for head dimension d (host only, no GPU):
+ * rows per query tile, rows per key/value tile, query tiles per work unit, and the
+ * number of key/value tile slots in the shared-memory ring.  Any output may be NULL.
+ * Returns FA_ERR_UNSUPPORTED_HEAD_DIM for an unsupported d.
+ */
+int fa_tile_config(int d, int *block_q, int *block_k, int *q_tiles_per_unit, int *kv_slots);
+
+/* Library ABI version (major * 100 + minor). */
+int fa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* EXACT_ATTENTION_FA_H */

@@ -1,0 +1,117 @@
+"""Host-only checks of the C ABI (no GPU needed): the library builds and loads, exports
+every symbol include/fa.h declares, reports the tiling per head dim, and rejects bad
+arguments synchronously, before touching any device (fake pointers are never
+dereferenced: validation runs first)."""
+import ctypes
+import json
+import re
+from pathlib import Path
+
+import pytest
+
+import exact_attention_146_b200 as fa
+from exact_attention_146_b200 import build as fa_build
+
+ROOT = Path(__file__).resolve().parent.parent
+GOLDEN = json.loads((ROOT / "tests" / "golden" / "pages_facts.json").read_text())
+
+
+@pytest.fixture(scope="module")
+def L():
+    fa_build.build()
+    return fa.lib()
+
+
+def header_functions():
+    text = (ROOT / "include" / "fa.h").read_text()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(fa_[a-z_0-9]+)\s*\(", text)))
+
+
+def test_header_symbols_exported(L):
+    names = header_functions()
+    assert set(names) == set(fa.EXPORTED)
+    for n in names:
+        assert hasattr(L, n), n
+
+
+def test_version(L):
+    assert L.fa_version() == 100
+
+
+def test_head_dims_from_pages(L):
+    supported = GOLDEN["head_dims_listed"]["value"] + GOLDEN["head_dims_added"]["value"]
+    assert sorted(supported) == sorted(fa.SUPPORTED_HEAD_DIMS)
+    for d in supported:
+        cfg = fa.tile_config(d)
+        assert cfg["block_q"] == 128 and cfg["block_k"] in (64, 128)
+        assert cfg["q_tiles_per_unit"] in (1, 2) and cfg["kv_slots"] >= 2
+    for d in GOLDEN["head_dims_rejected_examples"]["value"]:
+        assert L.fa_tile_config(d, None, None, None, None) == fa.FA_ERR_UNSUPPORTED_HEAD_DIM
+    msg = fa.status_string(fa.FA_ERR_UNSUPPORTED_HEAD_DIM)
+    for d in supported:
+        assert str(d) in msg
+
+
+def test_kv_block_counts_match_pages(L):
+    """With the d=128 tiling, the sequence lengths the pages quote split into the number
+    of key/value blocks they state."""
+    bk = fa.tile_config(128)["block_k"]
+    for n, blocks in GOLDEN["kv_blocks_at_seq_len"]["value"]:
+        assert -(-n // bk) == blocks
+
+
+FAKE = 1 << 40  # never dereferenced: every case below fails validation first
+
+
+def call(L, q=FAKE, k=FAKE + (1 << 30), v=FAKE + (2 << 30), out=FAKE + (3 << 30), lse=FAKE + (4 << 30),
+         B=1, Hq=2, Hkv=1, Nq=16, Nk=16, d=64, scale=0.125, causal=0):
+    return L.fa_fwd(q, k, v, out, lse, B, Hq, Hkv, Nq, Nk, d, scale, causal, None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(B=-1), fa.FA_ERR_INVALID_ARG),
+    (dict(Hq=0), fa.FA_ERR_INVALID_ARG),
+    (dict(Hkv=0), fa.FA_ERR_INVALID_ARG),
+    (dict(Nq=-3), fa.FA_ERR_INVALID_ARG),
+    (dict(Nk=-1), fa.FA_ERR_INVALID_ARG),
+    (dict(Hq=3, Hkv=2), fa.FA_ERR_INVALID_ARG),
+    (dict(causal=2), fa.FA_ERR_INVALID_ARG),
+    (dict(scale=0.0), fa.FA_ERR_INVALID_ARG),
+    (dict(scale=-0.5), fa.FA_ERR_INVALID_ARG),
+    (dict(scale=float("nan")), fa.FA_ERR_INVALID_ARG),
+    (dict(scale=float("inf")), fa.FA_ERR_INVALID_ARG),
+    (dict(d=48), fa.FA_ERR_UNSUPPORTED_HEAD_DIM),
+    (dict(d=512), fa.FA_ERR_UNSUPPORTED_HEAD_DIM),
+    (dict(q=None), fa.FA_ERR_INVALID_ARG),
+    (dict(out=None), fa.FA_ERR_INVALID_ARG),
+    (dict(k=None), fa.FA_ERR_INVALID_ARG),
+    (dict(v=None), fa.FA_ERR_INVALID_ARG),
+    (dict(q=FAKE + 8), fa.FA_ERR_MISALIGNED),
+    (dict(out=FAKE + (3 << 30) + 2), fa.FA_ERR_MISALIGNED),
+    (dict(lse=FAKE + (4 << 30) + 2), fa.FA_ERR_MISALIGNED),
+    (dict(out=FAKE + 64), fa.FA_ERR_OVERLAP),                 # out inside q
+    (dict(lse=FAKE + (3 << 30) + 128), fa.FA_ERR_OVERLAP),    # lse inside out
+    (dict(lse=FAKE + (1 << 30)), fa.FA_ERR_OVERLAP),          # lse on k
+])
+def test_validation_rejects(L, kw, code):
+    assert call(L, **kw) == code
+
+
+def test_empty_problems_are_noops(L):
+    # no output rows: nothing to validate against the device, nothing launched
+    assert call(L, B=0, q=None, k=None, v=None, out=None, lse=None) == fa.FA_OK
+    assert call(L, Nq=0, q=None, out=None, lse=None) == fa.FA_OK
+
+
+def test_valid_args_without_usable_device(L):
+    """Arguments pass validation; the library must then refuse (no device here, or the
+    fake pointers are not device memory on a GPU machine) instead of launching."""
+    assert call(L) in (fa.FA_ERR_UNSUPPORTED_DEVICE, fa.FA_ERR_NOT_DEVICE_MEMORY)
+
+
+def test_status_strings(L):
+    for c in range(0, 9):
+        s = fa.status_string(c)
+        assert s and s != "unknown status"
+    assert fa.status_string(99) == "unknown status"

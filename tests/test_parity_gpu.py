@@ -1,0 +1,204 @@
+"""Parity of the CUDA path (through the C ABI) with the CPU fp64 oracle, element by
+element, on seeded inputs: small shapes that span several tiles with ragged tails for
+every head dim, GQA ratios, Nq != Nk, empty rows, the degenerate sizes, and every
+workload of the table at its full size (rows sampled from the very launch the benchmark
+times, checked one by one against the oracle)."""
+import math
+
+import numpy as np
+import pytest
+
+import oracle
+import synth
+from tests import _parity
+
+pytestmark = pytest.mark.gpu
+
+HEAD_DIMS = (32, 64, 80, 96, 128, 192, 256)
+
+
+@pytest.fixture(scope="module")
+def orc():
+    return oracle.default()
+
+
+@pytest.fixture(scope="module", autouse=True)
+def cuda_ready():
+    import torch
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from exact_attention_146_b200 import build
+    build.build()
+    yield
+
+
+def tiny(B, Hq, Hkv, Nq, Nk, d, seed, **kw):
+    w = synth.Workload("t", 500 + seed, B, Hq, Hkv, Nq, Nk, d, False, seed=seed, **kw)
+    return synth.make_inputs(w)
+
+
+def check_full(orc, x, scale, causal, what):
+    O, L = _parity.run_cuda(x, scale, causal)
+    Oref, Lref = orc.forward(x["q"], x["k"], x["v"], scale, causal)
+    return _parity.compare(O, L, Oref, Lref, what)
+
+
+@pytest.mark.parametrize("d", HEAD_DIMS)
+@pytest.mark.parametrize("N", [1, 17, 128, 129, 300, 600])
+@pytest.mark.parametrize("causal", [False, True])
+def test_small_shapes(orc, d, N, causal):
+    x = tiny(1, 2, 1, N, N, d, seed=N + d)
+    check_full(orc, x, 1.0 / math.sqrt(d), causal, f"d={d} N={N} causal={causal}")
+
+
+@pytest.mark.parametrize("Hkv", [1, 2, 4, 8])
+@pytest.mark.parametrize("causal", [False, True])
+def test_gqa_ratios(orc, Hkv, causal):
+    x = tiny(2, 8, Hkv, 200, 200, 128, seed=40 + Hkv)
+    check_full(orc, x, 1.0 / math.sqrt(128), causal, f"GQA 8/{Hkv}")
+
+
+def test_gqa_32_query_heads_per_kv_head(orc):
+    x = tiny(1, 32, 1, 130, 130, 64, seed=49)
+    check_full(orc, x, 0.125, True, "GQA 32/1")
+
+
+@pytest.mark.parametrize("Nq,Nk", [(100, 300), (300, 100), (1, 700), (257, 256), (600, 5)])
+@pytest.mark.parametrize("causal", [False, True])
+def test_unequal_lengths(orc, Nq, Nk, causal):
+    """Bottom-right aligned causal mask; Nq > Nk leaves the first rows without a key."""
+    x = tiny(1, 4, 2, Nq, Nk, 64, seed=Nq * 7 + Nk)
+    check_full(orc, x, 0.125, causal, f"Nq={Nq} Nk={Nk}")
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_large_logits_rescale_path(orc, d):
+    """Q x 8 (exact in bf16): logits of tens, row maxima keep growing along the row."""
+    x = tiny(2, 4, 4, 700, 700, d, seed=60 + d, q_mult=8.0)
+    check_full(orc, x, 1.0 / math.sqrt(d), False, "qx8")
+    check_full(orc, x, 1.0 / math.sqrt(d), True, "qx8 causal")
+
+
+def test_increasing_logits_force_rescales(orc):
+    """Keys whose logits grow tile after tile, so the running max rises past the lazy
+    rescale threshold many times."""
+    x = tiny(1, 2, 2, 256, 1024, 128, seed=70)
+    q = synth.bf16_bits_to_f32(x["q"]).copy()
+    k = synth.bf16_bits_to_f32(x["k"]).copy()
+    q[..., :] = np.abs(q)
+    ramp = np.linspace(0.0, 6.0, 1024, dtype=np.float32)[None, :, None, None]
+    k = np.abs(k) * ramp
+    x = {"q": synth.f32_to_bf16_bits(q), "k": synth.f32_to_bf16_bits(k), "v": x["v"]}
+    check_full(orc, x, 1.0 / math.sqrt(128), False, "ramp")
+    check_full(orc, x, 1.0 / math.sqrt(128), True, "ramp causal")
+
+
+def test_lse_optional(orc):
+    x = tiny(1, 2, 1, 200, 200, 64, seed=80)
+    O, L = _parity.run_cuda(x, 0.125, True, with_lse=False)
+    Oref, _ = orc.forward(x["q"], x["k"], x["v"], 0.125, True)
+    _parity.compare(O, None, Oref, None, "no lse")
+
+
+def test_no_keys():
+    """Nk = 0: O = 0, LSE = -inf."""
+    x = tiny(2, 2, 1, 50, 0, 64, seed=81)
+    O, L = _parity.run_cuda(x, 0.125, False)
+    assert (O == 0).all() and np.isneginf(L).all()
+
+
+def test_empty_problems():
+    """B = 0 or Nq = 0: nothing to compute, FA_OK, nothing launched."""
+    import torch
+    import exact_attention_146_b200 as fa
+    kv = torch.zeros((1, 16, 2, 64), dtype=torch.bfloat16, device="cuda")
+    q0 = torch.zeros((0, 16, 2, 64), dtype=torch.bfloat16, device="cuda")
+    out, lse = fa.fa_fwd(q0, kv[:0], kv[:0])
+    assert out.shape == q0.shape and lse.shape == (0, 2, 16)
+    q1 = torch.zeros((1, 0, 2, 64), dtype=torch.bfloat16, device="cuda")
+    out, lse = fa.fa_fwd(q1, kv, kv)
+    assert out.numel() == 0 and lse.numel() == 0
+    assert fa.device_status()[0] == fa.FA_OK
+
+
+def test_rejects_host_memory():
+    import torch
+    import exact_attention_146_b200 as fa
+    qh = torch.zeros((1, 64, 2, 64), dtype=torch.int16).view(torch.bfloat16)
+    qd = torch.zeros((1, 64, 2, 64), dtype=torch.bfloat16, device="cuda")
+    od = torch.empty_like(qd)
+    rc = fa.fa_fwd_raw(qh.data_ptr(), qd.data_ptr(), qd.data_ptr(), od.data_ptr(), None,
+                       1, 2, 2, 64, 64, 64, 0.125, 0, 0)
+    assert rc == fa.FA_ERR_NOT_DEVICE_MEMORY
+    assert fa.device_status()[0] == fa.FA_OK
+
+
+def _cudart():
+    try:
+        from cuda.bindings import runtime as rt
+    except ImportError:
+        try:
+            from cuda import cudart as rt
+        except ImportError:
+            pytest.skip("cuda-python not available")
+    return rt
+
+
+def test_rejects_buffer_shorter_than_sizes():
+    """A K/V buffer shorter than B*Nk*Hkv*d elements is refused before any launch."""
+    import torch
+    import exact_attention_146_b200 as fa
+    rt = _cudart()
+    err, kbuf = rt.cudaMalloc(1 << 20)
+    assert int(err) == 0
+    try:
+        q = torch.zeros((1, 64, 2, 64), dtype=torch.bfloat16, device="cuda")
+        out = torch.empty_like(q)
+        Nk = 1 << 16                          # claims 16 MiB of K and of V
+        lo, hi = int(kbuf), int(kbuf) + Nk * 2 * 64 * 2
+        for t in (q, out):
+            if lo < t.data_ptr() + t.numel() * 2 and t.data_ptr() < hi:
+                pytest.skip("allocator placed the tensors inside the claimed range")
+        rc = fa.fa_fwd_raw(q.data_ptr(), int(kbuf), int(kbuf), out.data_ptr(), None,
+                           1, 2, 2, 64, Nk, 64, 0.125, 0, 0)
+        assert rc == fa.FA_ERR_NOT_DEVICE_MEMORY
+    finally:
+        rt.cudaFree(kbuf)
+    assert fa.device_status()[0] == fa.FA_OK
+
+
+def test_deterministic(orc):
+    x = tiny(2, 4, 2, 333, 333, 128, seed=90)
+    O1, L1 = _parity.run_cuda(x, 0.1, True)
+    O2, L2 = _parity.run_cuda(x, 0.1, True)
+    assert np.array_equal(O1, O2) and np.array_equal(L1, L2)
+
+
+# ------------------------------------------------------------------ workload table
+
+SMALL_FULL = ["yolo20x20_b1_h4_d64", "yolo20x20_b1_h4_d64_qx8", "yolo20x20_b32_h16_d64"]
+LARGE_SAMPLED = [n for n in synth.WORKLOADS if n not in SMALL_FULL]
+
+
+@pytest.mark.parametrize("name", SMALL_FULL)
+def test_workload_full(orc, name):
+    w = synth.WORKLOADS[name]
+    x = synth.make_inputs(w)
+    res = check_full(orc, x, w.scale, w.causal, name)
+    print(name, res)
+
+
+@pytest.mark.parametrize("name", LARGE_SAMPLED)
+def test_workload_sampled_rows(orc, name):
+    """Full-size launch (the one the benchmark times); sampled rows checked against the
+    oracle one by one, and every output row checked to be written and finite."""
+    w = synth.WORKLOADS[name]
+    x = synth.make_inputs(w)
+    O, L = _parity.run_cuda(x, w.scale, w.causal)
+    assert np.isfinite(O).all() and np.isfinite(L).all()
+    rows = _parity.sample_rows(w, 192, seed=w.wid)
+    Oref, Lref = orc.rows(x["q"], x["k"], x["v"], rows, w.scale, w.causal)
+    Os = O[rows[:, 0], rows[:, 2], rows[:, 1], :]
+    Ls = L[rows[:, 0], rows[:, 1], rows[:, 2]]
+    res = _parity.compare(Os, Ls, Oref, Lref, name)
+    print(name, len(rows), res)
