@@ -321,6 +321,53 @@ def run_ours(args, w, world, rank, local):
     return 0
 
 
+def run_sweep(args):
+    """Every workload of the table, one JSON line each (device time only, 1 GPU)."""
+    import torch
+    import exact_attention_146_b200 as fa
+    torch.cuda.set_device(0)
+    pk = peaks()
+    names = args.sweep_only.split(",") if args.sweep_only else list(synth.WORKLOADS)
+    for name in names:
+        w = synth.WORKLOADS[name]
+        x = synth.make_inputs(w)
+        q, k, v = (torch.from_numpy(x[n].view(np.int16)).view(torch.bfloat16).cuda() for n in ("q", "k", "v"))
+        out = torch.empty_like(q)
+        lse = torch.empty((w.B, w.Hq, w.Nq), dtype=torch.float32, device="cuda")
+        # inputs smaller than L2 are timed both warm and with an L2 flush before each launch
+        flush = torch.empty(int(2 * 126e6) // 4, dtype=torch.float32, device="cuda")
+        for _ in range(args.warmup):
+            fa.fa_fwd(q, k, v, causal=w.causal, scale=w.scale, out=out, lse=lse)
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(args.steps):
+            fa.fa_fwd(q, k, v, causal=w.causal, scale=w.scale, out=out, lse=lse)
+        e1.record()
+        torch.cuda.synchronize()
+        ms_warm = e0.elapsed_time(e1) / args.steps
+        cold = []
+        for _ in range(min(args.steps, 20)):
+            flush.zero_()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            fa.fa_fwd(q, k, v, causal=w.causal, scale=w.scale, out=out, lse=lse)
+            b.record()
+            torch.cuda.synchronize()
+            cold.append(a.elapsed_time(b))
+        ms_cold = statistics.median(cold)
+        st, word = fa.device_status()
+        roof_ms = max(w.flops / (pk["bf16_tflops"] * 1e12), w.io_bytes / (pk["hbm_gbs"] * 1e9)) * 1e3
+        print(json.dumps({
+            "workload": name, "ms_warm": ms_warm, "ms_l2_flushed": ms_cold,
+            "tflops": w.flops / (ms_cold * 1e-3) / 1e12, "pct_peak": 100 * w.flops / (ms_cold * 1e-3) / 1e12 / pk["bf16_tflops"],
+            "hbm_gbs": w.io_bytes / (ms_cold * 1e-3) / 1e9, "roofline_ms": roof_ms,
+            "roofline_frac": roof_ms / ms_cold, "status": st}), flush=True)
+        del q, k, v, out, lse, flush
+        torch.cuda.empty_cache()
+    return 0
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
@@ -333,9 +380,13 @@ def main(argv=None):
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-clocks", action="store_true")
+    ap.add_argument("--sweep", action="store_true", help="time every workload of the table (1 GPU)")
+    ap.add_argument("--sweep-only", default="", help="comma-separated workload names for --sweep")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
+    if args.sweep:
+        return run_sweep(args)
     w = synth.WORKLOADS[args.workload]
     world, rank, local = dist_setup(args.gpus)
     if args.impl == "reference":

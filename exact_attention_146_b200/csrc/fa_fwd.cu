@@ -38,6 +38,7 @@ struct DeviceState {
     int num_sms = 0;
     int *status_ptr = nullptr;
     bool smem_attr_set[8] = {};
+    int regs_ok[8] = {};          // 0 unknown, 1 verified, -1 mismatch
 };
 DeviceState g_devices[kMaxDevices];
 std::mutex g_mutex;
@@ -164,6 +165,17 @@ int launch(const Problem &pr, DeviceState &dev, int cfg_slot, cudaStream_t strea
         }
         dev.smem_attr_set[cfg_slot] = true;
     }
+    if (dev.regs_ok[cfg_slot] == 0) {
+        // The in-kernel register reallocation assumes the kernel is launched with exactly
+        // C::LAUNCH_REGS registers per thread; refuse to launch a build that differs.
+        cudaFuncAttributes fattr{};
+        if (cudaFuncGetAttributes(&fattr, kern) != cudaSuccess) {
+            cudaGetLastError();
+            return FA_ERR_CUDA;
+        }
+        dev.regs_ok[cfg_slot] = (!C::REALLOC_REGS || fattr.numRegs == C::LAUNCH_REGS) ? 1 : -1;
+    }
+    if (dev.regs_ok[cfg_slot] != 1) return FA_ERR_CUDA;
     CUtensorMap mq, mk, mv;
     int rc;
     if ((rc = encode_bnhd(&mq, pr.q, C::D, pr.Hq, pr.Nq, pr.B, C::CW, kBlockQ)) != FA_OK) return rc;

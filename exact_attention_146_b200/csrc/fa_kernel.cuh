@@ -88,11 +88,23 @@ struct TileCfg {
     // second CTA can never be resident on the same SM (it would only wait in alloc).
     static constexpr int SMEM_NEEDED = SMEM_MISC + 16 + 1024;
     static constexpr int SMEM_BYTES = SMEM_NEEDED > 120 * 1024 ? SMEM_NEEDED : 120 * 1024;
-    // warps: 4 per query tile (softmax), then the TMA warp and the MMA warp
+    // warps: one warpgroup per query tile (softmax), then a control warpgroup holding the
+    // TMA warp and the MMA warp (two warps of it idle: register reallocation works on
+    // whole warpgroups).
     static constexpr int SOFTMAX_WARPS = 4 * NQT;
     static constexpr int TMA_WARP = SOFTMAX_WARPS;
     static constexpr int MMA_WARP = SOFTMAX_WARPS + 1;
-    static constexpr int THREADS = 32 * (SOFTMAX_WARPS + 2);
+    static constexpr int THREADS = 32 * (SOFTMAX_WARPS + 4);
+    // Registers per thread: the launch budget (65536 / THREADS rounded down to 8) and,
+    // for two query tiles, the split moved from the control warpgroup to the softmax
+    // warpgroups.  LAUNCH_REGS is checked against the compiled kernel on the host before
+    // the first launch.
+    static constexpr int LAUNCH_REGS = ((65536 / THREADS) / 8) * 8 > 255 ? 255 : ((65536 / THREADS) / 8) * 8;
+    static constexpr bool REALLOC_REGS = (NQT == 2);
+    static constexpr int SOFTMAX_REGS = 216;
+    static constexpr int CONTROL_REGS = 72;
+    static_assert(!REALLOC_REGS || (SOFTMAX_REGS * 32 * SOFTMAX_WARPS + CONTROL_REGS * 128 <= LAUNCH_REGS * THREADS),
+                  "register split exceeds the launch budget");
     static constexpr uint32_t IDESC_S = sm100::idesc_bf16_f32(kBlockQ, BC, 0, 0);
     static constexpr uint32_t IDESC_O = sm100::idesc_bf16_f32(kBlockQ, D, 0, 1);
 
@@ -163,7 +175,7 @@ struct Ctl {
 // Poll `bar` until the phase of parity `parity` completes.  Gives up when another role
 // has raised the abort flag (unless `drain`: unwinding waits for the hardware's own
 // copies/MMAs regardless) or after `limit_ns`, recording the timeout in the status word.
-__device__ __noinline__ bool wait_slow(uint32_t bar, uint32_t parity, Ctl ctl, int site,
+__device__ __forceinline__ bool wait_slow(uint32_t bar, uint32_t parity, Ctl ctl, int site,
                                        uint64_t limit_ns, bool drain = false) {
     const uint64_t t0 = sm100::global_timer_ns();
     while (true) {
@@ -256,7 +268,9 @@ template <class C>
 __device__ __forceinline__ void issue_qk(uint32_t sbase, uint32_t tmem, int t, int slot) {
     const uint32_t qa = sbase + C::SMEM_Q + t * C::Q_TILE;
     const uint32_t kb = sbase + C::SMEM_KV + slot * C::KV_TILE;
-#pragma unroll
+    // Rolled loops: one MMA per 64+ tensor cycles leaves ample issue time, and keeps the
+    // control warpgroup's register needs small.
+#pragma unroll 1
     for (int kk = 0; kk < C::D / 16; ++kk) {
         const int ch = (kk * 16) / C::CW;
         const uint32_t off = uint32_t((kk * 16) % C::CW) * 2u;
@@ -269,7 +283,7 @@ __device__ __forceinline__ void issue_qk(uint32_t sbase, uint32_t tmem, int t, i
 template <class C>
 __device__ __forceinline__ void issue_pv(uint32_t sbase, uint32_t tmem, int t, int slot, bool accumulate) {
     const uint32_t vb = sbase + C::SMEM_KV + slot * C::KV_TILE;
-#pragma unroll
+#pragma unroll 1
     for (int kk = 0; kk < C::BC / 16; ++kk) {
         // V tile is [BC rows x d] row-major: MN-major B operand; 16 key rows per MMA,
         // 64-element column chunks C::KV_CHUNK bytes apart (leading byte offset).
@@ -347,6 +361,52 @@ __device__ void mma_role(const FwdParams &p, uint32_t sbase, uint32_t tmem, cons
 
 // ------------------------------------------------------------------ softmax / epilogue
 
+// p = 2^(s * c_log2 - m) for one row of a score tile, packed to bf16 pairs and stored
+// over the first BC/2 TMEM columns of the tile (P overwrites S); returns the fp32 row
+// sum of p.  On unmasked tiles a share of the pairs (kSoftExpPairsPer8 of every 8) take
+// the FMA-pipe exponential so the special-function unit is not the bottleneck; masked
+// tiles (which may hold -inf scores) use the hardware ex2 throughout.
+#ifndef FA_SOFT_EXP_PAIRS_PER_8
+#define FA_SOFT_EXP_PAIRS_PER_8 2
+#endif
+constexpr int kSoftExpPairsPer8 = FA_SOFT_EXP_PAIRS_PER_8;
+static_assert(kSoftExpPairsPer8 >= 0 && kSoftExpPairsPer8 <= 8, "share of software exponentials");
+
+template <int BC, bool MIXED>
+__device__ __forceinline__ float exp_pack_store(const uint32_t (&s)[BC], float c_log2, float neg_m,
+                                                uint32_t s_taddr) {
+    const uint64_t c2 = sm100::pack2(c_log2, c_log2);
+    const uint64_t nm2 = sm100::pack2(neg_m, neg_m);
+    uint64_t acc0 = sm100::pack2(0.f, 0.f), acc1 = acc0;
+#pragma unroll
+    for (int c = 0; c < BC / 64; ++c) {
+        uint32_t pk[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+            const int e = 64 * c + 2 * i;
+            const uint64_t x2 = sm100::fma2(sm100::pack2(__uint_as_float(s[e]), __uint_as_float(s[e + 1])), c2, nm2);
+            uint64_t p2;
+            if (MIXED && (i % 8) >= 8 - kSoftExpPairsPer8) {
+                p2 = sm100::ex2_poly_pair(x2);
+            } else {
+                float a, b;
+                sm100::unpack2(x2, a, b);
+                p2 = sm100::pack2(sm100::ex2_approx(a), sm100::ex2_approx(b));
+            }
+            if (i & 1) acc1 = sm100::add2(acc1, p2);
+            else acc0 = sm100::add2(acc0, p2);
+            float lo, hi;
+            sm100::unpack2(p2, lo, hi);
+            pk[i] = sm100::pack_bf16x2(lo, hi);
+        }
+        sm100::tmem_st32(s_taddr + uint32_t(32 * c), pk);
+    }
+    float a0, a1, b0, b1;
+    sm100::unpack2(acc0, a0, a1);
+    sm100::unpack2(acc1, b0, b1);
+    return (a0 + a1) + (b0 + b1);
+}
+
 template <class C>
 __device__ void softmax_role(const FwdParams &p, uint32_t sbase, uint32_t tmem, const Ctl &ctl,
                              int warp, int lane) {
@@ -375,32 +435,28 @@ __device__ void softmax_role(const FwdParams &p, uint32_t sbase, uint32_t tmem, 
             if (!warp_wait_bar(bar(C::B_SFULL + t), scnt & 1u, ctl, kSiteSFull)) goto unwind;
             ++scnt;
             sm100::tc_fence_after_sync();
-            uint32_t s[BC / 32][32];
-#pragma unroll
-            for (int c = 0; c < BC / 32; ++c) sm100::tmem_ld32_sync(s_taddr + uint32_t(32 * c), s[c]);
+            uint32_t s[BC];
+            if constexpr (BC == 128) sm100::tmem_ld128_sync(s_taddr, s);
+            else sm100::tmem_ld64_sync(s_taddr, s);
 
             const int k_lo = j * BC;
             const bool need_mask = (k_lo + BC > p.Nk) || (p.causal && k_lo + BC - 1 > q_lo + diag);
             if (need_mask) {
 #pragma unroll
-                for (int c = 0; c < BC / 32; ++c)
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) {
-                        const int key = k_lo + 32 * c + i;
-                        if (key > row_lim || key >= p.Nk) s[c][i] = __float_as_uint(-INFINITY);
-                    }
+                for (int i = 0; i < BC; ++i) {
+                    const int key = k_lo + i;
+                    if (key > row_lim || key >= p.Nk) s[i] = __float_as_uint(-INFINITY);
+                }
             }
             float mx0 = -INFINITY, mx1 = -INFINITY, mx2 = -INFINITY, mx3 = -INFINITY;
 #pragma unroll
-            for (int c = 0; c < BC / 32; ++c)
-#pragma unroll
-                for (int i = 0; i < 32; i += 4) {
-                    mx0 = fmaxf(mx0, __uint_as_float(s[c][i]));
-                    mx1 = fmaxf(mx1, __uint_as_float(s[c][i + 1]));
-                    mx2 = fmaxf(mx2, __uint_as_float(s[c][i + 2]));
-                    mx3 = fmaxf(mx3, __uint_as_float(s[c][i + 3]));
-                }
-            const float mx_s = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * c_log2;
+            for (int i = 0; i < BC; i += 8) {
+                mx0 = sm100::max3(mx0, __uint_as_float(s[i]), __uint_as_float(s[i + 1]));
+                mx1 = sm100::max3(mx1, __uint_as_float(s[i + 2]), __uint_as_float(s[i + 3]));
+                mx2 = sm100::max3(mx2, __uint_as_float(s[i + 4]), __uint_as_float(s[i + 5]));
+                mx3 = sm100::max3(mx3, __uint_as_float(s[i + 6]), __uint_as_float(s[i + 7]));
+            }
+            const float mx_s = sm100::max3(mx0, mx1, fmaxf(mx2, mx3)) * c_log2;
             float alpha = 1.f;
             bool need_rescale = false;
             if (j == 0) {
@@ -411,24 +467,9 @@ __device__ void softmax_role(const FwdParams &p, uint32_t sbase, uint32_t tmem, 
                 need_rescale = true;
             }
             const float neg_m = (m_ref == -INFINITY) ? 0.f : -m_ref;
-            float sum0 = 0.f, sum1 = 0.f, sum2 = 0.f, sum3 = 0.f;
-#pragma unroll
-            for (int c = 0; c < BC / 64; ++c) {
-                uint32_t pk[32];
-#pragma unroll
-                for (int i = 0; i < 32; i += 2) {
-                    const int e = 64 * c + 2 * i;          // element index of this pair
-                    const float p0 = sm100::ex2_approx(fmaf(__uint_as_float(s[e / 32][e % 32]), c_log2, neg_m));
-                    const float p1 = sm100::ex2_approx(fmaf(__uint_as_float(s[e / 32][e % 32 + 1]), c_log2, neg_m));
-                    const float p2 = sm100::ex2_approx(fmaf(__uint_as_float(s[e / 32][e % 32 + 2]), c_log2, neg_m));
-                    const float p3 = sm100::ex2_approx(fmaf(__uint_as_float(s[e / 32][e % 32 + 3]), c_log2, neg_m));
-                    sum0 += p0; sum1 += p1; sum2 += p2; sum3 += p3;
-                    pk[i] = sm100::pack_bf16x2(p0, p1);
-                    pk[i + 1] = sm100::pack_bf16x2(p2, p3);
-                }
-                sm100::tmem_st32(s_taddr + uint32_t(32 * c), pk);
-            }
-            l = l * alpha + ((sum0 + sum1) + (sum2 + sum3));
+            const float row_sum = need_mask ? exp_pack_store<BC, false>(s, c_log2, neg_m, s_taddr)
+                                            : exp_pack_store<BC, true>(s, c_log2, neg_m, s_taddr);
+            l = l * alpha + row_sum;
 
             if (__any_sync(0xffffffffu, need_rescale)) {
                 // O_t holds the sum up to block j-1 at the old reference; wait for that
@@ -536,11 +577,15 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     const uint32_t tmem = *tmem_holder;
 
     if (warp < C::SOFTMAX_WARPS) {
+        if constexpr (C::REALLOC_REGS) sm100::regs_increase<C::SOFTMAX_REGS>();
         softmax_role<C>(p, sbase, tmem, ctl, warp, lane);
-    } else if (warp == C::TMA_WARP) {
-        if (lane == 0) producer_role<C>(&tm_q, &tm_k, &tm_v, p, sbase, ctl);
-    } else if (warp == C::MMA_WARP) {
-        if (lane == 0) mma_role<C>(p, sbase, tmem, ctl);
+    } else {
+        if constexpr (C::REALLOC_REGS) sm100::regs_decrease<C::CONTROL_REGS>();
+        if (warp == C::TMA_WARP) {
+            if (lane == 0) producer_role<C>(&tm_q, &tm_k, &tm_v, p, sbase, ctl);
+        } else if (warp == C::MMA_WARP) {
+            if (lane == 0) mma_role<C>(p, sbase, tmem, ctl);
+        }
     }
     __syncwarp();
 
