@@ -125,6 +125,26 @@ def dist_setup(n_gpus):
     return world, rank, local
 
 
+def rank_workload(w: synth.Workload, rank: int) -> synth.Workload:
+    """Each rank's replica: the same shapes on its own seeded data (weak scaling)."""
+    return w.with_(seed=w.seed + rank)
+
+
+def max_over_ranks(value: float, dist=None, device=None) -> float:
+    """The max of a per-rank figure (time) over all ranks; the identity without a group."""
+    if dist is None:
+        return value
+    import torch
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def weak_scaling_tflops(w: synth.Workload, world: int, ms_max: float) -> float:
+    """Whole-job throughput: every rank processed one workload in (at most) ms_max."""
+    return world * w.flops / (ms_max * 1e-3) / 1e12
+
+
 def oracle_sample_tflops(w: synth.Workload, target_s: float, heads_cap: int | None = None):
     """Time the CPU oracle on a bounded sample of the workload: whole (b, hq) heads of
     batch element 0, as many as fit in ~target_s.  Returns (TFLOP/s, sample text, cores)."""
@@ -204,7 +224,7 @@ def run_ours(args, w, world, rank, local):
     stream = torch.cuda.current_stream()
 
     # per-rank replica of the workload on its own seeded data (weak scaling)
-    wr = w.with_(seed=w.seed + rank)
+    wr = rank_workload(w, rank)
     x = synth.make_inputs(wr)
     host = {n: torch.from_numpy(x[n].view(np.int16)).view(torch.bfloat16).pin_memory() for n in ("q", "k", "v")}
     q, k, v = (host[n].to(dev, non_blocking=True) for n in ("q", "k", "v"))
@@ -246,13 +266,8 @@ def run_ours(args, w, world, rank, local):
         time.sleep(0.15)
         sampler.stop()
         clocks = ClockSampler.summarize(sampler.window(t_wall0, t_wall1 + 0.1))
-    ms_max = ms
-    if pg:
-        t = torch.tensor([ms], device=dev, dtype=torch.float64)
-        pg.all_reduce(t, op=pg.ReduceOp.MAX)
-        ms_max = float(t.item())
-
-    value = world * w.flops / (ms_max * 1e-3) / 1e12
+    ms_max = max_over_ranks(ms, pg, dev)
+    value = weak_scaling_tflops(w, world, ms_max)
     pk = peaks()
     achieved = w.flops / (ms * 1e-3) / 1e12           # per launch on this rank
     roofline = {"bound": "tensor", "achieved": achieved, "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
@@ -286,14 +301,10 @@ def run_ours(args, w, world, rank, local):
             e2e_step()
         f1.record(stream)
         torch.cuda.synchronize()
-        ms_e2e = f0.elapsed_time(f1) / n_e2e
-        if pg:
-            t = torch.tensor([ms_e2e], device=dev, dtype=torch.float64)
-            pg.all_reduce(t, op=pg.ReduceOp.MAX)
-            ms_e2e = float(t.item())
+        ms_e2e = max_over_ranks(f0.elapsed_time(f1) / n_e2e, pg, dev)
         h2d = sum(host[n].numel() * 2 for n in ("q", "k", "v"))
         d2h = out.numel() * 2 + lse.numel() * 4
-        e2e = {"value": world * w.flops / (ms_e2e * 1e-3) / 1e12, "unit": "TFLOP/s", "ms_per_step": ms_e2e,
+        e2e = {"value": weak_scaling_tflops(w, world, ms_e2e), "unit": "TFLOP/s", "ms_per_step": ms_e2e,
                "steps": n_e2e, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
 
     cpu = None
