@@ -20,8 +20,8 @@ namespace {
 using namespace fa;
 
 // Tiling per head dim: TileCfg<d, key rows per tile, query tiles per unit, K/V slots>.
-using Cfg32 = TileCfg<32, 128, 2, 8>;
-using Cfg64 = TileCfg<64, 128, 2, 8>;
+using Cfg32 = TileCfg<32, 128, 2, 8, 2>;
+using Cfg64 = TileCfg<64, 128, 2, 8, 2>;
 using Cfg80 = TileCfg<80, 128, 2, 4>;
 using Cfg96 = TileCfg<96, 128, 2, 4>;
 using Cfg128 = TileCfg<128, 128, 2, 4>;

@@ -58,12 +58,13 @@ struct FwdParams {
 };
 
 // Compile-time tiling for one head dimension.
-template <int D_, int BC_, int NQT_, int NS_>
+template <int D_, int BC_, int NQT_, int NS_, int NQB_ = 1>
 struct TileCfg {
     static constexpr int D = D_;        // head dim
     static constexpr int BC = BC_;      // key/value rows per tile
     static constexpr int NQT = NQT_;    // query tiles per unit (1 or 2)
     static constexpr int NS = NS_;      // K/V slots in the ring
+    static constexpr int NQB = NQB_;    // buffers per query tile (2: next unit's Q loads early)
     static constexpr int CW = (D == 32) ? 32 : 64;       // elements per swizzled smem row
     static constexpr int RB = CW * 2;                     // bytes per swizzled row (64 or 128)
     static constexpr int NCH = (D + CW - 1) / CW;         // column chunks of a tile
@@ -80,9 +81,9 @@ struct TileCfg {
     static constexpr int O_CHUNKS = (D + 31) / 32;
     // shared memory (offsets from a 1024-byte aligned base)
     static constexpr int SMEM_Q = 0;
-    static constexpr int SMEM_KV = NQT * Q_TILE;
+    static constexpr int SMEM_KV = NQT * NQB * Q_TILE;
     static constexpr int SMEM_BAR = SMEM_KV + NS * KV_TILE;
-    static constexpr int NUM_BARS = 2 * NS + 6 * NQT + 1;
+    static constexpr int NUM_BARS = 2 * NS + 2 * NQT * NQB + 4 * NQT + 1;
     static constexpr int SMEM_MISC = SMEM_BAR + NUM_BARS * 8;
     // Each CTA holds all 512 TMEM columns, so ask for enough shared memory that a
     // second CTA can never be resident on the same SM (it would only wait in alloc).
@@ -109,15 +110,15 @@ struct TileCfg {
     static constexpr uint32_t IDESC_O = sm100::idesc_bf16_f32(kBlockQ, D, 0, 1);
 
     static_assert(NQT == 1 || NQT == 2, "one or two query tiles per unit");
+    static_assert(NQB == 1 || NQB == 2, "one or two buffers per query tile");
     static_assert(D % 16 == 0 && D >= 32 && D <= 256, "MMA N and K granularity");
     static_assert(BC % 64 == 0 && BC <= 256, "key tile: whole 32-column TMEM chunks of P");
     static_assert(O_COL0 + NQT * OST <= TMEM_COLS, "TMEM budget");
     static_assert(SMEM_BYTES <= 232448, "shared memory budget");
-    // barrier indices
-    static constexpr int B_FULL = 0, B_EMPTY = NS, B_QFULL = 2 * NS, B_QEMPTY = 2 * NS + NQT,
-                         B_SFULL = 2 * NS + 2 * NQT, B_PFULL = 2 * NS + 3 * NQT,
-                         B_ODONE = 2 * NS + 4 * NQT, B_OEMPTY = 2 * NS + 5 * NQT,
-                         B_DRAIN = 2 * NS + 6 * NQT;
+    // barrier indices (query-tile barriers are indexed t * NQB + buffer)
+    static constexpr int B_FULL = 0, B_EMPTY = NS, B_QFULL = 2 * NS, B_QEMPTY = 2 * NS + NQT * NQB,
+                         B_SFULL = 2 * NS + 2 * NQT * NQB, B_PFULL = B_SFULL + NQT,
+                         B_ODONE = B_PFULL + NQT, B_OEMPTY = B_ODONE + NQT, B_DRAIN = B_OEMPTY + NQT;
 };
 
 struct UnitInfo {
@@ -175,6 +176,9 @@ struct Ctl {
 // Poll `bar` until the phase of parity `parity` completes.  Gives up when another role
 // has raised the abort flag (unless `drain`: unwinding waits for the hardware's own
 // copies/MMAs regardless) or after `limit_ns`, recording the timeout in the status word.
+// Out of line and instantiated per role (ROLE), so each copy is compiled under the
+// register budget of the warpgroup that calls it.
+template <int ROLE>
 __device__ __forceinline__ bool wait_slow(uint32_t bar, uint32_t parity, Ctl ctl, int site,
                                        uint64_t limit_ns, bool drain = false) {
     const uint64_t t0 = sm100::global_timer_ns();
@@ -191,15 +195,19 @@ __device__ __forceinline__ bool wait_slow(uint32_t bar, uint32_t parity, Ctl ctl
     }
 }
 
+constexpr int kRoleSoftmax = 0, kRoleControl = 1;
+
+template <int ROLE = kRoleControl>
 __device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, const Ctl &ctl, int site,
                                          uint64_t limit_ns = kWaitLimitNs) {
     if (sm100::mbar_try_wait(bar, parity)) return true;
-    return wait_slow(bar, parity, ctl, site, limit_ns);
+    return wait_slow<ROLE>(bar, parity, ctl, site, limit_ns);
 }
 
 // Warp-uniform wait: every lane polls, the warp proceeds only if all lanes saw it.
+template <int ROLE = kRoleSoftmax>
 __device__ __forceinline__ bool warp_wait_bar(uint32_t bar, uint32_t parity, const Ctl &ctl, int site) {
-    const bool ok = wait_bar(bar, parity, ctl, site);
+    const bool ok = wait_bar<ROLE>(bar, parity, ctl, site);
     const bool all = __all_sync(0xffffffffu, ok);
     if (!all) *ctl.abort_flag = 1;
     return all;
@@ -223,27 +231,31 @@ __device__ void producer_role(const CUtensorMap *tm_q, const CUtensorMap *tm_k, 
 #pragma unroll
         for (int t = 0; t < C::NQT; ++t) {
             if (!ok || w.nk[t] == 0) continue;
-            if (!wait_bar(bar(C::B_QEMPTY + t), (qcnt[t] & 1u) ^ 1u, ctl, kSiteQEmpty)) { ok = false; break; }
+            const int qb = int(qcnt[t] % C::NQB);
+            if (!warp_wait_bar<kRoleControl>(bar(C::B_QEMPTY + t * C::NQB + qb), ((qcnt[t] / C::NQB) & 1u) ^ 1u, ctl, kSiteQEmpty)) {
+                ok = false;
+                break;
+            }
             ++qcnt[t];
-            const uint32_t fb = bar(C::B_QFULL + t);
-            sm100::mbar_arrive_expect_tx(fb, C::Q_TILE);
-            const uint32_t dst = sbase + C::SMEM_Q + t * C::Q_TILE;
+            const uint32_t fb = bar(C::B_QFULL + t * C::NQB + qb);
+            sm100::mbar_arrive_expect_tx_elected(fb, C::Q_TILE);
+            const uint32_t dst = sbase + C::SMEM_Q + (t * C::NQB + qb) * C::Q_TILE;
 #pragma unroll
             for (int c = 0; c < C::NCH; ++c)
-                sm100::tma_load_4d(dst + c * C::Q_CHUNK, tm_q, fb, c * C::CW, w.hq, w.q0 + t * kBlockQ, w.b);
+                sm100::tma_load_4d_elected(dst + c * C::Q_CHUNK, tm_q, fb, c * C::CW, w.hq, w.q0 + t * kBlockQ, w.b);
         }
         for (int j = 0; ok && j < w.nk_max; ++j) {
 #pragma unroll
             for (int which = 0; which < 2; ++which) {
                 const int s = int(kv_cnt % C::NS);
-                if (!wait_bar(bar(C::B_EMPTY + s), ((kv_cnt / C::NS) & 1u) ^ 1u, ctl, kSiteKvEmpty)) { ok = false; break; }
+                if (!warp_wait_bar<kRoleControl>(bar(C::B_EMPTY + s), ((kv_cnt / C::NS) & 1u) ^ 1u, ctl, kSiteKvEmpty)) { ok = false; break; }
                 const uint32_t fb = bar(C::B_FULL + s);
-                sm100::mbar_arrive_expect_tx(fb, C::KV_TILE);
+                sm100::mbar_arrive_expect_tx_elected(fb, C::KV_TILE);
                 const uint32_t dst = sbase + C::SMEM_KV + s * C::KV_TILE;
                 const CUtensorMap *m = which ? tm_v : tm_k;
 #pragma unroll
                 for (int c = 0; c < C::NCH; ++c)
-                    sm100::tma_load_4d(dst + c * C::KV_CHUNK, m, fb, c * C::CW, w.kvh, j * C::BC, w.b);
+                    sm100::tma_load_4d_elected(dst + c * C::KV_CHUNK, m, fb, c * C::CW, w.kvh, j * C::BC, w.b);
                 ++kv_cnt;
             }
         }
@@ -253,45 +265,49 @@ __device__ void producer_role(const CUtensorMap *tm_q, const CUtensorMap *tm_k, 
         // before the CTA exits (the last load issued into each slot, and each Q tile).
         const uint32_t first = kv_cnt > uint32_t(C::NS) ? kv_cnt - C::NS : 0u;
         for (uint32_t n = first; n < kv_cnt; ++n)
-            wait_slow(bar(C::B_FULL + int(n % C::NS)), (n / C::NS) & 1u, ctl, kSiteProducerDrain,
+            wait_slow<kRoleControl>(bar(C::B_FULL + int(n % C::NS)), (n / C::NS) & 1u, ctl, kSiteProducerDrain,
                       kWaitLimitNs / 10, true);
 #pragma unroll
-        for (int t = 0; t < C::NQT; ++t)
-            if (qcnt[t] > 0)
-                wait_slow(bar(C::B_QFULL + t), (qcnt[t] - 1) & 1u, ctl, kSiteProducerDrain, kWaitLimitNs / 10, true);
+        for (int t = 0; t < C::NQT; ++t) {
+            const uint32_t first_q = qcnt[t] > uint32_t(C::NQB) ? qcnt[t] - C::NQB : 0u;
+            for (uint32_t n = first_q; n < qcnt[t]; ++n)
+                wait_slow<kRoleControl>(bar(C::B_QFULL + t * C::NQB + int(n % C::NQB)), (n / C::NQB) & 1u, ctl,
+                          kSiteProducerDrain, kWaitLimitNs / 10, true);
+        }
     }
 }
 
 // ------------------------------------------------------------------ MMA issuer
 
 template <class C>
-__device__ __forceinline__ void issue_qk(uint32_t sbase, uint32_t tmem, int t, int slot) {
-    const uint32_t qa = sbase + C::SMEM_Q + t * C::Q_TILE;
-    const uint32_t kb = sbase + C::SMEM_KV + slot * C::KV_TILE;
-    // Rolled loops: one MMA per 64+ tensor cycles leaves ample issue time, and keeps the
-    // control warpgroup's register needs small.
-#pragma unroll 1
+__device__ __forceinline__ void issue_qk(uint32_t sbase, uint32_t tmem, int t, int qbuf, int slot) {
+    // Descriptors are built once; k-slice kk of the 128-byte (64-byte) swizzled rows
+    // starts at a compile-time byte offset, added to the start-address field (the
+    // address stays below 256 KB, so the 14-bit field never carries).
+    const uint64_t a0 = sm100::opaque(sm100::smem_desc(sbase + C::SMEM_Q + (t * C::NQB + qbuf) * C::Q_TILE, 16, C::SBO, C::LAYOUT));
+    const uint64_t b0 = sm100::opaque(sm100::smem_desc(sbase + C::SMEM_KV + slot * C::KV_TILE, 16, C::SBO, C::LAYOUT));
+    const uint32_t d_tmem = tmem + uint32_t(t * C::BC);
+#pragma unroll
     for (int kk = 0; kk < C::D / 16; ++kk) {
-        const int ch = (kk * 16) / C::CW;
-        const uint32_t off = uint32_t((kk * 16) % C::CW) * 2u;
-        const uint64_t a = sm100::smem_desc(qa + ch * C::Q_CHUNK + off, 16, C::SBO, C::LAYOUT);
-        const uint64_t b = sm100::smem_desc(kb + ch * C::KV_CHUNK + off, 16, C::SBO, C::LAYOUT);
-        sm100::mma_bf16_ss(tmem + uint32_t(t * C::BC), a, b, C::IDESC_S, kk > 0 ? 1u : 0u);
+        constexpr int kCW = C::CW;
+        const uint32_t a_off = uint32_t(((kk * 16) / kCW) * C::Q_CHUNK + ((kk * 16) % kCW) * 2);
+        const uint32_t b_off = uint32_t(((kk * 16) / kCW) * C::KV_CHUNK + ((kk * 16) % kCW) * 2);
+        sm100::mma_bf16_ss_elected(d_tmem, a0 + (a_off >> 4), b0 + (b_off >> 4), C::IDESC_S, kk > 0 ? 1u : 0u);
     }
 }
 
 template <class C>
 __device__ __forceinline__ void issue_pv(uint32_t sbase, uint32_t tmem, int t, int slot, bool accumulate) {
-    const uint32_t vb = sbase + C::SMEM_KV + slot * C::KV_TILE;
-#pragma unroll 1
-    for (int kk = 0; kk < C::BC / 16; ++kk) {
-        // V tile is [BC rows x d] row-major: MN-major B operand; 16 key rows per MMA,
-        // 64-element column chunks C::KV_CHUNK bytes apart (leading byte offset).
-        const uint64_t b = sm100::smem_desc(vb + uint32_t(kk * 16 * C::RB), C::KV_CHUNK, C::SBO, C::LAYOUT);
-        const uint32_t a_tmem = tmem + uint32_t(t * C::BC + kk * 8);   // 16 bf16 = 8 columns
-        sm100::mma_bf16_ts(tmem + uint32_t(C::O_COL0 + t * C::OST), a_tmem, b, C::IDESC_O,
+    // V tile is [BC rows x d] row-major: MN-major B operand; 16 key rows per MMA,
+    // 64-element column chunks C::KV_CHUNK bytes apart (leading byte offset).  P is the
+    // A operand, read from TMEM (16 bf16 = 8 columns per MMA).
+    const uint64_t b0 = sm100::opaque(sm100::smem_desc(sbase + C::SMEM_KV + slot * C::KV_TILE, C::KV_CHUNK, C::SBO, C::LAYOUT));
+    const uint32_t a_tmem = tmem + uint32_t(t * C::BC);
+    const uint32_t d_tmem = tmem + uint32_t(C::O_COL0 + t * C::OST);
+#pragma unroll
+    for (int kk = 0; kk < C::BC / 16; ++kk)
+        sm100::mma_bf16_ts_elected(d_tmem, a_tmem + uint32_t(kk * 8), b0 + uint64_t((kk * 16 * C::RB) >> 4), C::IDESC_O,
                            (accumulate || kk > 0) ? 1u : 0u);
-    }
 }
 
 template <class C>
@@ -306,57 +322,63 @@ __device__ void mma_role(const FwdParams &p, uint32_t sbase, uint32_t tmem, cons
         if (w.nk_max == 0) continue;
         // prologue: S_t,0 for every tile that has work
         const int s_k0 = int(kv_cnt % C::NS);
-        if (!wait_bar(bar(C::B_FULL + s_k0), (kv_cnt / C::NS) & 1u, ctl, kSiteKvFull)) { ok = false; break; }
+        if (!warp_wait_bar<kRoleControl>(bar(C::B_FULL + s_k0), (kv_cnt / C::NS) & 1u, ctl, kSiteKvFull)) { ok = false; break; }
         ++kv_cnt;
+        int qbuf[2] = {0, 0};
 #pragma unroll
         for (int t = 0; t < C::NQT; ++t) {
             if (!ok || w.nk[t] == 0) continue;
-            if (!wait_bar(bar(C::B_QFULL + t), qcnt[t] & 1u, ctl, kSiteQFull)) { ok = false; break; }
+            qbuf[t] = int(qcnt[t] % C::NQB);
+            if (!warp_wait_bar<kRoleControl>(bar(C::B_QFULL + t * C::NQB + qbuf[t]), (qcnt[t] / C::NQB) & 1u, ctl, kSiteQFull)) {
+                ok = false;
+                break;
+            }
             ++qcnt[t];
             sm100::tc_fence_after_sync();
-            issue_qk<C>(sbase, tmem, t, s_k0);
-            sm100::tc_commit(bar(C::B_SFULL + t));
-            if (w.nk[t] == 1) sm100::tc_commit(bar(C::B_QEMPTY + t));
+            issue_qk<C>(sbase, tmem, t, qbuf[t], s_k0);
+            sm100::tc_commit_elected(bar(C::B_SFULL + t));
+            if (w.nk[t] == 1) sm100::tc_commit_elected(bar(C::B_QEMPTY + t * C::NQB + qbuf[t]));
         }
         if (!ok) break;
-        sm100::tc_commit(bar(C::B_EMPTY + s_k0));
+        sm100::tc_commit_elected(bar(C::B_EMPTY + s_k0));
         for (int j = 0; ok && j < w.nk_max; ++j) {
             const int s_v = int(kv_cnt % C::NS);
-            if (!wait_bar(bar(C::B_FULL + s_v), (kv_cnt / C::NS) & 1u, ctl, kSiteKvFull)) { ok = false; break; }
+            if (!warp_wait_bar<kRoleControl>(bar(C::B_FULL + s_v), (kv_cnt / C::NS) & 1u, ctl, kSiteKvFull)) { ok = false; break; }
             ++kv_cnt;
-            const bool has_next = j + 1 < w.nk_max;
             int s_k = 0;
-            if (has_next) {
-                s_k = int(kv_cnt % C::NS);
-                if (!wait_bar(bar(C::B_FULL + s_k), (kv_cnt / C::NS) & 1u, ctl, kSiteKvFull)) { ok = false; break; }
-                ++kv_cnt;
-            }
+            bool k_ready = false;                      // K_{j+1} waited for lazily, before the first S of j+1
 #pragma unroll
             for (int t = 0; t < C::NQT; ++t) {
                 if (!ok) break;
+                if (j + 1 < w.nk[t] && !k_ready) {
+                    s_k = int(kv_cnt % C::NS);
+                    if (!warp_wait_bar<kRoleControl>(bar(C::B_FULL + s_k), (kv_cnt / C::NS) & 1u, ctl, kSiteKvFull)) { ok = false; break; }
+                    ++kv_cnt;
+                    k_ready = true;
+                }
                 if (j < w.nk[t]) {
-                    if (!wait_bar(bar(C::B_PFULL + t), pcnt[t] & 1u, ctl, kSitePFull)) { ok = false; break; }
+                    if (!warp_wait_bar<kRoleControl>(bar(C::B_PFULL + t), pcnt[t] & 1u, ctl, kSitePFull)) { ok = false; break; }
                     ++pcnt[t];
                     if (j == 0 && u_local > 0 &&
-                        !wait_bar(bar(C::B_OEMPTY + t), (u_local - 1) & 1u, ctl, kSiteOEmpty)) { ok = false; break; }
+                        !warp_wait_bar<kRoleControl>(bar(C::B_OEMPTY + t), (u_local - 1) & 1u, ctl, kSiteOEmpty)) { ok = false; break; }
                     sm100::tc_fence_after_sync();
                     issue_pv<C>(sbase, tmem, t, s_v, j > 0);
-                    sm100::tc_commit(bar(C::B_ODONE + t));
+                    sm100::tc_commit_elected(bar(C::B_ODONE + t));
                 }
                 if (j + 1 < w.nk[t]) {
-                    issue_qk<C>(sbase, tmem, t, s_k);
-                    sm100::tc_commit(bar(C::B_SFULL + t));
-                    if (j + 2 == w.nk[t]) sm100::tc_commit(bar(C::B_QEMPTY + t));
+                    issue_qk<C>(sbase, tmem, t, qbuf[t], s_k);
+                    sm100::tc_commit_elected(bar(C::B_SFULL + t));
+                    if (j + 2 == w.nk[t]) sm100::tc_commit_elected(bar(C::B_QEMPTY + t * C::NQB + qbuf[t]));
                 }
             }
             if (!ok) break;
-            sm100::tc_commit(bar(C::B_EMPTY + s_v));
-            if (has_next) sm100::tc_commit(bar(C::B_EMPTY + s_k));
+            sm100::tc_commit_elected(bar(C::B_EMPTY + s_v));
+            if (k_ready) sm100::tc_commit_elected(bar(C::B_EMPTY + s_k));
         }
     }
     // Every MMA this thread issued is complete before the CTA may free TMEM.
-    sm100::tc_commit(bar(C::B_DRAIN));
-    wait_slow(bar(C::B_DRAIN), 0u, ctl, kSiteDrain, kWaitLimitNs, true);
+    sm100::tc_commit_elected(bar(C::B_DRAIN));
+    wait_slow<kRoleControl>(bar(C::B_DRAIN), 0u, ctl, kSiteDrain, kWaitLimitNs, true);
 }
 
 // ------------------------------------------------------------------ softmax / epilogue
@@ -372,19 +394,25 @@ __device__ void mma_role(const FwdParams &p, uint32_t sbase, uint32_t tmem, cons
 constexpr int kSoftExpPairsPer8 = FA_SOFT_EXP_PAIRS_PER_8;
 static_assert(kSoftExpPairsPer8 >= 0 && kSoftExpPairsPer8 <= 8, "share of software exponentials");
 
-template <int BC, bool MIXED>
+template <int BC, bool MIXED, bool TRACK_MAX>
 __device__ __forceinline__ float exp_pack_store(const uint32_t (&s)[BC], float c_log2, float neg_m,
-                                                uint32_t s_taddr) {
+                                                uint32_t s_taddr, float &raw_max) {
     const uint64_t c2 = sm100::pack2(c_log2, c_log2);
     const uint64_t nm2 = sm100::pack2(neg_m, neg_m);
     uint64_t acc0 = sm100::pack2(0.f, 0.f), acc1 = acc0;
+    float mx0 = -INFINITY, mx1 = -INFINITY;
 #pragma unroll
     for (int c = 0; c < BC / 64; ++c) {
         uint32_t pk[32];
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
             const int e = 64 * c + 2 * i;
-            const uint64_t x2 = sm100::fma2(sm100::pack2(__uint_as_float(s[e]), __uint_as_float(s[e + 1])), c2, nm2);
+            const float s0 = __uint_as_float(s[e]), s1 = __uint_as_float(s[e + 1]);
+            if (TRACK_MAX) {
+                if (i & 1) mx1 = sm100::max3(mx1, s0, s1);
+                else mx0 = sm100::max3(mx0, s0, s1);
+            }
+            const uint64_t x2 = sm100::fma2(sm100::pack2(s0, s1), c2, nm2);
             uint64_t p2;
             if (MIXED && (i % 8) >= 8 - kSoftExpPairsPer8) {
                 p2 = sm100::ex2_poly_pair(x2);
@@ -401,6 +429,7 @@ __device__ __forceinline__ float exp_pack_store(const uint32_t (&s)[BC], float c
         }
         sm100::tmem_st32(s_taddr + uint32_t(32 * c), pk);
     }
+    if (TRACK_MAX) raw_max = fmaxf(mx0, mx1);
     float a0, a1, b0, b1;
     sm100::unpack2(acc0, a0, a1);
     sm100::unpack2(acc1, b0, b1);
@@ -441,34 +470,51 @@ __device__ void softmax_role(const FwdParams &p, uint32_t sbase, uint32_t tmem, 
 
             const int k_lo = j * BC;
             const bool need_mask = (k_lo + BC > p.Nk) || (p.causal && k_lo + BC - 1 > q_lo + diag);
-            if (need_mask) {
-#pragma unroll
-                for (int i = 0; i < BC; ++i) {
-                    const int key = k_lo + i;
-                    if (key > row_lim || key >= p.Nk) s[i] = __float_as_uint(-INFINITY);
-                }
-            }
-            float mx0 = -INFINITY, mx1 = -INFINITY, mx2 = -INFINITY, mx3 = -INFINITY;
-#pragma unroll
-            for (int i = 0; i < BC; i += 8) {
-                mx0 = sm100::max3(mx0, __uint_as_float(s[i]), __uint_as_float(s[i + 1]));
-                mx1 = sm100::max3(mx1, __uint_as_float(s[i + 2]), __uint_as_float(s[i + 3]));
-                mx2 = sm100::max3(mx2, __uint_as_float(s[i + 4]), __uint_as_float(s[i + 5]));
-                mx3 = sm100::max3(mx3, __uint_as_float(s[i + 6]), __uint_as_float(s[i + 7]));
-            }
-            const float mx_s = sm100::max3(mx0, mx1, fmaxf(mx2, mx3)) * c_log2;
             float alpha = 1.f;
             bool need_rescale = false;
-            if (j == 0) {
-                m_ref = mx_s;
-            } else if (mx_s > m_ref + kRescaleLog2) {
-                alpha = sm100::ex2_approx(m_ref - mx_s);
-                m_ref = mx_s;
-                need_rescale = true;
+            float row_sum;
+            if (j > 0 && !need_mask) {
+                // Exponentiate at once against the current reference max, tracking this
+                // tile's max in the same pass; only if it rose by more than 2^8 (rare) is
+                // the tile redone against the new reference.
+                float mx = -INFINITY;
+                row_sum = exp_pack_store<BC, true, true>(s, c_log2, -m_ref, s_taddr, mx);
+                const float mx_s = mx * c_log2;
+                if (mx_s > m_ref + kRescaleLog2) {
+                    alpha = sm100::ex2_approx(m_ref - mx_s);
+                    m_ref = mx_s;
+                    need_rescale = true;
+                    row_sum = exp_pack_store<BC, true, false>(s, c_log2, -m_ref, s_taddr, mx);
+                }
+            } else {
+                if (need_mask) {
+#pragma unroll
+                    for (int i = 0; i < BC; ++i) {
+                        const int key = k_lo + i;
+                        if (key > row_lim || key >= p.Nk) s[i] = __float_as_uint(-INFINITY);
+                    }
+                }
+                float mx0 = -INFINITY, mx1 = -INFINITY, mx2 = -INFINITY, mx3 = -INFINITY;
+#pragma unroll
+                for (int i = 0; i < BC; i += 8) {
+                    mx0 = sm100::max3(mx0, __uint_as_float(s[i]), __uint_as_float(s[i + 1]));
+                    mx1 = sm100::max3(mx1, __uint_as_float(s[i + 2]), __uint_as_float(s[i + 3]));
+                    mx2 = sm100::max3(mx2, __uint_as_float(s[i + 4]), __uint_as_float(s[i + 5]));
+                    mx3 = sm100::max3(mx3, __uint_as_float(s[i + 6]), __uint_as_float(s[i + 7]));
+                }
+                const float mx_s = sm100::max3(mx0, mx1, fmaxf(mx2, mx3)) * c_log2;
+                if (j == 0) {
+                    m_ref = mx_s;
+                } else if (mx_s > m_ref + kRescaleLog2) {
+                    alpha = sm100::ex2_approx(m_ref - mx_s);
+                    m_ref = mx_s;
+                    need_rescale = true;
+                }
+                const float neg_m = (m_ref == -INFINITY) ? 0.f : -m_ref;
+                float unused;
+                row_sum = need_mask ? exp_pack_store<BC, false, false>(s, c_log2, neg_m, s_taddr, unused)
+                                    : exp_pack_store<BC, true, false>(s, c_log2, neg_m, s_taddr, unused);
             }
-            const float neg_m = (m_ref == -INFINITY) ? 0.f : -m_ref;
-            const float row_sum = need_mask ? exp_pack_store<BC, false>(s, c_log2, neg_m, s_taddr)
-                                            : exp_pack_store<BC, true>(s, c_log2, neg_m, s_taddr);
             l = l * alpha + row_sum;
 
             if (__any_sync(0xffffffffu, need_rescale)) {
@@ -555,9 +601,11 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             sm100::mbar_init(bar(C::B_FULL + s), 1);
             sm100::mbar_init(bar(C::B_EMPTY + s), 1);
         }
+        for (int i = 0; i < C::NQT * C::NQB; ++i) {
+            sm100::mbar_init(bar(C::B_QFULL + i), 1);
+            sm100::mbar_init(bar(C::B_QEMPTY + i), 1);
+        }
         for (int t = 0; t < C::NQT; ++t) {
-            sm100::mbar_init(bar(C::B_QFULL + t), 1);
-            sm100::mbar_init(bar(C::B_QEMPTY + t), 1);
             sm100::mbar_init(bar(C::B_SFULL + t), 1);
             sm100::mbar_init(bar(C::B_PFULL + t), 128);
             sm100::mbar_init(bar(C::B_ODONE + t), 1);
@@ -582,9 +630,9 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     } else {
         if constexpr (C::REALLOC_REGS) sm100::regs_decrease<C::CONTROL_REGS>();
         if (warp == C::TMA_WARP) {
-            if (lane == 0) producer_role<C>(&tm_q, &tm_k, &tm_v, p, sbase, ctl);
+            producer_role<C>(&tm_q, &tm_k, &tm_v, p, sbase, ctl);
         } else if (warp == C::MMA_WARP) {
-            if (lane == 0) mma_role<C>(p, sbase, tmem, ctl);
+            mma_role<C>(p, sbase, tmem, ctl);
         }
     }
     __syncwarp();
