@@ -480,10 +480,15 @@ __device__ void softmax_role(const FwdParams &p, uint32_t sbase, uint32_t tmem, 
                 float mx = -INFINITY;
                 row_sum = exp_pack_store<BC, true, true>(s, c_log2, -m_ref, s_taddr, mx);
                 const float mx_s = mx * c_log2;
-                if (mx_s > m_ref + kRescaleLog2) {
-                    alpha = sm100::ex2_approx(m_ref - mx_s);
-                    m_ref = mx_s;
-                    need_rescale = true;
+                const bool grew = mx_s > m_ref + kRescaleLog2;
+                // The redo stores to TMEM with warp-collective instructions, so the whole
+                // warp takes it together; rows whose max did not grow recompute the same P.
+                if (__any_sync(0xffffffffu, grew)) {
+                    if (grew) {
+                        alpha = sm100::ex2_approx(m_ref - mx_s);
+                        m_ref = mx_s;
+                        need_rescale = true;
+                    }
                     row_sum = exp_pack_store<BC, true, false>(s, c_log2, -m_ref, s_taddr, mx);
                 }
             } else {
