@@ -19,14 +19,18 @@ namespace {
 
 using namespace fa;
 
-// Tiling per head dim: TileCfg<d, key rows per tile, query tiles per unit, K/V slots>.
-using Cfg32 = TileCfg<32, 128, 2, 8, 2>;
-using Cfg64 = TileCfg<64, 128, 2, 8, 2>;
-using Cfg80 = TileCfg<80, 128, 2, 4>;
-using Cfg96 = TileCfg<96, 128, 2, 4>;
-using Cfg128 = TileCfg<128, 128, 2, 4>;
-using Cfg192 = TileCfg<192, 64, 2, 4>;
-using Cfg256 = TileCfg<256, 64, 1, 4>;
+// Tiling per head dim: TileCfg<d, key rows per tile, query tiles per unit, K/V slots,
+// buffers per Q tile, S buffers per Q tile, P in TMEM columns of its own, exponential
+// pairs per 8 on the FMA pipe>.  d = 256 runs one 128-row query tile, so it has TMEM room
+// for a second S buffer (S_{j+1} computed while the softmax works on S_j); d <= 64 has
+// room to keep P apart from S, and is where the exponentials dominate.
+using Cfg32 = TileCfg<32, 128, 2, 8, 2, 1, true, 2>;
+using Cfg64 = TileCfg<64, 128, 2, 8, 2, 1, true, 2>;
+using Cfg80 = TileCfg<80, 128, 2, 4, 1, 1>;
+using Cfg96 = TileCfg<96, 128, 2, 4, 1, 1>;
+using Cfg128 = TileCfg<128, 128, 2, 4, 1, 1>;
+using Cfg192 = TileCfg<192, 64, 2, 4, 1, 1>;
+using Cfg256 = TileCfg<256, 64, 1, 4, 1, 2>;
 
 __device__ int g_fa_status;   // per-device kernel status word (0 = OK)
 

@@ -42,7 +42,8 @@ constexpr int kStatusTimeout = 6;                     // = FA_ERR_DEVICE_TIMEOUT
 // Which wait gave up (bits 8..15 of the status word).
 enum WaitSite : int {
     kSiteQEmpty = 1, kSiteKvEmpty = 2, kSiteKvFull = 3, kSiteQFull = 4, kSitePFull = 5,
-    kSiteOEmpty = 6, kSiteSFull = 7, kSiteODone = 8, kSiteDrain = 9, kSiteProducerDrain = 10
+    kSiteOEmpty = 6, kSiteSFull = 7, kSiteODone = 8, kSiteDrain = 9, kSiteProducerDrain = 10,
+    kSitePvDone = 11, kSiteOFinal = 12
 };
 
 struct FwdParams {
@@ -58,13 +59,16 @@ struct FwdParams {
 };
 
 // Compile-time tiling for one head dimension.
-template <int D_, int BC_, int NQT_, int NS_, int NQB_ = 1>
+template <int D_, int BC_, int NQT_, int NS_, int NQB_ = 1, int SB_ = 1, bool PSEP_ = false, int SOFT_EXP_ = 0>
 struct TileCfg {
     static constexpr int D = D_;        // head dim
     static constexpr int BC = BC_;      // key/value rows per tile
     static constexpr int NQT = NQT_;    // query tiles per unit (1 or 2)
     static constexpr int NS = NS_;      // K/V slots in the ring
     static constexpr int NQB = NQB_;    // buffers per query tile (2: next unit's Q loads early)
+    static constexpr int SB = SB_;      // S buffers per query tile (2: S_{j+1} computed during softmax j)
+    static constexpr bool PSEP = PSEP_; // P in TMEM columns of its own instead of over S
+    static constexpr int SOFT_EXP = SOFT_EXP_;   // exponentials on the FMA pipe: pairs per 8
     static constexpr int CW = (D == 32) ? 32 : 64;       // elements per swizzled smem row
     static constexpr int RB = CW * 2;                     // bytes per swizzled row (64 or 128)
     static constexpr int NCH = (D + CW - 1) / CW;         // column chunks of a tile
@@ -74,16 +78,18 @@ struct TileCfg {
     static constexpr int KV_TILE = NCH * KV_CHUNK;
     static constexpr uint32_t LAYOUT = (RB == 128) ? 2u : 4u;   // UMMA 128B / 64B swizzle
     static constexpr int SBO = 8 * RB;                          // 8-row swizzle atom
-    // TMEM columns: S_t at t*BC (P_t reuses its first BC/2 columns), O_t after all S.
+    // TMEM columns: S buffer b of tile t at (t*SB + b)*BC, O_t after all S buffers, and
+    // P_t either over the first BC/2 columns of its S buffer or (PSEP) after all O.
     static constexpr int OST = (D == 256) ? 256 : ((D + 63) / 64) * 64;
-    static constexpr int O_COL0 = NQT * BC;
+    static constexpr int O_COL0 = NQT * SB * BC;
+    static constexpr int P_COL0 = O_COL0 + NQT * OST;
     static constexpr int TMEM_COLS = 512;
     static constexpr int O_CHUNKS = (D + 31) / 32;
     // shared memory (offsets from a 1024-byte aligned base)
     static constexpr int SMEM_Q = 0;
     static constexpr int SMEM_KV = NQT * NQB * Q_TILE;
     static constexpr int SMEM_BAR = SMEM_KV + NS * KV_TILE;
-    static constexpr int NUM_BARS = 2 * NS + 2 * NQT * NQB + 4 * NQT + 1;
+    static constexpr int NUM_BARS = 2 * NS + 2 * NQT * NQB + 3 * NQT * SB + 3 * NQT + 1;
     static constexpr int SMEM_MISC = SMEM_BAR + NUM_BARS * 8;
     // Each CTA holds all 512 TMEM columns, so ask for enough shared memory that a
     // second CTA can never be resident on the same SM (it would only wait in alloc).
@@ -111,14 +117,23 @@ struct TileCfg {
 
     static_assert(NQT == 1 || NQT == 2, "one or two query tiles per unit");
     static_assert(NQB == 1 || NQB == 2, "one or two buffers per query tile");
+    static_assert(SB == 1 || SB == 2, "one or two S buffers per query tile");
     static_assert(D % 16 == 0 && D >= 32 && D <= 256, "MMA N and K granularity");
     static_assert(BC % 64 == 0 && BC <= 256, "key tile: whole 32-column TMEM chunks of P");
-    static_assert(O_COL0 + NQT * OST <= TMEM_COLS, "TMEM budget");
+    static_assert(P_COL0 + (PSEP ? NQT * BC / 2 : 0) <= TMEM_COLS, "TMEM budget");
     static_assert(SMEM_BYTES <= 232448, "shared memory budget");
-    // barrier indices (query-tile barriers are indexed t * NQB + buffer)
+    // Barrier indices (Q barriers indexed t * NQB + buffer, S/P barriers t * SB + buffer).
+    // Every barrier is waited on densely (each completion in order) by its waiter, except
+    // O_DONE, whose rare waits provably trail it by at most one phase; parity waits
+    // cannot tell phases two apart.
     static constexpr int B_FULL = 0, B_EMPTY = NS, B_QFULL = 2 * NS, B_QEMPTY = 2 * NS + NQT * NQB,
-                         B_SFULL = 2 * NS + 2 * NQT * NQB, B_PFULL = B_SFULL + NQT,
-                         B_ODONE = B_PFULL + NQT, B_OEMPTY = B_ODONE + NQT, B_DRAIN = B_OEMPTY + NQT;
+                         B_SFULL = 2 * NS + 2 * NQT * NQB,   // S_t in buffer b computed
+                         B_PFULL = B_SFULL + NQT * SB,       // P_t written over buffer b
+                         B_PVDONE = B_PFULL + NQT * SB,      // the P V MMA reading buffer b done
+                         B_ODONE = B_PVDONE + NQT * SB,      // a P V MMA of tile t done (rescale)
+                         B_OFINAL = B_ODONE + NQT,           // the last P V of tile t in a unit done
+                         B_OEMPTY = B_OFINAL + NQT,          // epilogue finished reading O_t
+                         B_DRAIN = B_OEMPTY + NQT;
 };
 
 struct UnitInfo {
@@ -280,13 +295,13 @@ __device__ void producer_role(const CUtensorMap *tm_q, const CUtensorMap *tm_k, 
 // ------------------------------------------------------------------ MMA issuer
 
 template <class C>
-__device__ __forceinline__ void issue_qk(uint32_t sbase, uint32_t tmem, int t, int qbuf, int slot) {
+__device__ __forceinline__ void issue_qk(uint32_t sbase, uint32_t tmem, int t, int qbuf, int slot, int sbuf) {
     // Descriptors are built once; k-slice kk of the 128-byte (64-byte) swizzled rows
     // starts at a compile-time byte offset, added to the start-address field (the
     // address stays below 256 KB, so the 14-bit field never carries).
     const uint64_t a0 = sm100::opaque(sm100::smem_desc(sbase + C::SMEM_Q + (t * C::NQB + qbuf) * C::Q_TILE, 16, C::SBO, C::LAYOUT));
     const uint64_t b0 = sm100::opaque(sm100::smem_desc(sbase + C::SMEM_KV + slot * C::KV_TILE, 16, C::SBO, C::LAYOUT));
-    const uint32_t d_tmem = tmem + uint32_t(t * C::BC);
+    const uint32_t d_tmem = tmem + uint32_t((t * C::SB + sbuf) * C::BC);
 #pragma unroll
     for (int kk = 0; kk < C::D / 16; ++kk) {
         constexpr int kCW = C::CW;
@@ -297,12 +312,12 @@ __device__ __forceinline__ void issue_qk(uint32_t sbase, uint32_t tmem, int t, i
 }
 
 template <class C>
-__device__ __forceinline__ void issue_pv(uint32_t sbase, uint32_t tmem, int t, int slot, bool accumulate) {
+__device__ __forceinline__ void issue_pv(uint32_t sbase, uint32_t tmem, int t, int slot, int sbuf, bool accumulate) {
     // V tile is [BC rows x d] row-major: MN-major B operand; 16 key rows per MMA,
     // 64-element column chunks C::KV_CHUNK bytes apart (leading byte offset).  P is the
     // A operand, read from TMEM (16 bf16 = 8 columns per MMA).
     const uint64_t b0 = sm100::opaque(sm100::smem_desc(sbase + C::SMEM_KV + slot * C::KV_TILE, C::KV_CHUNK, C::SBO, C::LAYOUT));
-    const uint32_t a_tmem = tmem + uint32_t(t * C::BC);
+    const uint32_t a_tmem = tmem + uint32_t(C::PSEP ? C::P_COL0 + t * (C::BC / 2) : (t * C::SB + sbuf) * C::BC);
     const uint32_t d_tmem = tmem + uint32_t(C::O_COL0 + t * C::OST);
 #pragma unroll
     for (int kk = 0; kk < C::BC / 16; ++kk)
@@ -313,68 +328,130 @@ __device__ __forceinline__ void issue_pv(uint32_t sbase, uint32_t tmem, int t, i
 template <class C>
 __device__ void mma_role(const FwdParams &p, uint32_t sbase, uint32_t tmem, const Ctl &ctl) {
     auto bar = [&](int i) { return sbase + C::SMEM_BAR + 8u * uint32_t(i); };
-    uint32_t kv_cnt = 0;
-    uint32_t qcnt[2] = {0, 0}, pcnt[2] = {0, 0};
+    // K/V loads arrive in the order K_0, V_0, K_1, V_1, ...: load n sits in slot n % NS
+    // with phase (n / NS) & 1; kv_base is the first load index of the current unit.
+    uint32_t kv_base = 0;
+    uint32_t qcnt[2] = {0, 0};
+    uint32_t s_iss[2] = {0, 0};      // S tiles issued per query tile (S buffer = count % SB)
+    uint32_t p_got[2] = {0, 0};      // P tiles consumed per query tile (= P V MMAs issued)
     uint32_t u_local = 0;
     bool ok = true;
+    auto wait_load = [&](uint32_t n, int &slot) -> bool {
+        slot = int(n % C::NS);
+        return warp_wait_bar<kRoleControl>(bar(C::B_FULL + slot), (n / C::NS) & 1u, ctl, kSiteKvFull);
+    };
+    // An S MMA must not overwrite TMEM columns that an earlier P V MMA is still reading as
+    // its A operand (P lives in the S buffer it was computed from): the tensor core does
+    // not order one MMA's operand reads before a later MMA's accumulator writes.  S number
+    // n of a tile goes into buffer n % SB, which P V number n - SB read: wait for that one
+    // (each completion of the buffer's PVDONE barrier is waited for once, in order).
+    auto wait_buffer_free = [&](int t) -> bool {
+        const uint32_t n = s_iss[t];
+        // With P in columns of its own, S never overwrites an operand still being read;
+        // the softmax writes the next P only after the next S's commit, which completes
+        // after every earlier MMA of this thread (the previous P V included).
+        if (C::PSEP || n < uint32_t(C::SB)) return true;
+        const int b = int(n % C::SB);
+        return warp_wait_bar<kRoleControl>(bar(C::B_PVDONE + t * C::SB + b), ((n / C::SB) - 1u) & 1u, ctl,
+                                           kSitePvDone);
+    };
     for (int u = blockIdx.x; ok && u < p.num_units; u += gridDim.x, ++u_local) {
         const UnitInfo w = decode_unit<C>(u, p);
         if (w.nk_max == 0) continue;
-        // prologue: S_t,0 for every tile that has work
-        const int s_k0 = int(kv_cnt % C::NS);
-        if (!warp_wait_bar<kRoleControl>(bar(C::B_FULL + s_k0), (kv_cnt / C::NS) & 1u, ctl, kSiteKvFull)) { ok = false; break; }
-        ++kv_cnt;
         int qbuf[2] = {0, 0};
+        // S_t,j for query tile t, from the K tile in `slot`.
+        auto issue_s = [&](int t, int j, int slot) -> bool {
+            if (!wait_buffer_free(t)) return false;
+            sm100::tc_fence_after_sync();
+            const int sb = int(s_iss[t] % C::SB);
+            issue_qk<C>(sbase, tmem, t, qbuf[t], slot, sb);
+            sm100::tc_commit_elected(bar(C::B_SFULL + t * C::SB + sb));
+            ++s_iss[t];
+            if (j == w.nk[t] - 1) sm100::tc_commit_elected(bar(C::B_QEMPTY + t * C::NQB + qbuf[t]));
+            return true;
+        };
+        // O_t += P_t,j V_j from the V tile in `slot`.
+        auto issue_o = [&](int t, int j, int slot) -> bool {
+            const int sb = int(p_got[t] % C::SB);
+            if (!warp_wait_bar<kRoleControl>(bar(C::B_PFULL + t * C::SB + sb), (p_got[t] / C::SB) & 1u, ctl,
+                                             kSitePFull))
+                return false;
+            if (j == 0 && u_local > 0 &&
+                !warp_wait_bar<kRoleControl>(bar(C::B_OEMPTY + t), (u_local - 1) & 1u, ctl, kSiteOEmpty))
+                return false;
+            sm100::tc_fence_after_sync();
+            issue_pv<C>(sbase, tmem, t, slot, sb, j > 0);
+            sm100::tc_commit_elected(bar(C::B_ODONE + t));
+            if (!C::PSEP) sm100::tc_commit_elected(bar(C::B_PVDONE + t * C::SB + sb));
+            if (j == w.nk[t] - 1) sm100::tc_commit_elected(bar(C::B_OFINAL + t));
+            ++p_got[t];
+            return true;
+        };
+
+        // Q tiles of this unit
 #pragma unroll
         for (int t = 0; t < C::NQT; ++t) {
             if (!ok || w.nk[t] == 0) continue;
             qbuf[t] = int(qcnt[t] % C::NQB);
-            if (!warp_wait_bar<kRoleControl>(bar(C::B_QFULL + t * C::NQB + qbuf[t]), (qcnt[t] / C::NQB) & 1u, ctl, kSiteQFull)) {
+            if (!warp_wait_bar<kRoleControl>(bar(C::B_QFULL + t * C::NQB + qbuf[t]), (qcnt[t] / C::NQB) & 1u, ctl,
+                                             kSiteQFull))
                 ok = false;
-                break;
-            }
             ++qcnt[t];
-            sm100::tc_fence_after_sync();
-            issue_qk<C>(sbase, tmem, t, qbuf[t], s_k0);
-            sm100::tc_commit_elected(bar(C::B_SFULL + t));
-            if (w.nk[t] == 1) sm100::tc_commit_elected(bar(C::B_QEMPTY + t * C::NQB + qbuf[t]));
         }
         if (!ok) break;
-        sm100::tc_commit_elected(bar(C::B_EMPTY + s_k0));
-        for (int j = 0; ok && j < w.nk_max; ++j) {
-            const int s_v = int(kv_cnt % C::NS);
-            if (!warp_wait_bar<kRoleControl>(bar(C::B_FULL + s_v), (kv_cnt / C::NS) & 1u, ctl, kSiteKvFull)) { ok = false; break; }
-            ++kv_cnt;
-            int s_k = 0;
-            bool k_ready = false;                      // K_{j+1} waited for lazily, before the first S of j+1
+        sm100::tc_fence_after_sync();
+        int slot_k = 0, slot_v = 0;
+        // S for the first SB key tiles
+        for (int j = 0; ok && j < C::SB && j < w.nk_max; ++j) {
+            if (!wait_load(kv_base + 2u * j, slot_k)) { ok = false; break; }
 #pragma unroll
-            for (int t = 0; t < C::NQT; ++t) {
-                if (!ok) break;
-                if (j + 1 < w.nk[t] && !k_ready) {
-                    s_k = int(kv_cnt % C::NS);
-                    if (!warp_wait_bar<kRoleControl>(bar(C::B_FULL + s_k), (kv_cnt / C::NS) & 1u, ctl, kSiteKvFull)) { ok = false; break; }
-                    ++kv_cnt;
-                    k_ready = true;
-                }
-                if (j < w.nk[t]) {
-                    if (!warp_wait_bar<kRoleControl>(bar(C::B_PFULL + t), pcnt[t] & 1u, ctl, kSitePFull)) { ok = false; break; }
-                    ++pcnt[t];
-                    if (j == 0 && u_local > 0 &&
-                        !warp_wait_bar<kRoleControl>(bar(C::B_OEMPTY + t), (u_local - 1) & 1u, ctl, kSiteOEmpty)) { ok = false; break; }
-                    sm100::tc_fence_after_sync();
-                    issue_pv<C>(sbase, tmem, t, s_v, j > 0);
-                    sm100::tc_commit_elected(bar(C::B_ODONE + t));
-                }
-                if (j + 1 < w.nk[t]) {
-                    issue_qk<C>(sbase, tmem, t, qbuf[t], s_k);
-                    sm100::tc_commit_elected(bar(C::B_SFULL + t));
-                    if (j + 2 == w.nk[t]) sm100::tc_commit_elected(bar(C::B_QEMPTY + t * C::NQB + qbuf[t]));
-                }
-            }
-            if (!ok) break;
-            sm100::tc_commit_elected(bar(C::B_EMPTY + s_v));
-            if (k_ready) sm100::tc_commit_elected(bar(C::B_EMPTY + s_k));
+            for (int t = 0; t < C::NQT; ++t)
+                if (ok && j < w.nk[t] && !issue_s(t, j, slot_k)) ok = false;
+            sm100::tc_commit_elected(bar(C::B_EMPTY + slot_k));
         }
+        if (!ok) break;
+        for (int j = 0; ok && j < w.nk_max; ++j) {
+            if (!wait_load(kv_base + 2u * j + 1u, slot_v)) { ok = false; break; }
+            const int jn = j + C::SB;
+            bool k_ready = false;
+            if constexpr (C::SB == 2) {
+                // P V for both tiles first (keeps the tensor core busy while the S for key
+                // tile j + 2 waits for them), then S_{j+2}, which is not needed until the
+                // softmax has finished S_{j+1}.
+#pragma unroll
+                for (int t = 0; t < C::NQT; ++t)
+                    if (ok && j < w.nk[t] && !issue_o(t, j, slot_v)) ok = false;
+                if (!ok) break;
+                sm100::tc_commit_elected(bar(C::B_EMPTY + slot_v));
+                if (jn < w.nk_max) {
+                    if (!wait_load(kv_base + 2u * jn, slot_k)) { ok = false; break; }
+                    k_ready = true;
+#pragma unroll
+                    for (int t = 0; t < C::NQT; ++t)
+                        if (ok && jn < w.nk[t] && !issue_s(t, jn, slot_k)) ok = false;
+                    if (!ok) break;
+                }
+            } else {
+                // One S buffer: per tile, P V then (once it is done) the next S.
+#pragma unroll
+                for (int t = 0; t < C::NQT; ++t) {
+                    if (!ok) break;
+                    if (j < w.nk[t] && !issue_o(t, j, slot_v)) { ok = false; break; }
+                    if (jn < w.nk[t]) {
+                        if (!k_ready) {
+                            if (!wait_load(kv_base + 2u * jn, slot_k)) { ok = false; break; }
+                            k_ready = true;
+                        }
+                        if (!issue_s(t, jn, slot_k)) { ok = false; break; }
+                    }
+                }
+                if (!ok) break;
+                sm100::tc_commit_elected(bar(C::B_EMPTY + slot_v));
+            }
+            if (k_ready) sm100::tc_commit_elected(bar(C::B_EMPTY + slot_k));
+        }
+        if (!ok) break;
+        kv_base += 2u * uint32_t(w.nk_max);
     }
     // Every MMA this thread issued is complete before the CTA may free TMEM.
     sm100::tc_commit_elected(bar(C::B_DRAIN));
@@ -384,23 +461,17 @@ __device__ void mma_role(const FwdParams &p, uint32_t sbase, uint32_t tmem, cons
 // ------------------------------------------------------------------ softmax / epilogue
 
 // p = 2^(s * c_log2 - m) for one row of a score tile, packed to bf16 pairs and stored
-// over the first BC/2 TMEM columns of the tile (P overwrites S); returns the fp32 row
-// sum of p.  On unmasked tiles a share of the pairs (kSoftExpPairsPer8 of every 8) take
-// the FMA-pipe exponential so the special-function unit is not the bottleneck; masked
-// tiles (which may hold -inf scores) use the hardware ex2 throughout.
-#ifndef FA_SOFT_EXP_PAIRS_PER_8
-#define FA_SOFT_EXP_PAIRS_PER_8 2
-#endif
-constexpr int kSoftExpPairsPer8 = FA_SOFT_EXP_PAIRS_PER_8;
-static_assert(kSoftExpPairsPer8 >= 0 && kSoftExpPairsPer8 <= 8, "share of software exponentials");
-
-template <int BC, bool MIXED, bool TRACK_MAX>
+// to BC/2 TMEM columns at p_taddr (over the S tile itself, or P's own columns); returns
+// the fp32 row sum of p.  On unmasked tiles SOFT_EXP of every 8 pairs take the FMA-pipe
+// exponential to relieve the special-function unit (worth it where the exponentials
+// dominate, i.e. small head dims); masked tiles (which may hold -inf scores) use the
+// hardware ex2 throughout.
+template <int BC, int SOFT_EXP, bool MIXED>
 __device__ __forceinline__ float exp_pack_store(const uint32_t (&s)[BC], float c_log2, float neg_m,
-                                                uint32_t s_taddr, float &raw_max) {
+                                                uint32_t p_taddr) {
     const uint64_t c2 = sm100::pack2(c_log2, c_log2);
     const uint64_t nm2 = sm100::pack2(neg_m, neg_m);
     uint64_t acc0 = sm100::pack2(0.f, 0.f), acc1 = acc0;
-    float mx0 = -INFINITY, mx1 = -INFINITY;
 #pragma unroll
     for (int c = 0; c < BC / 64; ++c) {
         uint32_t pk[32];
@@ -408,13 +479,9 @@ __device__ __forceinline__ float exp_pack_store(const uint32_t (&s)[BC], float c
         for (int i = 0; i < 32; ++i) {
             const int e = 64 * c + 2 * i;
             const float s0 = __uint_as_float(s[e]), s1 = __uint_as_float(s[e + 1]);
-            if (TRACK_MAX) {
-                if (i & 1) mx1 = sm100::max3(mx1, s0, s1);
-                else mx0 = sm100::max3(mx0, s0, s1);
-            }
             const uint64_t x2 = sm100::fma2(sm100::pack2(s0, s1), c2, nm2);
             uint64_t p2;
-            if (MIXED && (i % 8) >= 8 - kSoftExpPairsPer8) {
+            if (MIXED && (i % 8) >= 8 - SOFT_EXP) {
                 p2 = sm100::ex2_poly_pair(x2);
             } else {
                 float a, b;
@@ -427,9 +494,8 @@ __device__ __forceinline__ float exp_pack_store(const uint32_t (&s)[BC], float c
             sm100::unpack2(p2, lo, hi);
             pk[i] = sm100::pack_bf16x2(lo, hi);
         }
-        sm100::tmem_st32(s_taddr + uint32_t(32 * c), pk);
+        sm100::tmem_st32(p_taddr + uint32_t(32 * c), pk);
     }
-    if (TRACK_MAX) raw_max = fmaxf(mx0, mx1);
     float a0, a1, b0, b1;
     sm100::unpack2(acc0, a0, a1);
     sm100::unpack2(acc1, b0, b1);
@@ -445,10 +511,11 @@ __device__ void softmax_role(const FwdParams &p, uint32_t sbase, uint32_t tmem, 
     const int quarter = warp % 4;                  // TMEM lanes 32*quarter .. +31
     const int row_in_tile = quarter * 32 + lane;
     const uint32_t lane_off = uint32_t(quarter * 32) << 16;
-    const uint32_t s_taddr = tmem + lane_off + uint32_t(t * BC);
+    const uint32_t s_taddr0 = tmem + lane_off + uint32_t(t * C::SB * BC);   // S buffer 0 of this tile
+    const uint32_t p_taddr_sep = tmem + lane_off + uint32_t(C::P_COL0 + t * (BC / 2));
     const uint32_t o_taddr = tmem + lane_off + uint32_t(C::O_COL0 + t * C::OST);
     const float c_log2 = p.scale_log2;
-    uint32_t scnt = 0, ocnt = 0;
+    uint32_t scnt = 0, ocnt = 0, ofin = 0;
 
     for (int u = blockIdx.x; u < p.num_units; u += gridDim.x) {
         const UnitInfo w = decode_unit<C>(u, p);
@@ -461,7 +528,10 @@ __device__ void softmax_role(const FwdParams &p, uint32_t sbase, uint32_t tmem, 
         float l = 0.f;                             // running sum of 2^(s*c - m_ref)
 
         for (int j = 0; j < nk; ++j) {
-            if (!warp_wait_bar(bar(C::B_SFULL + t), scnt & 1u, ctl, kSiteSFull)) goto unwind;
+            const int sb = int(scnt % C::SB);
+            const uint32_t s_taddr = s_taddr0 + uint32_t(sb * BC);
+            const uint32_t p_taddr = C::PSEP ? p_taddr_sep : s_taddr;
+            if (!warp_wait_bar(bar(C::B_SFULL + t * C::SB + sb), (scnt / C::SB) & 1u, ctl, kSiteSFull)) goto unwind;
             ++scnt;
             sm100::tc_fence_after_sync();
             uint32_t s[BC];
@@ -473,25 +543,7 @@ __device__ void softmax_role(const FwdParams &p, uint32_t sbase, uint32_t tmem, 
             float alpha = 1.f;
             bool need_rescale = false;
             float row_sum;
-            if (j > 0 && !need_mask) {
-                // Exponentiate at once against the current reference max, tracking this
-                // tile's max in the same pass; only if it rose by more than 2^8 (rare) is
-                // the tile redone against the new reference.
-                float mx = -INFINITY;
-                row_sum = exp_pack_store<BC, true, true>(s, c_log2, -m_ref, s_taddr, mx);
-                const float mx_s = mx * c_log2;
-                const bool grew = mx_s > m_ref + kRescaleLog2;
-                // The redo stores to TMEM with warp-collective instructions, so the whole
-                // warp takes it together; rows whose max did not grow recompute the same P.
-                if (__any_sync(0xffffffffu, grew)) {
-                    if (grew) {
-                        alpha = sm100::ex2_approx(m_ref - mx_s);
-                        m_ref = mx_s;
-                        need_rescale = true;
-                    }
-                    row_sum = exp_pack_store<BC, true, false>(s, c_log2, -m_ref, s_taddr, mx);
-                }
-            } else {
+            {
                 if (need_mask) {
 #pragma unroll
                     for (int i = 0; i < BC; ++i) {
@@ -499,15 +551,17 @@ __device__ void softmax_role(const FwdParams &p, uint32_t sbase, uint32_t tmem, 
                         if (key > row_lim || key >= p.Nk) s[i] = __float_as_uint(-INFINITY);
                     }
                 }
-                float mx0 = -INFINITY, mx1 = -INFINITY, mx2 = -INFINITY, mx3 = -INFINITY;
+                // Row max: eight independent 3-input-max chains, then a short tree, so
+                // the dependency depth stays small.
+                float mx[8];
 #pragma unroll
-                for (int i = 0; i < BC; i += 8) {
-                    mx0 = sm100::max3(mx0, __uint_as_float(s[i]), __uint_as_float(s[i + 1]));
-                    mx1 = sm100::max3(mx1, __uint_as_float(s[i + 2]), __uint_as_float(s[i + 3]));
-                    mx2 = sm100::max3(mx2, __uint_as_float(s[i + 4]), __uint_as_float(s[i + 5]));
-                    mx3 = sm100::max3(mx3, __uint_as_float(s[i + 6]), __uint_as_float(s[i + 7]));
-                }
-                const float mx_s = sm100::max3(mx0, mx1, fmaxf(mx2, mx3)) * c_log2;
+                for (int c = 0; c < 8; ++c) mx[c] = fmaxf(__uint_as_float(s[2 * c]), __uint_as_float(s[2 * c + 1]));
+#pragma unroll
+                for (int i = 16; i < BC; i += 16)
+#pragma unroll
+                    for (int c = 0; c < 8; ++c)
+                        mx[c] = sm100::max3(mx[c], __uint_as_float(s[i + 2 * c]), __uint_as_float(s[i + 2 * c + 1]));
+                const float mx_s = fmaxf(sm100::max3(mx[0], mx[1], mx[2]), sm100::max3(mx[3], mx[4], sm100::max3(mx[5], mx[6], mx[7]))) * c_log2;
                 if (j == 0) {
                     m_ref = mx_s;
                 } else if (mx_s > m_ref + kRescaleLog2) {
@@ -516,9 +570,8 @@ __device__ void softmax_role(const FwdParams &p, uint32_t sbase, uint32_t tmem, 
                     need_rescale = true;
                 }
                 const float neg_m = (m_ref == -INFINITY) ? 0.f : -m_ref;
-                float unused;
-                row_sum = need_mask ? exp_pack_store<BC, false, false>(s, c_log2, neg_m, s_taddr, unused)
-                                    : exp_pack_store<BC, true, false>(s, c_log2, neg_m, s_taddr, unused);
+                row_sum = need_mask ? exp_pack_store<BC, C::SOFT_EXP, false>(s, c_log2, neg_m, p_taddr)
+                                    : exp_pack_store<BC, C::SOFT_EXP, true>(s, c_log2, neg_m, p_taddr);
             }
             l = l * alpha + row_sum;
 
@@ -538,12 +591,13 @@ __device__ void softmax_role(const FwdParams &p, uint32_t sbase, uint32_t tmem, 
             }
             sm100::tmem_st_wait();
             sm100::tc_fence_before_sync();
-            sm100::mbar_arrive(bar(C::B_PFULL + t));
+            sm100::mbar_arrive(bar(C::B_PFULL + t * C::SB + sb));
         }
 
         // epilogue: O / l -> bf16 -> out, LSE -> lse
         if (nk > 0) {
-            if (!warp_wait_bar(bar(C::B_ODONE + t), (ocnt + uint32_t(nk) - 1u) & 1u, ctl, kSiteODone)) goto unwind;
+            if (!warp_wait_bar(bar(C::B_OFINAL + t), ofin & 1u, ctl, kSiteOFinal)) goto unwind;
+            ++ofin;
             sm100::tc_fence_after_sync();
         }
         ocnt += uint32_t(nk);
@@ -610,10 +664,14 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             sm100::mbar_init(bar(C::B_QFULL + i), 1);
             sm100::mbar_init(bar(C::B_QEMPTY + i), 1);
         }
+        for (int i = 0; i < C::NQT * C::SB; ++i) {
+            sm100::mbar_init(bar(C::B_SFULL + i), 1);
+            sm100::mbar_init(bar(C::B_PFULL + i), 128);
+            sm100::mbar_init(bar(C::B_PVDONE + i), 1);
+        }
         for (int t = 0; t < C::NQT; ++t) {
-            sm100::mbar_init(bar(C::B_SFULL + t), 1);
-            sm100::mbar_init(bar(C::B_PFULL + t), 128);
             sm100::mbar_init(bar(C::B_ODONE + t), 1);
+            sm100::mbar_init(bar(C::B_OFINAL + t), 1);
             sm100::mbar_init(bar(C::B_OEMPTY + t), 128);
         }
         sm100::mbar_init(bar(C::B_DRAIN), 1);
