@@ -17,8 +17,9 @@
  *    "where the memory black hole of standard attention comes from";
  *  - the softmax definition softmax(x_i) = e^{x_i} / sum_j e^{x_j}: same article,
  *    section "online softmax: keeping block-wise computation exact";
- *  - causal mask ("only see content before the current position") and no mask:
- *    same article, "performance tuning" item 3 (mask modes);
+ *  - causal mask ("only see content before the current position"), sliding-window mask
+ *    ("only look at the most recent positions") and no mask: same article,
+ *    "performance tuning" item 3 (mask modes);
  *  - GQA: query head h uses KV head floor(h / n_rep), n_rep = Hq / Hkv, i.e. the
  *    repeat_interleave(n_rep, dim=1) expansion of K and V: "Transformer efficient
  *    attention: Flash Attention vs GQA" (yunthe.com), section "GQA principle and
@@ -29,6 +30,8 @@
  * Readings where the pages are silent (each also listed in the design notes):
  *  - the causal mask keeps the diagonal (key j visible to query i iff j <= i) and,
  *    for Nq != Nk, is aligned to the bottom-right: j <= i + (Nk - Nq);
+ *  - the sliding window of W >= 1 keys is causal and ends at that diagonal:
+ *    i + (Nk - Nq) - W < j <= i + (Nk - Nq);
  *  - a row with no visible key (only possible when Nq > Nk under the causal mask,
  *    or Nk == 0) has O = 0 and LSE = -inf, the limit of an empty sum;
  *  - LSE is the natural-log log-sum-exp of the scaled, masked logits;
@@ -65,6 +68,7 @@ typedef struct {
     int B, Hq, Hkv, Nq, Nk, d;
     double scale;
     int causal;
+    int window;     /* 0: no window; W >= 1: sliding window of W keys (implies causal) */
 } problem_t;
 
 static int kv_head_of(const problem_t *p, int hq) {
@@ -76,11 +80,19 @@ static int kv_head_of(const problem_t *p, int hq) {
 }
 
 static int key_visible(const problem_t *p, int i, int j) {
-    if (!p->causal) return 1;
-#ifdef ORACLE_PLANT_CAUSAL_STRICT
-    return (long)j < (long)i + (long)(p->Nk - p->Nq);
+    const long diag = (long)i + (long)(p->Nk - p->Nq);   /* last key row i may see */
+    if (p->window > 0) {
+#ifdef ORACLE_PLANT_WINDOW_OFF_BY_ONE
+        if ((long)j < diag - p->window) return 0;
 #else
-    return (long)j <= (long)i + (long)(p->Nk - p->Nq);
+        if ((long)j <= diag - p->window) return 0;
+#endif
+    }
+    if (!p->causal && p->window == 0) return 1;
+#ifdef ORACLE_PLANT_CAUSAL_STRICT
+    return (long)j < diag;
+#else
+    return (long)j <= diag;
 #endif
 }
 
@@ -180,6 +192,7 @@ static void *head_rows_worker(void *arg) {
 static int check_problem(const problem_t *p) {
     if (p->B < 0 || p->Hq <= 0 || p->Hkv <= 0 || p->Nq < 0 || p->Nk < 0 || p->d <= 0) return 0;
     if (p->Hq % p->Hkv != 0) return 0;
+    if (p->window < 0) return 0;
     if (!isfinite(p->scale)) return 0;
     return 1;
 }
@@ -221,13 +234,14 @@ static int run_full(const problem_t *p, double *out, double *lse, double *probs,
 /*
  * oracle_attention_fwd: the whole forward.
  *   q [B,Nq,Hq,d], k/v [B,Nk,Hkv,d]: bf16 bit patterns (host memory).
+ *   causal in {0,1}; window = 0 (none) or W >= 1 keys (sliding window, causal).
  *   out [B,Nq,Hq,d] fp64, lse [B,Hq,Nq] fp64 (natural log).
  * Returns 0, or a negative code (bad sizes, no memory, thread failure).
  */
 int oracle_attention_fwd(const uint16_t *q, const uint16_t *k, const uint16_t *v,
                          double *out, double *lse, int B, int Hq, int Hkv, int Nq, int Nk,
-                         int d, double scale, int causal, int nthreads) {
-    problem_t p = {q, k, v, B, Hq, Hkv, Nq, Nk, d, scale, causal ? 1 : 0};
+                         int d, double scale, int causal, int window, int nthreads) {
+    problem_t p = {q, k, v, B, Hq, Hkv, Nq, Nk, d, scale, causal ? 1 : 0, window};
     return run_full(&p, out, lse, NULL, nthreads);
 }
 
@@ -237,8 +251,8 @@ int oracle_attention_fwd(const uint16_t *q, const uint16_t *k, const uint16_t *v
  */
 int oracle_attention_probs(const uint16_t *q, const uint16_t *k, const uint16_t *v,
                            double *out, double *lse, double *probs, int B, int Hq, int Hkv,
-                           int Nq, int Nk, int d, double scale, int causal) {
-    problem_t p = {q, k, v, B, Hq, Hkv, Nq, Nk, d, scale, causal ? 1 : 0};
+                           int Nq, int Nk, int d, double scale, int causal, int window) {
+    problem_t p = {q, k, v, B, Hq, Hkv, Nq, Nk, d, scale, causal ? 1 : 0, window};
     return run_full(&p, out, lse, probs, 1);
 }
 
@@ -273,8 +287,8 @@ static void *rows_worker(void *arg) {
 int oracle_attention_rows(const uint16_t *q, const uint16_t *k, const uint16_t *v,
                           const int32_t *rows, long nrows, double *out_rows, double *lse_rows,
                           int B, int Hq, int Hkv, int Nq, int Nk, int d, double scale,
-                          int causal, int nthreads) {
-    problem_t p = {q, k, v, B, Hq, Hkv, Nq, Nk, d, scale, causal ? 1 : 0};
+                          int causal, int window, int nthreads) {
+    problem_t p = {q, k, v, B, Hq, Hkv, Nq, Nk, d, scale, causal ? 1 : 0, window};
     if (!check_problem(&p) || nrows < 0) return ORACLE_EINVAL;
     for (long r = 0; r < nrows; ++r) {
         int b = rows[3 * r], hq = rows[3 * r + 1], i = rows[3 * r + 2];

@@ -35,14 +35,18 @@ def tiny_inputs(B, Hq, Hkv, Nq, Nk, d, seed, q_mult=1.0):
     return synth.make_inputs(w)
 
 
-def visible(i, j, Nq, Nk, causal):
-    """Causal reading: keep the diagonal, align bottom-right (j <= i + Nk - Nq)."""
-    return (not causal) or j <= i + (Nk - Nq)
+def visible(i, j, Nq, Nk, causal, window=0):
+    """Causal reading: keep the diagonal, align bottom-right (j <= i + Nk - Nq); a window
+    of W keys ends at that diagonal (i + Nk - Nq - W < j)."""
+    diag = i + (Nk - Nq)
+    if window and j <= diag - window:
+        return False
+    return (not causal and not window) or j <= diag
 
 
 # ---------------------------------------------------------------- brute force
 
-def brute_force_decimal(x, scale, causal, prec=40):
+def brute_force_decimal(x, scale, causal, prec=40, window=0):
     """O and LSE by the definition in `prec`-digit decimal arithmetic (tiny inputs)."""
     getcontext().prec = prec
     q, k, v = (bits_f64(x[n]) for n in ("q", "k", "v"))
@@ -63,7 +67,7 @@ def brute_force_decimal(x, scale, causal, prec=40):
                 num = [D(0)] * d
                 Z = D(0)
                 for j in range(Nk):
-                    if not visible(i, j, Nq, Nk, causal):
+                    if not visible(i, j, Nq, Nk, causal, window):
                         continue
                     s = sc * sum(qi[c] * kd[b][j][g][c] for c in range(d))
                     e = s.exp()
@@ -81,7 +85,7 @@ def brute_force_decimal(x, scale, causal, prec=40):
 
 # ---------------------------------------------------------------- second statement
 
-def online_softmax_blocks(x, scale, causal, block):
+def online_softmax_blocks(x, scale, causal, block, window=0):
     """The block-wise recurrence: running row max m, running sum l, output rescaled by
     exp(m_old - m_new) at every block, divided by l at the end (fp64)."""
     q, k, v = (bits_f64(x[n]) for n in ("q", "k", "v"))
@@ -102,9 +106,13 @@ def online_softmax_blocks(x, scale, causal, block):
                 Kb = k[b, j0:j0 + block, g, :]
                 Vb = v[b, j0:j0 + block, g, :]
                 s = scale * (Q @ Kb.T)
-                if causal:
+                if causal or window:
                     jj = np.arange(j0, j0 + Kb.shape[0])[None, :]
-                    s = np.where(jj <= ii + (Nk - Nq), s, -np.inf)
+                    diag = ii + (Nk - Nq)
+                    keep = jj <= diag
+                    if window:
+                        keep &= jj > diag - window
+                    s = np.where(keep, s, -np.inf)
                 m_new = np.maximum(m, s.max(axis=1))
                 safe = np.where(np.isfinite(m_new), m_new, 0.0)
                 corr = np.where(np.isfinite(m), np.exp(m - safe), 0.0)
@@ -290,3 +298,69 @@ ALL_PINS = [
     pin_zero_q, pin_causal_row0, pin_gqa_equals_repeated_mha, pin_key_permutation,
     pin_causal_prefix, pin_online_recurrence, pin_rows_match_full,
 ]
+
+
+# ---------------------------------------------------------------- sliding window
+
+WINDOW_CASES = [
+    # B, Hq, Hkv, Nq, Nk, d, window, seed
+    (1, 2, 1, 9, 9, 32, 3, 40),
+    (1, 2, 2, 6, 11, 64, 4, 41),      # Nq < Nk
+    (1, 1, 1, 10, 4, 16, 2, 42),      # Nq > Nk: early rows see nothing
+    (2, 4, 2, 7, 7, 80, 1, 43),
+]
+
+
+def pin_window_brute_force(orc):
+    for (B, Hq, Hkv, Nq, Nk, d, W, seed) in WINDOW_CASES:
+        x = tiny_inputs(B, Hq, Hkv, Nq, Nk, d, seed)
+        scale = 1.0 / math.sqrt(d)
+        O, L = orc.forward(x["q"], x["k"], x["v"], scale, True, window=W)
+        Ob, Lb = brute_force_decimal(x, scale, True, window=W)
+        assert_close(O, Ob, what=f"window O {W}")
+        assert_close(L, Lb, what=f"window LSE {W}")
+
+
+def pin_window_one_key(orc):
+    """W = 1: row i sees only key i + Nk - Nq: O = v, LSE = that single logit."""
+    x = tiny_inputs(1, 2, 2, 6, 8, 32, seed=44)
+    O, L = orc.forward(x["q"], x["k"], x["v"], 0.25, True, window=1)
+    q, k, v = (bits_f64(x[n]) for n in ("q", "k", "v"))
+    for i in range(6):
+        j = i + 2
+        for h in range(2):
+            assert_close(O[0, i, h], v[0, j, h], what="W=1 O")
+            assert_close(L[0, h, i], 0.25 * float(q[0, i, h] @ k[0, j, h]), what="W=1 LSE")
+
+
+def pin_window_wide_is_causal(orc):
+    x = tiny_inputs(1, 2, 1, 12, 12, 32, seed=45)
+    Oc, Lc = orc.forward(x["q"], x["k"], x["v"], 0.2, True)
+    Ow, Lw = orc.forward(x["q"], x["k"], x["v"], 0.2, True, window=12)
+    assert np.array_equal(Oc, Ow) and np.array_equal(Lc, Lw)
+
+
+def pin_window_row_is_segment(orc):
+    """Row i with window W equals unmasked attention of query i over keys i-W+1 .. i."""
+    x = tiny_inputs(1, 1, 1, 10, 10, 32, seed=46)
+    W = 4
+    O, L = orc.forward(x["q"], x["k"], x["v"], 0.3, True, window=W)
+    for i in (0, 2, 7, 9):
+        lo = max(0, i - W + 1)
+        Oi, Li = orc.forward(x["q"][:, i:i + 1], x["k"][:, lo:i + 1], x["v"][:, lo:i + 1], 0.3, False)
+        assert_close(O[0, i, 0], Oi[0, 0, 0], what="segment O")
+        assert_close(L[0, 0, i], Li[0, 0, 0], what="segment LSE")
+
+
+def pin_window_online_recurrence(orc):
+    x = tiny_inputs(1, 2, 1, 40, 40, 32, seed=47)
+    O, L = orc.forward(x["q"], x["k"], x["v"], 0.2, True, window=13)
+    for block in (1, 7, 16, 64):
+        Ob, Lb = online_softmax_blocks(x, 0.2, True, block, window=13)
+        assert_close(O, Ob, what="window online O")
+        assert_close(L, Lb, what="window online LSE")
+
+
+WINDOW_PINS = [pin_window_brute_force, pin_window_one_key, pin_window_wide_is_causal,
+               pin_window_row_is_segment, pin_window_online_recurrence]
+ALL_PINS = ALL_PINS + WINDOW_PINS
