@@ -233,7 +233,7 @@ def run_ours(args, w, world, rank, local):
     torch.cuda.synchronize()
 
     def step():
-        fa.fa_fwd(q, k, v, causal=w.causal, scale=w.scale, out=out, lse=lse)
+        fa.fa_fwd(q, k, v, causal=w.causal, scale=w.scale, out=out, lse=lse, window=w.window or None)
 
     for _ in range(args.warmup):
         step()
@@ -287,7 +287,7 @@ def run_ours(args, w, world, rank, local):
             q.copy_(host["q"], non_blocking=True)
             k.copy_(host["k"], non_blocking=True)
             v.copy_(host["v"], non_blocking=True)
-            fa.fa_fwd(q, k, v, causal=w.causal, scale=w.scale, out=out, lse=lse)
+            fa.fa_fwd(q, k, v, causal=w.causal, scale=w.scale, out=out, lse=lse, window=w.window or None)
             out_h.copy_(out, non_blocking=True)
             lse_h.copy_(lse, non_blocking=True)
 
@@ -347,13 +347,14 @@ def run_sweep(args):
         lse = torch.empty((w.B, w.Hq, w.Nq), dtype=torch.float32, device="cuda")
         # inputs smaller than L2 are timed both warm and with an L2 flush before each launch
         flush = torch.empty(int(2 * 126e6) // 4, dtype=torch.float32, device="cuda")
+        win = w.window or None
         for _ in range(args.warmup):
-            fa.fa_fwd(q, k, v, causal=w.causal, scale=w.scale, out=out, lse=lse)
+            fa.fa_fwd(q, k, v, causal=w.causal, scale=w.scale, out=out, lse=lse, window=win)
         torch.cuda.synchronize()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record()
         for _ in range(args.steps):
-            fa.fa_fwd(q, k, v, causal=w.causal, scale=w.scale, out=out, lse=lse)
+            fa.fa_fwd(q, k, v, causal=w.causal, scale=w.scale, out=out, lse=lse, window=win)
         e1.record()
         torch.cuda.synchronize()
         ms_warm = e0.elapsed_time(e1) / args.steps
@@ -362,7 +363,7 @@ def run_sweep(args):
             flush.zero_()
             a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             a.record()
-            fa.fa_fwd(q, k, v, causal=w.causal, scale=w.scale, out=out, lse=lse)
+            fa.fa_fwd(q, k, v, causal=w.causal, scale=w.scale, out=out, lse=lse, window=win)
             b.record()
             torch.cuda.synchronize()
             cold.append(a.elapsed_time(b))

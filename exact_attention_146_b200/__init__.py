@@ -27,7 +27,7 @@ FA_ERR_DEVICE_TIMEOUT = 6
 FA_ERR_NOT_DEVICE_MEMORY = 7
 FA_ERR_OVERLAP = 8
 
-EXPORTED = ("fa_fwd", "fa_status_string", "fa_device_status", "fa_tile_config", "fa_version")
+EXPORTED = ("fa_fwd", "fa_fwd_window", "fa_status_string", "fa_device_status", "fa_tile_config", "fa_version")
 
 
 class FaError(RuntimeError):
@@ -49,6 +49,8 @@ def lib() -> ctypes.CDLL:
         vp, ci, cf = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
         L.fa_fwd.argtypes = [vp, vp, vp, vp, vp, ci, ci, ci, ci, ci, ci, cf, ci, vp]
         L.fa_fwd.restype = ci
+        L.fa_fwd_window.argtypes = [vp, vp, vp, vp, vp, ci, ci, ci, ci, ci, ci, cf, ci, vp]
+        L.fa_fwd_window.restype = ci
         L.fa_status_string.argtypes = [ci]
         L.fa_status_string.restype = ctypes.c_char_p
         L.fa_device_status.argtypes = [vp, ctypes.POINTER(ci)]
@@ -88,13 +90,15 @@ def fa_fwd_raw(q_ptr, k_ptr, v_ptr, out_ptr, lse_ptr, B, Hq, Hkv, Nq, Nk, d, sca
 
 
 def fa_fwd(q, k, v, *, causal: bool = False, scale: float | None = None, out=None, lse=None,
-           return_lse: bool = True, stream=None):
+           return_lse: bool = True, stream=None, window: int | None = None):
     """Exact attention forward on [B, N, H, d] bf16 CUDA tensors.
 
     q: [B, Nq, Hq, d]; k, v: [B, Nk, Hkv, d] with Hq % Hkv == 0 (GQA: query head h
     uses KV head h // (Hq // Hkv)).  Returns (out [B, Nq, Hq, d] bf16, lse [B, Hq, Nq]
     fp32 natural-log log-sum-exp, or None if return_lse is False).  scale defaults to
-    1/sqrt(d).  Runs asynchronously on `stream` (default: torch's current stream)."""
+    1/sqrt(d).  window = W (>= 1) selects the sliding-window mask: row i sees the W keys
+    ending at its causal diagonal (fa_fwd_window).  Runs asynchronously on `stream`
+    (default: torch's current stream)."""
     import torch
     for name, t in (("q", q), ("k", k), ("v", v)):
         if t.dtype != torch.bfloat16 or not t.is_cuda or not t.is_contiguous() or t.dim() != 4:
@@ -111,9 +115,13 @@ def fa_fwd(q, k, v, *, causal: bool = False, scale: float | None = None, out=Non
         lse = torch.empty((B, Hq, Nq), dtype=torch.float32, device=q.device)
     if not return_lse:
         lse = None
-    rc = fa_fwd_raw(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
-                    lse.data_ptr() if lse is not None else None, B, Hq, Hkv, Nq, Nk, d, scale,
-                    1 if causal else 0, _stream_handle(stream))
+    lse_ptr = lse.data_ptr() if lse is not None else None
+    if window is not None:
+        rc = lib().fa_fwd_window(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse_ptr,
+                                 B, Hq, Hkv, Nq, Nk, d, float(scale), int(window), _stream_handle(stream))
+    else:
+        rc = fa_fwd_raw(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse_ptr,
+                        B, Hq, Hkv, Nq, Nk, d, scale, 1 if causal else 0, _stream_handle(stream))
     if rc != FA_OK:
         raise FaError(rc)
     return out, lse

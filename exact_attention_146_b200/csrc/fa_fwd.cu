@@ -156,6 +156,7 @@ struct Problem {
     int B, Hq, Hkv, Nq, Nk, d;
     float scale;
     int causal;
+    int window;
 };
 
 template <class C>
@@ -197,6 +198,7 @@ int launch(const Problem &pr, DeviceState &dev, int cfg_slot, cudaStream_t strea
     p.Nk = pr.Nk;
     p.n_rep = pr.Hq / pr.Hkv;
     p.causal = pr.causal;
+    p.window = pr.window;
     p.nqb = (pr.Nq + C::NQT * kBlockQ - 1) / (C::NQT * kBlockQ);
     const long long units = (long long)pr.B * pr.Hq * p.nqb;
     if (units > 0x7fffffffLL) return FA_ERR_INVALID_ARG;
@@ -257,12 +259,19 @@ int fa_tile_config(int d, int *block_q, int *block_k, int *q_tiles_per_unit, int
     return tile_config(d, block_q, block_k, q_tiles_per_unit, kv_slots);
 }
 
-int fa_fwd(const void *q, const void *k, const void *v, void *out, float *lse, int B, int Hq, int Hkv,
-           int Nq, int Nk, int d, float scale, int causal, void *stream) {
+}  // extern "C"
+
+namespace {
+
+// The shared forward: mask = none (causal 0, window 0), causal (1, 0) or sliding window
+// (1, W >= 1).
+int forward(const void *q, const void *k, const void *v, void *out, float *lse, int B, int Hq, int Hkv,
+            int Nq, int Nk, int d, float scale, int causal, int window, void *stream) {
     // ---- host-only validation (no CUDA call before this block passes)
     if (B < 0 || Hq <= 0 || Hkv <= 0 || Nq < 0 || Nk < 0) return FA_ERR_INVALID_ARG;
     if (Hq % Hkv != 0) return FA_ERR_INVALID_ARG;
     if (causal != 0 && causal != 1) return FA_ERR_INVALID_ARG;
+    if (window < 0 || (window > 0 && !causal)) return FA_ERR_INVALID_ARG;
     if (!std::isfinite(scale) || !(scale > 0.f)) return FA_ERR_INVALID_ARG;
     if (tile_config(d, nullptr, nullptr, nullptr, nullptr) != FA_OK) return FA_ERR_UNSUPPORTED_HEAD_DIM;
     const size_t q_bytes = size_t(B) * size_t(Nq) * size_t(Hq) * size_t(d) * 2;
@@ -302,7 +311,7 @@ int fa_fwd(const void *q, const void *k, const void *v, void *out, float *lse, i
         return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
     }
 
-    const Problem pr{q, k, v, out, lse, B, Hq, Hkv, Nq, Nk, d, scale, causal};
+    const Problem pr{q, k, v, out, lse, B, Hq, Hkv, Nq, Nk, d, scale, causal, window};
     switch (d) {
         case 32: return launch<Cfg32>(pr, *dev, 0, st);
         case 64: return launch<Cfg64>(pr, *dev, 1, st);
@@ -313,6 +322,21 @@ int fa_fwd(const void *q, const void *k, const void *v, void *out, float *lse, i
         case 256: return launch<Cfg256>(pr, *dev, 6, st);
         default: return FA_ERR_UNSUPPORTED_HEAD_DIM;
     }
+}
+
+}  // namespace
+
+extern "C" {
+
+int fa_fwd(const void *q, const void *k, const void *v, void *out, float *lse, int B, int Hq, int Hkv,
+           int Nq, int Nk, int d, float scale, int causal, void *stream) {
+    return forward(q, k, v, out, lse, B, Hq, Hkv, Nq, Nk, d, scale, causal, 0, stream);
+}
+
+int fa_fwd_window(const void *q, const void *k, const void *v, void *out, float *lse, int B, int Hq,
+                  int Hkv, int Nq, int Nk, int d, float scale, int window, void *stream) {
+    if (window < 1) return FA_ERR_INVALID_ARG;
+    return forward(q, k, v, out, lse, B, Hq, Hkv, Nq, Nk, d, scale, 1, window, stream);
 }
 
 int fa_device_status(void *stream, int *detail) {

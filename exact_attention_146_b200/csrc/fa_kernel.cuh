@@ -52,7 +52,8 @@ struct FwdParams {
     int *status;          // device status word
     int B, Hq, Hkv, Nq, Nk;
     int n_rep;            // Hq / Hkv
-    int causal;
+    int causal;           // 1 for the causal and the sliding-window masks
+    int window;           // 0, or the sliding-window width W (keys i+Nk-Nq-W < j <= i+Nk-Nq)
     int nqb;              // query blocks of NQT*128 rows per (b, hq)
     int num_units;        // B * Hq * nqb
     float scale_log2;     // scale * log2(e)
@@ -138,8 +139,8 @@ struct TileCfg {
 
 struct UnitInfo {
     int b, hq, kvh, q0;
-    int nk[2];     // key tiles each query tile visits
-    int nk_max;
+    int js[2], je[2];   // key tiles [js, je) each query tile visits (empty: js == je)
+    int j_lo, j_hi;     // union of the ranges: the K/V tiles the unit loads
 };
 
 // Static schedule shared by all roles.  Causal: longest query blocks first, heads of
@@ -163,23 +164,34 @@ __device__ __forceinline__ UnitInfo decode_unit(int u, const FwdParams &p) {
     w.kvh = w.hq / p.n_rep;
     w.q0 = qb * (C::NQT * kBlockQ);
     const int nkv = (p.Nk + C::BC - 1) / C::BC;
-    w.nk_max = 0;
+    const int diag = p.Nk - p.Nq;    // row i sees keys up to i + diag (causal / window)
+    w.j_lo = 0x7fffffff;
+    w.j_hi = 0;
 #pragma unroll
     for (int t = 0; t < 2; ++t) {
-        int n = 0;
+        int js = 0, je = 0;
         const int q_lo = w.q0 + t * kBlockQ;
         if (t < C::NQT && q_lo < p.Nq) {
-            if (!p.causal) {
-                n = nkv;
-            } else {
+            je = nkv;
+            if (p.causal) {
                 const int q_hi = min(q_lo + kBlockQ - 1, p.Nq - 1);
-                const int lim = q_hi + (p.Nk - p.Nq);   // last visible key of the tile's last row
-                n = lim < 0 ? 0 : min(nkv, lim / C::BC + 1);
+                const int lim = q_hi + diag;   // last visible key of the tile's last row
+                je = lim < 0 ? 0 : min(nkv, lim / C::BC + 1);
             }
+            if (p.window > 0) {
+                const int first = q_lo + diag - p.window + 1;   // first visible key of the first row
+                js = first <= 0 ? 0 : min(first / C::BC, nkv);
+            }
+            if (je <= js) js = je = 0;
         }
-        w.nk[t] = n;
-        w.nk_max = max(w.nk_max, n);
+        w.js[t] = js;
+        w.je[t] = je;
+        if (je > js) {
+            w.j_lo = min(w.j_lo, js);
+            w.j_hi = max(w.j_hi, je);
+        }
     }
+    if (w.j_hi == 0) w.j_lo = 0;
     return w;
 }
 
@@ -242,10 +254,10 @@ __device__ void producer_role(const CUtensorMap *tm_q, const CUtensorMap *tm_k, 
     bool ok = true;
     for (int u = blockIdx.x; ok && u < p.num_units; u += gridDim.x) {
         const UnitInfo w = decode_unit<C>(u, p);
-        if (w.nk_max == 0) continue;
+        if (w.j_hi == w.j_lo) continue;
 #pragma unroll
         for (int t = 0; t < C::NQT; ++t) {
-            if (!ok || w.nk[t] == 0) continue;
+            if (!ok || w.je[t] == w.js[t]) continue;
             const int qb = int(qcnt[t] % C::NQB);
             if (!warp_wait_bar<kRoleControl>(bar(C::B_QEMPTY + t * C::NQB + qb), ((qcnt[t] / C::NQB) & 1u) ^ 1u, ctl, kSiteQEmpty)) {
                 ok = false;
@@ -259,7 +271,7 @@ __device__ void producer_role(const CUtensorMap *tm_q, const CUtensorMap *tm_k, 
             for (int c = 0; c < C::NCH; ++c)
                 sm100::tma_load_4d_elected(dst + c * C::Q_CHUNK, tm_q, fb, c * C::CW, w.hq, w.q0 + t * kBlockQ, w.b);
         }
-        for (int j = 0; ok && j < w.nk_max; ++j) {
+        for (int j = w.j_lo; ok && j < w.j_hi; ++j) {
 #pragma unroll
             for (int which = 0; which < 2; ++which) {
                 const int s = int(kv_cnt % C::NS);
@@ -357,8 +369,9 @@ __device__ void mma_role(const FwdParams &p, uint32_t sbase, uint32_t tmem, cons
     };
     for (int u = blockIdx.x; ok && u < p.num_units; u += gridDim.x, ++u_local) {
         const UnitInfo w = decode_unit<C>(u, p);
-        if (w.nk_max == 0) continue;
+        if (w.j_hi == w.j_lo) continue;
         int qbuf[2] = {0, 0};
+        auto visits = [&](int t, int j) { return w.js[t] <= j && j < w.je[t]; };
         // S_t,j for query tile t, from the K tile in `slot`.
         auto issue_s = [&](int t, int j, int slot) -> bool {
             if (!wait_buffer_free(t)) return false;
@@ -367,7 +380,7 @@ __device__ void mma_role(const FwdParams &p, uint32_t sbase, uint32_t tmem, cons
             issue_qk<C>(sbase, tmem, t, qbuf[t], slot, sb);
             sm100::tc_commit_elected(bar(C::B_SFULL + t * C::SB + sb));
             ++s_iss[t];
-            if (j == w.nk[t] - 1) sm100::tc_commit_elected(bar(C::B_QEMPTY + t * C::NQB + qbuf[t]));
+            if (j == w.je[t] - 1) sm100::tc_commit_elected(bar(C::B_QEMPTY + t * C::NQB + qbuf[t]));
             return true;
         };
         // O_t += P_t,j V_j from the V tile in `slot`.
@@ -376,14 +389,14 @@ __device__ void mma_role(const FwdParams &p, uint32_t sbase, uint32_t tmem, cons
             if (!warp_wait_bar<kRoleControl>(bar(C::B_PFULL + t * C::SB + sb), (p_got[t] / C::SB) & 1u, ctl,
                                              kSitePFull))
                 return false;
-            if (j == 0 && u_local > 0 &&
+            if (j == w.js[t] && u_local > 0 &&
                 !warp_wait_bar<kRoleControl>(bar(C::B_OEMPTY + t), (u_local - 1) & 1u, ctl, kSiteOEmpty))
                 return false;
             sm100::tc_fence_after_sync();
-            issue_pv<C>(sbase, tmem, t, slot, sb, j > 0);
+            issue_pv<C>(sbase, tmem, t, slot, sb, j > w.js[t]);
             sm100::tc_commit_elected(bar(C::B_ODONE + t));
             if (!C::PSEP) sm100::tc_commit_elected(bar(C::B_PVDONE + t * C::SB + sb));
-            if (j == w.nk[t] - 1) sm100::tc_commit_elected(bar(C::B_OFINAL + t));
+            if (j == w.je[t] - 1) sm100::tc_commit_elected(bar(C::B_OFINAL + t));
             ++p_got[t];
             return true;
         };
@@ -391,7 +404,7 @@ __device__ void mma_role(const FwdParams &p, uint32_t sbase, uint32_t tmem, cons
         // Q tiles of this unit
 #pragma unroll
         for (int t = 0; t < C::NQT; ++t) {
-            if (!ok || w.nk[t] == 0) continue;
+            if (!ok || w.je[t] == w.js[t]) continue;
             qbuf[t] = int(qcnt[t] % C::NQB);
             if (!warp_wait_bar<kRoleControl>(bar(C::B_QFULL + t * C::NQB + qbuf[t]), (qcnt[t] / C::NQB) & 1u, ctl,
                                              kSiteQFull))
@@ -401,17 +414,17 @@ __device__ void mma_role(const FwdParams &p, uint32_t sbase, uint32_t tmem, cons
         if (!ok) break;
         sm100::tc_fence_after_sync();
         int slot_k = 0, slot_v = 0;
-        // S for the first SB key tiles
-        for (int j = 0; ok && j < C::SB && j < w.nk_max; ++j) {
-            if (!wait_load(kv_base + 2u * j, slot_k)) { ok = false; break; }
+        // S for the first SB key tiles (K/V tile j is load pair j - j_lo of the unit)
+        for (int j = w.j_lo; ok && j < w.j_lo + C::SB && j < w.j_hi; ++j) {
+            if (!wait_load(kv_base + 2u * (j - w.j_lo), slot_k)) { ok = false; break; }
 #pragma unroll
             for (int t = 0; t < C::NQT; ++t)
-                if (ok && j < w.nk[t] && !issue_s(t, j, slot_k)) ok = false;
+                if (ok && visits(t, j) && !issue_s(t, j, slot_k)) ok = false;
             sm100::tc_commit_elected(bar(C::B_EMPTY + slot_k));
         }
         if (!ok) break;
-        for (int j = 0; ok && j < w.nk_max; ++j) {
-            if (!wait_load(kv_base + 2u * j + 1u, slot_v)) { ok = false; break; }
+        for (int j = w.j_lo; ok && j < w.j_hi; ++j) {
+            if (!wait_load(kv_base + 2u * (j - w.j_lo) + 1u, slot_v)) { ok = false; break; }
             const int jn = j + C::SB;
             bool k_ready = false;
             if constexpr (C::SB == 2) {
@@ -420,15 +433,15 @@ __device__ void mma_role(const FwdParams &p, uint32_t sbase, uint32_t tmem, cons
                 // softmax has finished S_{j+1}.
 #pragma unroll
                 for (int t = 0; t < C::NQT; ++t)
-                    if (ok && j < w.nk[t] && !issue_o(t, j, slot_v)) ok = false;
+                    if (ok && visits(t, j) && !issue_o(t, j, slot_v)) ok = false;
                 if (!ok) break;
                 sm100::tc_commit_elected(bar(C::B_EMPTY + slot_v));
-                if (jn < w.nk_max) {
-                    if (!wait_load(kv_base + 2u * jn, slot_k)) { ok = false; break; }
+                if (jn < w.j_hi) {
+                    if (!wait_load(kv_base + 2u * (jn - w.j_lo), slot_k)) { ok = false; break; }
                     k_ready = true;
 #pragma unroll
                     for (int t = 0; t < C::NQT; ++t)
-                        if (ok && jn < w.nk[t] && !issue_s(t, jn, slot_k)) ok = false;
+                        if (ok && visits(t, jn) && !issue_s(t, jn, slot_k)) ok = false;
                     if (!ok) break;
                 }
             } else {
@@ -436,10 +449,10 @@ __device__ void mma_role(const FwdParams &p, uint32_t sbase, uint32_t tmem, cons
 #pragma unroll
                 for (int t = 0; t < C::NQT; ++t) {
                     if (!ok) break;
-                    if (j < w.nk[t] && !issue_o(t, j, slot_v)) { ok = false; break; }
-                    if (jn < w.nk[t]) {
+                    if (visits(t, j) && !issue_o(t, j, slot_v)) { ok = false; break; }
+                    if (visits(t, jn)) {
                         if (!k_ready) {
-                            if (!wait_load(kv_base + 2u * jn, slot_k)) { ok = false; break; }
+                            if (!wait_load(kv_base + 2u * (jn - w.j_lo), slot_k)) { ok = false; break; }
                             k_ready = true;
                         }
                         if (!issue_s(t, jn, slot_k)) { ok = false; break; }
@@ -451,7 +464,7 @@ __device__ void mma_role(const FwdParams &p, uint32_t sbase, uint32_t tmem, cons
             if (k_ready) sm100::tc_commit_elected(bar(C::B_EMPTY + slot_k));
         }
         if (!ok) break;
-        kv_base += 2u * uint32_t(w.nk_max);
+        kv_base += 2u * uint32_t(w.j_hi - w.j_lo);
     }
     // Every MMA this thread issued is complete before the CTA may free TMEM.
     sm100::tc_commit_elected(bar(C::B_DRAIN));
@@ -519,15 +532,19 @@ __device__ void softmax_role(const FwdParams &p, uint32_t sbase, uint32_t tmem, 
 
     for (int u = blockIdx.x; u < p.num_units; u += gridDim.x) {
         const UnitInfo w = decode_unit<C>(u, p);
-        const int nk = w.nk[t];
+        const int js = w.js[t], je = w.je[t];
+        const int nk = je - js;
         const int q_lo = w.q0 + t * kBlockQ;
         const int row = q_lo + row_in_tile;
         const int diag = p.Nk - p.Nq;              // causal: key j visible to row i iff j <= i + diag
         const int row_lim = p.causal ? row + diag : 0x7fffffff;
+        // sliding window: keys j > i + diag - W; the tile's first row has the lowest bound
+        const int row_lo = p.window > 0 ? row + diag - p.window + 1 : -0x7fffffff;
+        const int tile_lo_hi = p.window > 0 ? q_lo + kBlockQ - 1 + diag - p.window + 1 : -0x7fffffff;
         float m_ref = -INFINITY;                   // reference max, log2 units (scaled)
         float l = 0.f;                             // running sum of 2^(s*c - m_ref)
 
-        for (int j = 0; j < nk; ++j) {
+        for (int j = js; j < je; ++j) {
             const int sb = int(scnt % C::SB);
             const uint32_t s_taddr = s_taddr0 + uint32_t(sb * BC);
             const uint32_t p_taddr = C::PSEP ? p_taddr_sep : s_taddr;
@@ -539,7 +556,9 @@ __device__ void softmax_role(const FwdParams &p, uint32_t sbase, uint32_t tmem, 
             else sm100::tmem_ld64_sync(s_taddr, s);
 
             const int k_lo = j * BC;
-            const bool need_mask = (k_lo + BC > p.Nk) || (p.causal && k_lo + BC - 1 > q_lo + diag);
+            // boundary tiles: the key tail, the causal diagonal, the window's lower edge
+            const bool need_mask = (k_lo + BC > p.Nk) || (p.causal && k_lo + BC - 1 > q_lo + diag) ||
+                                   (k_lo < tile_lo_hi);
             float alpha = 1.f;
             bool need_rescale = false;
             float row_sum;
@@ -548,7 +567,7 @@ __device__ void softmax_role(const FwdParams &p, uint32_t sbase, uint32_t tmem, 
 #pragma unroll
                     for (int i = 0; i < BC; ++i) {
                         const int key = k_lo + i;
-                        if (key > row_lim || key >= p.Nk) s[i] = __float_as_uint(-INFINITY);
+                        if (key > row_lim || key >= p.Nk || key < row_lo) s[i] = __float_as_uint(-INFINITY);
                     }
                 }
                 // Row max: eight independent 3-input-max chains, then a short tree, so
@@ -562,7 +581,7 @@ __device__ void softmax_role(const FwdParams &p, uint32_t sbase, uint32_t tmem, 
                     for (int c = 0; c < 8; ++c)
                         mx[c] = sm100::max3(mx[c], __uint_as_float(s[i + 2 * c]), __uint_as_float(s[i + 2 * c + 1]));
                 const float mx_s = fmaxf(sm100::max3(mx[0], mx[1], mx[2]), sm100::max3(mx[3], mx[4], sm100::max3(mx[5], mx[6], mx[7]))) * c_log2;
-                if (j == 0) {
+                if (j == js) {
                     m_ref = mx_s;
                 } else if (mx_s > m_ref + kRescaleLog2) {
                     alpha = sm100::ex2_approx(m_ref - mx_s);
@@ -578,7 +597,7 @@ __device__ void softmax_role(const FwdParams &p, uint32_t sbase, uint32_t tmem, 
             if (__any_sync(0xffffffffu, need_rescale)) {
                 // O_t holds the sum up to block j-1 at the old reference; wait for that
                 // MMA, then scale this warp's rows by alpha (1 where the max held).
-                if (!warp_wait_bar(bar(C::B_ODONE + t), (ocnt + uint32_t(j) - 1u) & 1u, ctl, kSiteODone)) goto unwind;
+                if (!warp_wait_bar(bar(C::B_ODONE + t), (ocnt + uint32_t(j - js) - 1u) & 1u, ctl, kSiteODone)) goto unwind;
                 sm100::tc_fence_after_sync();
 #pragma unroll
                 for (int c = 0; c < C::O_CHUNKS; ++c) {

@@ -74,6 +74,22 @@ int fa_fwd(const void *q, const void *k, const void *v, void *out, float *lse,
            int B, int Hq, int Hkv, int Nq, int Nk, int d, float scale, int causal,
            void *stream);
 
+/*
+ * fa_fwd_window -- exact attention forward with a sliding-window (local) causal mask:
+ * query row i sees the `window` keys ending at its causal diagonal,
+ *
+ *     i + (Nk - Nq) - window < j <= i + (Nk - Nq),
+ *
+ * the third mask mode of the hwcomputing.csdn.net FlashAttention article ("performance
+ * tuning", item 3: only the most recent positions, for long texts).  Arguments, layouts,
+ * ownership and errors as fa_fwd, with window >= 1 (FA_ERR_INVALID_ARG otherwise); a
+ * window of at least Nk keys is the causal mask.  Key tiles wholly outside a query tile's
+ * window are not visited.
+ */
+int fa_fwd_window(const void *q, const void *k, const void *v, void *out, float *lse,
+                  int B, int Hq, int Hkv, int Nq, int Nk, int d, float scale, int window,
+                  void *stream);
+
 /* Human-readable text of a status code (static storage; never NULL). */
 const char *fa_status_string(int status);
 

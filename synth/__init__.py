@@ -116,6 +116,7 @@ class Workload:
     q_mult: float = 1.0      # exact power-of-two multiplier applied to the bf16 Q values
     k_mult: float = 1.0      # same for K
     seed: int = 0
+    window: int = 0          # sliding window of W keys (0: none; implies causal)
 
     @property
     def scale(self) -> float:
@@ -123,7 +124,13 @@ class Workload:
 
     @property
     def flops(self) -> float:
-        """4*B*Hq*Nq*Nk*d, halved when causal (the throughput convention used here)."""
+        """4*B*Hq*Nq*Nk*d, halved when causal (the throughput convention used here); with a
+        sliding window of W keys, 4*B*Hq*d times the number of visible (query, key) pairs."""
+        if self.window:
+            off = self.Nk - self.Nq
+            pairs = sum(max(0, min(i + off + 1, self.Nk) - max(0, i + off - self.window + 1))
+                        for i in range(self.Nq))
+            return 4.0 * self.B * self.Hq * self.d * pairs
         f = 4.0 * self.B * self.Hq * self.Nq * self.Nk * self.d
         return f / 2 if self.causal else f
 
@@ -176,6 +183,7 @@ for _w in [
     _wl("hdim96_b2_n4096_h16", 14, 2, 16, 4096, 96),
     _wl("hdim192_b2_n4096_h16", 15, 2, 16, 4096, 192),
     _wl("hdim256_b2_n4096_h16", 16, 2, 16, 4096, 256),
+    _wl("window4k_long16k_b1_h32_d128", 17, 1, 32, 16384, 128, causal=True, window=4096),
 ]:
     WORKLOADS[_w.name] = _w
 

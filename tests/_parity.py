@@ -24,7 +24,7 @@ def bf16_to_f64(t):
     return t.float().cpu().numpy().astype(np.float64)
 
 
-def run_cuda(x, scale, causal, with_lse=True, canary=True):
+def run_cuda(x, scale, causal, with_lse=True, canary=True, window=None):
     """fa_fwd through the C ABI; out/lse pre-filled with NaN so unwritten rows show up."""
     import torch
     import exact_attention_146_b200 as fa
@@ -32,7 +32,7 @@ def run_cuda(x, scale, causal, with_lse=True, canary=True):
     out = torch.full_like(q, float("nan")) if canary else torch.empty_like(q)
     B, Nq, Hq, d = q.shape
     lse = torch.full((B, Hq, Nq), float("nan"), dtype=torch.float32, device="cuda") if with_lse else None
-    fa.fa_fwd(q, k, v, causal=causal, scale=scale, out=out, lse=lse, return_lse=with_lse)
+    fa.fa_fwd(q, k, v, causal=causal, scale=scale, out=out, lse=lse, return_lse=with_lse, window=window)
     st, word = fa.device_status()
     assert st == fa.FA_OK, f"device status {st} (word {word:#x})"
     torch.cuda.synchronize()

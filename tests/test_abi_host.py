@@ -90,6 +90,12 @@ def test_validation_rejects(L, kw, code):
     assert call(L, **kw) == code
 
 
+@pytest.mark.parametrize("window", [0, -1, -100])
+def test_window_must_be_positive(L, window):
+    assert L.fa_fwd_window(FAKE, FAKE + (1 << 30), FAKE + (2 << 30), FAKE + (3 << 30), None,
+                           1, 2, 1, 16, 16, 64, 0.125, window, None) == fa.FA_ERR_INVALID_ARG
+
+
 def test_empty_problems_are_noops(L):
     # no output rows: nothing to validate against the device, nothing launched
     assert call(L, B=0, q=None, k=None, v=None, out=None, lse=None) == fa.FA_OK

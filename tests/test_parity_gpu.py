@@ -93,6 +93,24 @@ def test_increasing_logits_force_rescales(orc):
     check_full(orc, x, 1.0 / math.sqrt(128), True, "ramp causal")
 
 
+@pytest.mark.parametrize("d", [64, 128, 256])
+@pytest.mark.parametrize("N", [129, 300, 700])
+@pytest.mark.parametrize("W", [1, 17, 128, 129, 250, 1000])
+def test_sliding_window(orc, d, N, W):
+    x = tiny(1, 2, 1, N, N, d, seed=N + W + d)
+    O, L = _parity.run_cuda(x, 1.0 / math.sqrt(d), True, window=W)
+    Oref, Lref = orc.forward(x["q"], x["k"], x["v"], 1.0 / math.sqrt(d), True, window=W)
+    _parity.compare(O, L, Oref, Lref, f"window d={d} N={N} W={W}")
+
+
+@pytest.mark.parametrize("Nq,Nk,W", [(100, 300, 64), (300, 100, 40), (257, 700, 300), (1, 500, 130)])
+def test_sliding_window_unequal_lengths(orc, Nq, Nk, W):
+    x = tiny(2, 4, 2, Nq, Nk, 64, seed=Nq + Nk + W)
+    O, L = _parity.run_cuda(x, 0.125, True, window=W)
+    Oref, Lref = orc.forward(x["q"], x["k"], x["v"], 0.125, True, window=W)
+    _parity.compare(O, L, Oref, Lref, f"window Nq={Nq} Nk={Nk} W={W}")
+
+
 def test_lse_optional(orc):
     x = tiny(1, 2, 1, 200, 200, 64, seed=80)
     O, L = _parity.run_cuda(x, 0.125, True, with_lse=False)
@@ -194,10 +212,10 @@ def test_workload_sampled_rows(orc, name):
     oracle one by one, and every output row checked to be written and finite."""
     w = synth.WORKLOADS[name]
     x = synth.make_inputs(w)
-    O, L = _parity.run_cuda(x, w.scale, w.causal)
+    O, L = _parity.run_cuda(x, w.scale, w.causal, window=w.window or None)
     assert np.isfinite(O).all() and np.isfinite(L).all()
     rows = _parity.sample_rows(w, 192, seed=w.wid)
-    Oref, Lref = orc.rows(x["q"], x["k"], x["v"], rows, w.scale, w.causal)
+    Oref, Lref = orc.rows(x["q"], x["k"], x["v"], rows, w.scale, w.causal, window=w.window)
     Os = O[rows[:, 0], rows[:, 2], rows[:, 1], :]
     Ls = L[rows[:, 0], rows[:, 1], rows[:, 2]]
     res = _parity.compare(Os, Ls, Oref, Lref, name)
