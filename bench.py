@@ -348,13 +348,16 @@ def run_sweep(args):
         # inputs smaller than L2 are timed both warm and with an L2 flush before each launch
         flush = torch.empty(int(2 * 126e6) // 4, dtype=torch.float32, device="cuda")
         win = w.window or None
+        splits = fa.splitkv_default_splits(w.B, w.Hq, w.Nq, w.Nk, w.d, torch.cuda.get_device_properties(0).multi_processor_count) if w.splitkv else None
+        ws = torch.empty(max(1, fa.splitkv_workspace_bytes(w.B, w.Hq, w.Nq, w.d, splits)), dtype=torch.uint8, device="cuda") if splits else None
+        kw = dict(window=win, num_splits=splits, workspace=ws)
         for _ in range(args.warmup):
-            fa.fa_fwd(q, k, v, causal=w.causal, scale=w.scale, out=out, lse=lse, window=win)
+            fa.fa_fwd(q, k, v, causal=w.causal, scale=w.scale, out=out, lse=lse, **kw)
         torch.cuda.synchronize()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record()
         for _ in range(args.steps):
-            fa.fa_fwd(q, k, v, causal=w.causal, scale=w.scale, out=out, lse=lse, window=win)
+            fa.fa_fwd(q, k, v, causal=w.causal, scale=w.scale, out=out, lse=lse, **kw)
         e1.record()
         torch.cuda.synchronize()
         ms_warm = e0.elapsed_time(e1) / args.steps
@@ -363,7 +366,7 @@ def run_sweep(args):
             flush.zero_()
             a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             a.record()
-            fa.fa_fwd(q, k, v, causal=w.causal, scale=w.scale, out=out, lse=lse, window=win)
+            fa.fa_fwd(q, k, v, causal=w.causal, scale=w.scale, out=out, lse=lse, **kw)
             b.record()
             torch.cuda.synchronize()
             cold.append(a.elapsed_time(b))
@@ -372,7 +375,7 @@ def run_sweep(args):
         roof_ms = max(w.flops / (pk["bf16_tflops"] * 1e12), w.io_bytes / (pk["hbm_gbs"] * 1e9)) * 1e3
         print(json.dumps({
             "workload": name, "ms_warm": ms_warm, "ms_l2_flushed": ms_cold,
-            "tflops": w.flops / (ms_cold * 1e-3) / 1e12, "pct_peak": 100 * w.flops / (ms_cold * 1e-3) / 1e12 / pk["bf16_tflops"],
+            "splits": splits, "tflops": w.flops / (ms_cold * 1e-3) / 1e12, "pct_peak": 100 * w.flops / (ms_cold * 1e-3) / 1e12 / pk["bf16_tflops"],
             "hbm_gbs": w.io_bytes / (ms_cold * 1e-3) / 1e9, "roofline_ms": roof_ms,
             "roofline_frac": roof_ms / ms_cold, "status": st}), flush=True)
         del q, k, v, out, lse, flush

@@ -27,7 +27,8 @@ FA_ERR_DEVICE_TIMEOUT = 6
 FA_ERR_NOT_DEVICE_MEMORY = 7
 FA_ERR_OVERLAP = 8
 
-EXPORTED = ("fa_fwd", "fa_fwd_window", "fa_status_string", "fa_device_status", "fa_tile_config", "fa_version")
+EXPORTED = ("fa_fwd", "fa_fwd_window", "fa_fwd_splitkv", "fa_splitkv_workspace_bytes", "fa_splitkv_default_splits",
+            "fa_status_string", "fa_device_status", "fa_tile_config", "fa_version")
 
 
 class FaError(RuntimeError):
@@ -51,6 +52,12 @@ def lib() -> ctypes.CDLL:
         L.fa_fwd.restype = ci
         L.fa_fwd_window.argtypes = [vp, vp, vp, vp, vp, ci, ci, ci, ci, ci, ci, cf, ci, vp]
         L.fa_fwd_window.restype = ci
+        L.fa_fwd_splitkv.argtypes = [vp, vp, vp, vp, vp, ci, ci, ci, ci, ci, ci, cf, ci, ci, vp, ctypes.c_size_t, vp]
+        L.fa_fwd_splitkv.restype = ci
+        L.fa_splitkv_workspace_bytes.argtypes = [ci, ci, ci, ci, ci]
+        L.fa_splitkv_workspace_bytes.restype = ctypes.c_size_t
+        L.fa_splitkv_default_splits.argtypes = [ci, ci, ci, ci, ci, ci]
+        L.fa_splitkv_default_splits.restype = ci
         L.fa_status_string.argtypes = [ci]
         L.fa_status_string.restype = ctypes.c_char_p
         L.fa_device_status.argtypes = [vp, ctypes.POINTER(ci)]
@@ -89,15 +96,26 @@ def fa_fwd_raw(q_ptr, k_ptr, v_ptr, out_ptr, lse_ptr, B, Hq, Hkv, Nq, Nk, d, sca
                         int(d), float(scale), int(causal), stream_ptr)
 
 
+def splitkv_workspace_bytes(B: int, Hq: int, Nq: int, d: int, num_splits: int) -> int:
+    return int(lib().fa_splitkv_workspace_bytes(int(B), int(Hq), int(Nq), int(d), int(num_splits)))
+
+
+def splitkv_default_splits(B: int, Hq: int, Nq: int, Nk: int, d: int, sm_count: int) -> int:
+    return int(lib().fa_splitkv_default_splits(int(B), int(Hq), int(Nq), int(Nk), int(d), int(sm_count)))
+
+
 def fa_fwd(q, k, v, *, causal: bool = False, scale: float | None = None, out=None, lse=None,
-           return_lse: bool = True, stream=None, window: int | None = None):
+           return_lse: bool = True, stream=None, window: int | None = None,
+           num_splits: int | None = None, workspace=None):
     """Exact attention forward on [B, N, H, d] bf16 CUDA tensors.
 
     q: [B, Nq, Hq, d]; k, v: [B, Nk, Hkv, d] with Hq % Hkv == 0 (GQA: query head h
     uses KV head h // (Hq // Hkv)).  Returns (out [B, Nq, Hq, d] bf16, lse [B, Hq, Nq]
     fp32 natural-log log-sum-exp, or None if return_lse is False).  scale defaults to
     1/sqrt(d).  window = W (>= 1) selects the sliding-window mask: row i sees the W keys
-    ending at its causal diagonal (fa_fwd_window).  Runs asynchronously on `stream`
+    ending at its causal diagonal (fa_fwd_window).  num_splits = S (> 1) runs the
+    split-KV forward (fa_fwd_splitkv) with `workspace` (a device tensor of at least
+    splitkv_workspace_bytes; allocated here if None).  Runs asynchronously on `stream`
     (default: torch's current stream)."""
     import torch
     for name, t in (("q", q), ("k", k), ("v", v)):
@@ -116,7 +134,17 @@ def fa_fwd(q, k, v, *, causal: bool = False, scale: float | None = None, out=Non
     if not return_lse:
         lse = None
     lse_ptr = lse.data_ptr() if lse is not None else None
-    if window is not None:
+    if num_splits is not None and num_splits > 1:
+        if window is not None:
+            raise ValueError("split-KV takes the causal or no mask")
+        need = splitkv_workspace_bytes(B, Hq, Nq, d, num_splits)
+        if workspace is None:
+            workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
+        rc = lib().fa_fwd_splitkv(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse_ptr,
+                                  B, Hq, Hkv, Nq, Nk, d, float(scale), 1 if causal else 0, int(num_splits),
+                                  workspace.data_ptr(), workspace.numel() * workspace.element_size(),
+                                  _stream_handle(stream))
+    elif window is not None:
         rc = lib().fa_fwd_window(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse_ptr,
                                  B, Hq, Hkv, Nq, Nk, d, float(scale), int(window), _stream_handle(stream))
     else:

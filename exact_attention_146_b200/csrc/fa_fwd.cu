@@ -35,6 +35,7 @@ using Cfg256 = TileCfg<256, 64, 1, 4, 1, 2>;
 __device__ int g_fa_status;   // per-device kernel status word (0 = OK)
 
 constexpr int kMaxDevices = 64;
+constexpr int kMaxSplits = 256;
 
 struct DeviceState {
     bool probed = false;
@@ -157,7 +158,20 @@ struct Problem {
     float scale;
     int causal;
     int window;
+    int num_splits;     // 1: plain forward; > 1: split-KV into the workspace, then merge
+    float *o_part;      // workspace: fp32 partial O [split][B][Nq][Hq][d]
+    float *lse_part;    // workspace: partial LSE [split][B][Hq][Nq]
 };
+
+// Workspace layout of the split-KV forward: partial O, then (256-byte aligned) partial LSE.
+size_t splitkv_o_bytes(int B, int Hq, int Nq, int d, int splits) {
+    return size_t(splits) * size_t(B) * size_t(Nq) * size_t(Hq) * size_t(d) * 4;
+}
+size_t splitkv_bytes(int B, int Hq, int Nq, int d, int splits) {
+    if (splits <= 1) return 0;
+    const size_t o = (splitkv_o_bytes(B, Hq, Nq, d, splits) + 255) & ~size_t(255);
+    return o + size_t(splits) * size_t(B) * size_t(Hq) * size_t(Nq) * 4;
+}
 
 template <class C>
 int launch(const Problem &pr, DeviceState &dev, int cfg_slot, cudaStream_t stream) {
@@ -200,7 +214,12 @@ int launch(const Problem &pr, DeviceState &dev, int cfg_slot, cudaStream_t strea
     p.causal = pr.causal;
     p.window = pr.window;
     p.nqb = (pr.Nq + C::NQT * kBlockQ - 1) / (C::NQT * kBlockQ);
-    const long long units = (long long)pr.B * pr.Hq * p.nqb;
+    const int nkv = (pr.Nk + C::BC - 1) / C::BC;
+    p.num_splits = pr.num_splits > 1 ? pr.num_splits : 1;
+    p.split_tiles = (nkv + p.num_splits - 1) / p.num_splits;
+    p.o_part = pr.o_part;
+    p.lse_part = pr.lse_part;
+    const long long units = (long long)pr.B * pr.Hq * p.nqb * p.num_splits;
     if (units > 0x7fffffffLL) return FA_ERR_INVALID_ARG;
     p.num_units = int(units);
     p.scale_log2 = pr.scale * 1.4426950408889634f;
@@ -208,6 +227,14 @@ int launch(const Problem &pr, DeviceState &dev, int cfg_slot, cudaStream_t strea
     const int grid = int(units < dev.num_sms ? units : dev.num_sms);
     fa_fwd_kernel<C><<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(mq, mk, mv, p);
     if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
+    if (p.num_splits > 1) {
+        const long long rows = (long long)pr.B * pr.Nq * pr.Hq;
+        const long long want = (rows + 7) / 8;   // 8 rows (warps) per 256-thread block
+        const int mgrid = int(want < 8LL * dev.num_sms ? want : 8LL * dev.num_sms);
+        fa_splitkv_merge_kernel<C::D><<<mgrid > 0 ? mgrid : 1, 256, 0, stream>>>(
+            pr.o_part, pr.lse_part, static_cast<__nv_bfloat16 *>(pr.out), pr.lse, pr.B, pr.Hq, pr.Nq, p.num_splits);
+        if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
+    }
     return FA_OK;
 }
 
@@ -266,12 +293,14 @@ namespace {
 // The shared forward: mask = none (causal 0, window 0), causal (1, 0) or sliding window
 // (1, W >= 1).
 int forward(const void *q, const void *k, const void *v, void *out, float *lse, int B, int Hq, int Hkv,
-            int Nq, int Nk, int d, float scale, int causal, int window, void *stream) {
+            int Nq, int Nk, int d, float scale, int causal, int window, int num_splits, void *workspace,
+            size_t workspace_bytes, void *stream) {
     // ---- host-only validation (no CUDA call before this block passes)
     if (B < 0 || Hq <= 0 || Hkv <= 0 || Nq < 0 || Nk < 0) return FA_ERR_INVALID_ARG;
     if (Hq % Hkv != 0) return FA_ERR_INVALID_ARG;
     if (causal != 0 && causal != 1) return FA_ERR_INVALID_ARG;
     if (window < 0 || (window > 0 && !causal)) return FA_ERR_INVALID_ARG;
+    if (num_splits < 1 || num_splits > kMaxSplits) return FA_ERR_INVALID_ARG;
     if (!std::isfinite(scale) || !(scale > 0.f)) return FA_ERR_INVALID_ARG;
     if (tile_config(d, nullptr, nullptr, nullptr, nullptr) != FA_OK) return FA_ERR_UNSUPPORTED_HEAD_DIM;
     const size_t q_bytes = size_t(B) * size_t(Nq) * size_t(Hq) * size_t(d) * 2;
@@ -288,6 +317,15 @@ int forward(const void *q, const void *k, const void *v, void *out, float *lse, 
         overlaps(lse, lse_bytes, k, kv_bytes) || overlaps(lse, lse_bytes, v, kv_bytes) ||
         overlaps(lse, lse_bytes, out, q_bytes))
         return FA_ERR_OVERLAP;
+    const size_t ws_bytes = (Nk > 0) ? splitkv_bytes(B, Hq, Nq, d, num_splits) : 0;
+    if (ws_bytes > 0) {
+        if (workspace == nullptr || workspace_bytes < ws_bytes) return FA_ERR_INVALID_ARG;
+        if (mis(workspace, 256)) return FA_ERR_MISALIGNED;
+        if (overlaps(workspace, ws_bytes, q, q_bytes) || overlaps(workspace, ws_bytes, k, kv_bytes) ||
+            overlaps(workspace, ws_bytes, v, kv_bytes) || overlaps(workspace, ws_bytes, out, q_bytes) ||
+            overlaps(workspace, ws_bytes, lse, lse_bytes))
+            return FA_ERR_OVERLAP;
+    }
 
     // ---- device checks
     DeviceState *dev = nullptr;
@@ -301,6 +339,7 @@ int forward(const void *q, const void *k, const void *v, void *out, float *lse, 
         if ((rc = check_device_range(v, kv_bytes, dev_id)) != FA_OK) return rc;
     }
     if (lse && (rc = check_device_range(lse, lse_bytes, dev_id)) != FA_OK) return rc;
+    if (ws_bytes > 0 && (rc = check_device_range(workspace, ws_bytes, dev_id)) != FA_OK) return rc;
 
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     if (Nk == 0) {
@@ -311,7 +350,14 @@ int forward(const void *q, const void *k, const void *v, void *out, float *lse, 
         return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
     }
 
-    const Problem pr{q, k, v, out, lse, B, Hq, Hkv, Nq, Nk, d, scale, causal, window};
+    float *o_part = nullptr, *lse_part = nullptr;
+    if (ws_bytes > 0) {
+        o_part = static_cast<float *>(workspace);
+        lse_part = reinterpret_cast<float *>(static_cast<char *>(workspace) +
+                                             ((splitkv_o_bytes(B, Hq, Nq, d, num_splits) + 255) & ~size_t(255)));
+    }
+    const Problem pr{q, k, v, out, lse, B, Hq, Hkv, Nq, Nk, d, scale, causal, window,
+                     ws_bytes > 0 ? num_splits : 1, o_part, lse_part};
     switch (d) {
         case 32: return launch<Cfg32>(pr, *dev, 0, st);
         case 64: return launch<Cfg64>(pr, *dev, 1, st);
@@ -330,13 +376,38 @@ extern "C" {
 
 int fa_fwd(const void *q, const void *k, const void *v, void *out, float *lse, int B, int Hq, int Hkv,
            int Nq, int Nk, int d, float scale, int causal, void *stream) {
-    return forward(q, k, v, out, lse, B, Hq, Hkv, Nq, Nk, d, scale, causal, 0, stream);
+    return forward(q, k, v, out, lse, B, Hq, Hkv, Nq, Nk, d, scale, causal, 0, 1, nullptr, 0, stream);
+}
+
+size_t fa_splitkv_workspace_bytes(int B, int Hq, int Nq, int d, int num_splits) {
+    if (B < 0 || Hq < 0 || Nq < 0 || d <= 0 || num_splits < 1 || num_splits > kMaxSplits) return 0;
+    return splitkv_bytes(B, Hq, Nq, d, num_splits);
+}
+
+int fa_splitkv_default_splits(int B, int Hq, int Nq, int Nk, int d, int sm_count) {
+    int bq, bk, nqt, ns;
+    if (tile_config(d, &bq, &bk, &nqt, &ns) != FA_OK || B <= 0 || Hq <= 0 || Nq <= 0 || Nk <= 0 || sm_count <= 0)
+        return 1;
+    const long long units = (long long)B * Hq * ((Nq + bq * nqt - 1) / (bq * nqt));
+    if (units >= sm_count) return 1;
+    const int nkv = (Nk + bk - 1) / bk;
+    long long s = (sm_count + units - 1) / units;   // fill the SMs once
+    if (s > nkv / 4) s = nkv / 4;                    // keep >= 4 key tiles per split
+    if (s > kMaxSplits) s = kMaxSplits;
+    return s < 1 ? 1 : int(s);
+}
+
+int fa_fwd_splitkv(const void *q, const void *k, const void *v, void *out, float *lse, int B, int Hq,
+                   int Hkv, int Nq, int Nk, int d, float scale, int causal, int num_splits, void *workspace,
+                   size_t workspace_bytes, void *stream) {
+    return forward(q, k, v, out, lse, B, Hq, Hkv, Nq, Nk, d, scale, causal, 0, num_splits, workspace,
+                   workspace_bytes, stream);
 }
 
 int fa_fwd_window(const void *q, const void *k, const void *v, void *out, float *lse, int B, int Hq,
                   int Hkv, int Nq, int Nk, int d, float scale, int window, void *stream) {
     if (window < 1) return FA_ERR_INVALID_ARG;
-    return forward(q, k, v, out, lse, B, Hq, Hkv, Nq, Nk, d, scale, 1, window, stream);
+    return forward(q, k, v, out, lse, B, Hq, Hkv, Nq, Nk, d, scale, 1, window, 1, nullptr, 0, stream);
 }
 
 int fa_device_status(void *stream, int *detail) {

@@ -55,7 +55,11 @@ struct FwdParams {
     int causal;           // 1 for the causal and the sliding-window masks
     int window;           // 0, or the sliding-window width W (keys i+Nk-Nq-W < j <= i+Nk-Nq)
     int nqb;              // query blocks of NQT*128 rows per (b, hq)
-    int num_units;        // B * Hq * nqb
+    int num_splits;       // key-range splits per query block (1: no split)
+    int split_tiles;      // key tiles per split
+    int num_units;        // B * Hq * nqb * num_splits
+    float *o_part;        // num_splits > 1: fp32 partial O [split][B][Nq][Hq][d], normalised
+    float *lse_part;      // num_splits > 1: partial LSE [split][B][Hq][Nq]
     float scale_log2;     // scale * log2(e)
 };
 
@@ -141,6 +145,7 @@ struct UnitInfo {
     int b, hq, kvh, q0;
     int js[2], je[2];   // key tiles [js, je) each query tile visits (empty: js == je)
     int j_lo, j_hi;     // union of the ranges: the K/V tiles the unit loads
+    int split;          // which key-range split (0 when not split)
 };
 
 // Static schedule shared by all roles.  Causal: longest query blocks first, heads of
@@ -149,6 +154,8 @@ struct UnitInfo {
 template <class C>
 __device__ __forceinline__ UnitInfo decode_unit(int u, const FwdParams &p) {
     UnitInfo w;
+    w.split = u % p.num_splits;
+    u /= p.num_splits;
     const int bh = p.B * p.Hq;
     int qb, r;
     if (p.causal) {
@@ -181,6 +188,10 @@ __device__ __forceinline__ UnitInfo decode_unit(int u, const FwdParams &p) {
             if (p.window > 0) {
                 const int first = q_lo + diag - p.window + 1;   // first visible key of the first row
                 js = first <= 0 ? 0 : min(first / C::BC, nkv);
+            }
+            if (p.num_splits > 1) {   // this split's share of the key tiles
+                js = max(js, w.split * p.split_tiles);
+                je = min(je, (w.split + 1) * p.split_tiles);
             }
             if (je <= js) js = je = 0;
         }
@@ -623,7 +634,10 @@ __device__ void softmax_role(const FwdParams &p, uint32_t sbase, uint32_t tmem, 
         {
             const float inv_l = l > 0.f ? 1.f / l : 0.f;
             const bool store = row < p.Nq;
-            __nv_bfloat16 *orow = p.out + ((size_t(w.b) * p.Nq + size_t(row)) * p.Hq + w.hq) * C::D;
+            const size_t row_off = (size_t(w.b) * p.Nq + size_t(row)) * p.Hq + w.hq;   // [b][row][hq]
+            const bool split_mode = p.num_splits > 1;
+            __nv_bfloat16 *orow = p.out + row_off * C::D;
+            float *prow = split_mode ? p.o_part + (size_t(w.split) * p.B * p.Nq * p.Hq + row_off) * C::D : nullptr;
 #pragma unroll
             for (int c = 0; c < C::O_CHUNKS; ++c) {
                 uint32_t o[32];
@@ -632,6 +646,20 @@ __device__ void softmax_role(const FwdParams &p, uint32_t sbase, uint32_t tmem, 
                 } else {
 #pragma unroll
                     for (int i = 0; i < 32; ++i) o[i] = 0u;
+                }
+                if (split_mode) {
+                    // fp32 partial for the merge (normalised by this split's own l)
+                    if (store) {
+#pragma unroll
+                        for (int v4 = 0; v4 < 8; ++v4) {
+                            const int col = 32 * c + 4 * v4;
+                            if (col < C::D)
+                                *reinterpret_cast<float4 *>(prow + col) =
+                                    make_float4(__uint_as_float(o[4 * v4]) * inv_l, __uint_as_float(o[4 * v4 + 1]) * inv_l,
+                                                __uint_as_float(o[4 * v4 + 2]) * inv_l, __uint_as_float(o[4 * v4 + 3]) * inv_l);
+                        }
+                    }
+                    continue;
                 }
                 uint32_t pk[16];
 #pragma unroll
@@ -649,9 +677,13 @@ __device__ void softmax_role(const FwdParams &p, uint32_t sbase, uint32_t tmem, 
             }
             sm100::tc_fence_before_sync();
             sm100::mbar_arrive(bar(C::B_OEMPTY + t));
-            if (p.lse != nullptr && store)
-                p.lse[(size_t(w.b) * p.Hq + w.hq) * p.Nq + row] =
-                    l > 0.f ? (m_ref + log2f(l)) * 0.6931471805599453f : -INFINITY;
+            const float lse_row = l > 0.f ? (m_ref + log2f(l)) * 0.6931471805599453f : -INFINITY;
+            const size_t lse_off = (size_t(w.b) * p.Hq + w.hq) * p.Nq + row;
+            if (split_mode) {
+                if (store) p.lse_part[size_t(w.split) * p.B * p.Hq * p.Nq + lse_off] = lse_row;
+            } else if (p.lse != nullptr && store) {
+                p.lse[lse_off] = lse_row;
+            }
         }
     }
 unwind:
@@ -723,6 +755,53 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     __syncthreads();
     sm100::tc_fence_after_sync();
     if (warp == 0) sm100::tmem_dealloc(tmem, C::TMEM_COLS);
+}
+
+// Split-KV merge: one warp per output row (b, i, hq).  With m = max_s LSE_s, the weights
+// w_s = e^(LSE_s - m) combine the per-split normalised outputs O = sum_s w_s O_s / sum_s w_s,
+// and LSE = m + ln sum_s w_s; a row no split saw (all LSE_s = -inf) gets O = 0, LSE = -inf.
+template <int D>
+__global__ void __launch_bounds__(256) fa_splitkv_merge_kernel(const float *o_part, const float *lse_part,
+                                                               __nv_bfloat16 *out, float *lse, int B, int Hq,
+                                                               int Nq, int num_splits) {
+    constexpr int PER_LANE = (D + 31) / 32;
+    const long rows = long(B) * Nq * Hq;
+    const long split_stride_o = rows * D, split_stride_l = rows;
+    const int lane = int(threadIdx.x) % 32;
+    for (long r = (long(blockIdx.x) * blockDim.x + threadIdx.x) / 32; r < rows;
+         r += long(gridDim.x) * blockDim.x / 32) {
+        const int hq = int(r % Hq);
+        const long bi = r / Hq;                 // b * Nq + i
+        const int i = int(bi % Nq);
+        const int b = int(bi / Nq);
+        const long lse_off = (long(b) * Hq + hq) * Nq + i;
+        float m = -INFINITY;
+        for (int sp = 0; sp < num_splits; ++sp) m = fmaxf(m, lse_part[sp * split_stride_l + lse_off]);
+        float acc[PER_LANE];
+#pragma unroll
+        for (int e = 0; e < PER_LANE; ++e) acc[e] = 0.f;
+        float wsum = 0.f;
+        if (m != -INFINITY) {
+            for (int sp = 0; sp < num_splits; ++sp) {
+                const float ls = lse_part[sp * split_stride_l + lse_off];
+                const float wgt = ls == -INFINITY ? 0.f : __expf(ls - m);
+                wsum += wgt;
+                const float *src = o_part + sp * split_stride_o + r * D;
+#pragma unroll
+                for (int e = 0; e < PER_LANE; ++e) {
+                    const int col = lane + 32 * e;
+                    if (col < D) acc[e] = fmaf(wgt, src[col], acc[e]);
+                }
+            }
+        }
+        const float inv = wsum > 0.f ? 1.f / wsum : 0.f;
+#pragma unroll
+        for (int e = 0; e < PER_LANE; ++e) {
+            const int col = lane + 32 * e;
+            if (col < D) out[r * D + col] = __float2bfloat16_rn(acc[e] * inv);
+        }
+        if (lse != nullptr && lane == 0) lse[lse_off] = wsum > 0.f ? m + logf(wsum) : -INFINITY;
+    }
 }
 
 // Nk == 0: no key at all, so every output row is 0 and every LSE is -inf.

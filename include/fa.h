@@ -32,6 +32,8 @@
 #ifndef EXACT_ATTENTION_FA_H
 #define EXACT_ATTENTION_FA_H
 
+#include <stddef.h>
+
 #ifdef __cplusplus
 extern "C" {
 #endif
@@ -89,6 +91,36 @@ int fa_fwd(const void *q, const void *k, const void *v, void *out, float *lse,
 int fa_fwd_window(const void *q, const void *k, const void *v, void *out, float *lse,
                   int B, int Hq, int Hkv, int Nq, int Nk, int d, float scale, int window,
                   void *stream);
+
+/*
+ * Split-KV forward, for shapes with too few (batch, head, query block) units to fill the
+ * GPU, e.g. decoding (Nq much smaller than Nk).  The key range is cut into num_splits
+ * slices of whole key tiles; each (unit, slice) runs the same tiled online softmax and
+ * writes its own normalised output O_s and log-sum-exp LSE_s (fp32) into the workspace;
+ * a merge kernel on the same stream then writes
+ *
+ *     LSE = ln sum_s exp(LSE_s),   O = sum_s exp(LSE_s - LSE) O_s,
+ *
+ * which is exactly the softmax over the whole key range (the same identity the online
+ * softmax's running rescale applies block by block; slices that see no key have
+ * LSE_s = -inf and weight 0).  Results equal fa_fwd up to rounding.
+ *
+ * fa_splitkv_workspace_bytes: device bytes the workspace needs (0 for num_splits == 1);
+ *   0 also for invalid sizes.
+ * fa_splitkv_default_splits: a split count that fills sm_count SMs once (1 when the
+ *   plain forward already does), keeping at least four key tiles per slice.
+ * fa_fwd_splitkv: as fa_fwd (causal in {0, 1}), plus 1 <= num_splits <= 256 and a
+ *   caller-owned device workspace of at least fa_splitkv_workspace_bytes bytes, 256-byte
+ *   aligned, not overlapping any tensor (FA_ERR_INVALID_ARG / FA_ERR_MISALIGNED /
+ *   FA_ERR_OVERLAP / FA_ERR_NOT_DEVICE_MEMORY otherwise).  The workspace is scratch: its
+ *   contents are undefined afterwards, and two calls must not share one concurrently.
+ *   num_splits == 1 needs no workspace and is fa_fwd.
+ */
+size_t fa_splitkv_workspace_bytes(int B, int Hq, int Nq, int d, int num_splits);
+int fa_splitkv_default_splits(int B, int Hq, int Nq, int Nk, int d, int sm_count);
+int fa_fwd_splitkv(const void *q, const void *k, const void *v, void *out, float *lse,
+                   int B, int Hq, int Hkv, int Nq, int Nk, int d, float scale, int causal,
+                   int num_splits, void *workspace, size_t workspace_bytes, void *stream);
 
 /* Human-readable text of a status code (static storage; never NULL). */
 const char *fa_status_string(int status);

@@ -117,6 +117,7 @@ class Workload:
     k_mult: float = 1.0      # same for K
     seed: int = 0
     window: int = 0          # sliding window of W keys (0: none; implies causal)
+    splitkv: bool = False    # run with the library's default split-KV count (decode shapes)
 
     @property
     def scale(self) -> float:
@@ -160,8 +161,8 @@ def make_inputs(w: Workload) -> dict[str, np.ndarray]:
     return out
 
 
-def _wl(name, wid, B, H, N, d, causal=False, Hkv=None, **kw):
-    return Workload(name, wid, B, H, Hkv or H, N, N, d, causal, **kw)
+def _wl(name, wid, B, H, N, d, causal=False, Hkv=None, Nk=None, **kw):
+    return Workload(name, wid, B, H, Hkv or H, N, Nk or N, d, causal, **kw)
 
 
 # The workload table.  Ids are stable: changing one changes every seeded input of it.
@@ -184,6 +185,7 @@ for _w in [
     _wl("hdim192_b2_n4096_h16", 15, 2, 16, 4096, 192),
     _wl("hdim256_b2_n4096_h16", 16, 2, 16, 4096, 256),
     _wl("window4k_long16k_b1_h32_d128", 17, 1, 32, 16384, 128, causal=True, window=4096),
+    _wl("decode_b4_hq32_hkv8_nq16_nk32k_d128", 18, 4, 32, 16, 128, Hkv=8, Nk=32768, splitkv=True),
 ]:
     WORKLOADS[_w.name] = _w
 

@@ -24,7 +24,7 @@ def bf16_to_f64(t):
     return t.float().cpu().numpy().astype(np.float64)
 
 
-def run_cuda(x, scale, causal, with_lse=True, canary=True, window=None):
+def run_cuda(x, scale, causal, with_lse=True, canary=True, window=None, num_splits=None):
     """fa_fwd through the C ABI; out/lse pre-filled with NaN so unwritten rows show up."""
     import torch
     import exact_attention_146_b200 as fa
@@ -32,7 +32,8 @@ def run_cuda(x, scale, causal, with_lse=True, canary=True, window=None):
     out = torch.full_like(q, float("nan")) if canary else torch.empty_like(q)
     B, Nq, Hq, d = q.shape
     lse = torch.full((B, Hq, Nq), float("nan"), dtype=torch.float32, device="cuda") if with_lse else None
-    fa.fa_fwd(q, k, v, causal=causal, scale=scale, out=out, lse=lse, return_lse=with_lse, window=window)
+    fa.fa_fwd(q, k, v, causal=causal, scale=scale, out=out, lse=lse, return_lse=with_lse, window=window,
+              num_splits=num_splits)
     st, word = fa.device_status()
     assert st == fa.FA_OK, f"device status {st} (word {word:#x})"
     torch.cuda.synchronize()
@@ -58,6 +59,14 @@ def compare(O, L, Oref, Lref, what=""):
     if L is not None:
         assert res["max_abs_LSE"] <= TOL_LSE, f"{what}: max|dLSE| = {res['max_abs_LSE']:.3e}"
     return res
+
+
+def workload_splits(w: synth.Workload) -> int | None:
+    """The split count a workload runs with (the library's default for split-KV ones)."""
+    if not w.splitkv:
+        return None
+    import exact_attention_146_b200 as fa
+    return fa.splitkv_default_splits(w.B, w.Hq, w.Nq, w.Nk, w.d, 148)
 
 
 def sample_rows(w: synth.Workload, n: int, seed: int = 0):

@@ -96,6 +96,33 @@ def test_window_must_be_positive(L, window):
                            1, 2, 1, 16, 16, 64, 0.125, window, None) == fa.FA_ERR_INVALID_ARG
 
 
+def test_splitkv_workspace_and_default_splits(L):
+    assert fa.splitkv_workspace_bytes(2, 4, 100, 128, 1) == 0
+    o = 3 * 2 * 100 * 4 * 128 * 4
+    assert fa.splitkv_workspace_bytes(2, 4, 100, 128, 3) == ((o + 255) // 256) * 256 + 3 * 2 * 4 * 100 * 4
+    assert fa.splitkv_workspace_bytes(2, 4, 100, 128, 0) == 0 and fa.splitkv_workspace_bytes(2, 4, 100, 128, 999) == 0
+    assert fa.splitkv_default_splits(8, 32, 4096, 4096, 128, 148) == 1       # already fills the GPU
+    s = fa.splitkv_default_splits(4, 32, 16, 32768, 128, 148)                 # 128 units
+    assert s == 2
+    assert fa.splitkv_default_splits(1, 1, 1, 65536, 128, 148) == 128        # capped by 4 tiles per split
+    assert fa.splitkv_default_splits(1, 1, 1, 300, 64, 148) == 1             # too few key tiles
+
+
+def _splitkv(L, splits=4, ws=FAKE + (5 << 30), ws_bytes=1 << 30, out=FAKE + (3 << 30)):
+    return L.fa_fwd_splitkv(FAKE, FAKE + (1 << 30), FAKE + (2 << 30), out, FAKE + (4 << 30),
+                            1, 2, 1, 16, 4096, 64, 0.125, 0, splits, ws, ws_bytes, None)
+
+
+def test_splitkv_validation(L):
+    assert _splitkv(L, splits=0) == fa.FA_ERR_INVALID_ARG
+    assert _splitkv(L, splits=257) == fa.FA_ERR_INVALID_ARG
+    assert _splitkv(L, ws=None) == fa.FA_ERR_INVALID_ARG
+    assert _splitkv(L, ws_bytes=100) == fa.FA_ERR_INVALID_ARG
+    assert _splitkv(L, ws=FAKE + (5 << 30) + 16) == fa.FA_ERR_MISALIGNED
+    assert _splitkv(L, ws=FAKE + (3 << 30)) == fa.FA_ERR_OVERLAP            # workspace on out
+    assert _splitkv(L) in (fa.FA_ERR_UNSUPPORTED_DEVICE, fa.FA_ERR_NOT_DEVICE_MEMORY)
+
+
 def test_empty_problems_are_noops(L):
     # no output rows: nothing to validate against the device, nothing launched
     assert call(L, B=0, q=None, k=None, v=None, out=None, lse=None) == fa.FA_OK

@@ -111,6 +111,25 @@ def test_sliding_window_unequal_lengths(orc, Nq, Nk, W):
     _parity.compare(O, L, Oref, Lref, f"window Nq={Nq} Nk={Nk} W={W}")
 
 
+@pytest.mark.parametrize("d", [64, 128, 256])
+@pytest.mark.parametrize("Nq,Nk", [(1, 1000), (16, 2049), (130, 700)])
+@pytest.mark.parametrize("splits", [2, 3, 7, 40])
+@pytest.mark.parametrize("causal", [False, True])
+def test_splitkv(orc, d, Nq, Nk, splits, causal):
+    """Split-KV (40 splits leaves some slices without a key tile) equals the oracle."""
+    x = tiny(1, 4, 2, Nq, Nk, d, seed=Nq + Nk + splits + d)
+    O, L = _parity.run_cuda(x, 1.0 / math.sqrt(d), causal, num_splits=splits)
+    Oref, Lref = orc.forward(x["q"], x["k"], x["v"], 1.0 / math.sqrt(d), causal)
+    _parity.compare(O, L, Oref, Lref, f"splitkv d={d} Nq={Nq} Nk={Nk} S={splits} causal={causal}")
+
+
+def test_splitkv_matches_plain_forward():
+    x = tiny(2, 8, 2, 64, 4096, 128, seed=99)
+    O1, L1 = _parity.run_cuda(x, 0.08, False)
+    O2, L2 = _parity.run_cuda(x, 0.08, False, num_splits=5)
+    assert np.abs(O1 - O2).max() < 1e-2 and np.abs(L1 - L2).max() < 1e-4
+
+
 def test_lse_optional(orc):
     x = tiny(1, 2, 1, 200, 200, 64, seed=80)
     O, L = _parity.run_cuda(x, 0.125, True, with_lse=False)
@@ -212,7 +231,7 @@ def test_workload_sampled_rows(orc, name):
     oracle one by one, and every output row checked to be written and finite."""
     w = synth.WORKLOADS[name]
     x = synth.make_inputs(w)
-    O, L = _parity.run_cuda(x, w.scale, w.causal, window=w.window or None)
+    O, L = _parity.run_cuda(x, w.scale, w.causal, window=w.window or None, num_splits=_parity.workload_splits(w))
     assert np.isfinite(O).all() and np.isfinite(L).all()
     rows = _parity.sample_rows(w, 192, seed=w.wid)
     Oref, Lref = orc.rows(x["q"], x["k"], x["v"], rows, w.scale, w.causal, window=w.window)
