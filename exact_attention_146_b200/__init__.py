@@ -26,9 +26,11 @@ FA_ERR_CUDA = 5
 FA_ERR_DEVICE_TIMEOUT = 6
 FA_ERR_NOT_DEVICE_MEMORY = 7
 FA_ERR_OVERLAP = 8
+FA_ERR_SCRATCH_LIMIT = 9
+SPLITKV_STATIC_SCRATCH_BYTES = 16 * 1024 * 1024
 
 EXPORTED = ("fa_fwd", "fa_fwd_window", "fa_fwd_splitkv", "fa_splitkv_workspace_bytes", "fa_splitkv_default_splits",
-            "fa_status_string", "fa_device_status", "fa_tile_config", "fa_version")
+            "fa_fwd_splitkv_static", "fa_status_string", "fa_device_status", "fa_tile_config", "fa_version")
 
 
 class FaError(RuntimeError):
@@ -54,6 +56,8 @@ def lib() -> ctypes.CDLL:
         L.fa_fwd_window.restype = ci
         L.fa_fwd_splitkv.argtypes = [vp, vp, vp, vp, vp, ci, ci, ci, ci, ci, ci, cf, ci, ci, vp, ctypes.c_size_t, vp]
         L.fa_fwd_splitkv.restype = ci
+        L.fa_fwd_splitkv_static.argtypes = [vp, vp, vp, vp, vp, ci, ci, ci, ci, ci, ci, cf, ci, ci, vp]
+        L.fa_fwd_splitkv_static.restype = ci
         L.fa_splitkv_workspace_bytes.argtypes = [ci, ci, ci, ci, ci]
         L.fa_splitkv_workspace_bytes.restype = ctypes.c_size_t
         L.fa_splitkv_default_splits.argtypes = [ci, ci, ci, ci, ci, ci]

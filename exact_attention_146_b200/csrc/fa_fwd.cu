@@ -278,6 +278,9 @@ const char *fa_status_string(int status) {
         case FA_ERR_NOT_DEVICE_MEMORY:
             return "a tensor is not device memory of the current device, or runs past its allocation";
         case FA_ERR_OVERLAP: return "out or lse overlaps an input or each other";
+        case FA_ERR_SCRATCH_LIMIT:
+            return "the split-KV partials need more than the library's 16 MiB static scratch: use "
+                   "fa_fwd_splitkv with a caller workspace, or fewer splits";
         default: return "unknown status";
     }
 }
@@ -292,9 +295,11 @@ namespace {
 
 // The shared forward: mask = none (causal 0, window 0), causal (1, 0) or sliding window
 // (1, W >= 1).
+// `library_scratch`: the workspace is the library's own static scratch (already known to be
+// device memory of the current device), so its device-range check is skipped.
 int forward(const void *q, const void *k, const void *v, void *out, float *lse, int B, int Hq, int Hkv,
             int Nq, int Nk, int d, float scale, int causal, int window, int num_splits, void *workspace,
-            size_t workspace_bytes, void *stream) {
+            size_t workspace_bytes, void *stream, bool library_scratch = false) {
     // ---- host-only validation (no CUDA call before this block passes)
     if (B < 0 || Hq <= 0 || Hkv <= 0 || Nq < 0 || Nk < 0) return FA_ERR_INVALID_ARG;
     if (Hq % Hkv != 0) return FA_ERR_INVALID_ARG;
@@ -339,7 +344,8 @@ int forward(const void *q, const void *k, const void *v, void *out, float *lse, 
         if ((rc = check_device_range(v, kv_bytes, dev_id)) != FA_OK) return rc;
     }
     if (lse && (rc = check_device_range(lse, lse_bytes, dev_id)) != FA_OK) return rc;
-    if (ws_bytes > 0 && (rc = check_device_range(workspace, ws_bytes, dev_id)) != FA_OK) return rc;
+    if (ws_bytes > 0 && !library_scratch && (rc = check_device_range(workspace, ws_bytes, dev_id)) != FA_OK)
+        return rc;
 
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     if (Nk == 0) {
@@ -402,6 +408,56 @@ int fa_fwd_splitkv(const void *q, const void *k, const void *v, void *out, float
                    size_t workspace_bytes, void *stream) {
     return forward(q, k, v, out, lse, B, Hq, Hkv, Nq, Nk, d, scale, causal, 0, num_splits, workspace,
                    workspace_bytes, stream);
+}
+
+}  // extern "C"
+
+namespace {
+
+// Scratch of fa_fwd_splitkv_static, for callers that cannot allocate device memory around
+// the call (see include/fa.h).  One array per device (a __device__ variable exists once in
+// every device context); its address is looked up once per device, with that device current.
+static __device__ __align__(256) unsigned char g_splitkv_scratch[FA_SPLITKV_STATIC_SCRATCH_BYTES];
+void *g_scratch_addr[kMaxDevices] = {};
+
+int static_scratch(void **out) {
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+        cudaGetLastError();
+        return FA_ERR_UNSUPPORTED_DEVICE;
+    }
+    std::lock_guard<std::mutex> lock(g_mutex);
+    if (g_scratch_addr[dev] == nullptr) {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_splitkv_scratch) != cudaSuccess || p == nullptr) {
+            cudaGetLastError();
+            return FA_ERR_CUDA;
+        }
+        g_scratch_addr[dev] = p;
+    }
+    *out = g_scratch_addr[dev];
+    return FA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int fa_fwd_splitkv_static(const void *q, const void *k, const void *v, void *out, float *lse, int B, int Hq,
+                          int Hkv, int Nq, int Nk, int d, float scale, int causal, int num_splits,
+                          void *stream) {
+    if (B < 0 || Hq <= 0 || Hkv <= 0 || Nq < 0 || Nk < 0 || num_splits < 1 || num_splits > kMaxSplits)
+        return FA_ERR_INVALID_ARG;
+    if (tile_config(d, nullptr, nullptr, nullptr, nullptr) != FA_OK) return FA_ERR_UNSUPPORTED_HEAD_DIM;
+    const size_t need = (Nk > 0) ? splitkv_bytes(B, Hq, Nq, d, num_splits) : 0;
+    if (need > sizeof(g_splitkv_scratch)) return FA_ERR_SCRATCH_LIMIT;
+    void *scratch = nullptr;
+    if (need > 0) {
+        const int rc = static_scratch(&scratch);
+        if (rc != FA_OK) return rc;
+    }
+    return forward(q, k, v, out, lse, B, Hq, Hkv, Nq, Nk, d, scale, causal, 0, num_splits, scratch,
+                   sizeof(g_splitkv_scratch), stream, true);
 }
 
 int fa_fwd_window(const void *q, const void *k, const void *v, void *out, float *lse, int B, int Hq,

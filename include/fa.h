@@ -51,7 +51,9 @@ enum fa_status_code {
                                         gave up after its time limit; outputs are undefined */
     FA_ERR_NOT_DEVICE_MEMORY = 7,    /* a tensor pointer is not device memory of the current device,
                                         or its extent runs past the end of its allocation */
-    FA_ERR_OVERLAP = 8               /* out or lse overlaps an input or each other */
+    FA_ERR_OVERLAP = 8,              /* out or lse overlaps an input or each other */
+    FA_ERR_SCRATCH_LIMIT = 9         /* fa_fwd_splitkv_static: the partials need more than the
+                                        library's static scratch (FA_SPLITKV_STATIC_SCRATCH_BYTES) */
 };
 
 /*
@@ -121,6 +123,31 @@ int fa_splitkv_default_splits(int B, int Hq, int Nq, int Nk, int d, int sm_count
 int fa_fwd_splitkv(const void *q, const void *k, const void *v, void *out, float *lse,
                    int B, int Hq, int Hkv, int Nq, int Nk, int d, float scale, int causal,
                    int num_splits, void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * fa_fwd_splitkv_static -- fa_fwd_splitkv without a caller workspace and without any
+ * allocation: the per-split partials go to a scratch array the library holds in static
+ * device memory, FA_SPLITKV_STATIC_SCRATCH_BYTES (16 MiB) per device.  The paper has no
+ * counterpart; it exists for callers that cannot allocate device memory around the call:
+ * a plain C host program that embeds the library with no device allocator of its own, or a
+ * serving loop whose device memory is planned up front, where a cudaMalloc in the middle
+ * of a step would synchronise the device and could fail under memory pressure.
+ *
+ * Arguments, layouts, ownership and errors as fa_fwd_splitkv minus the workspace.  A problem
+ * whose partials (fa_splitkv_workspace_bytes) exceed the static scratch returns
+ * FA_ERR_SCRATCH_LIMIT and launches nothing; use fa_fwd_splitkv or fewer splits then.
+ * Nothing in the scratch has to start at zero: each call writes every partial the merge
+ * reads before the merge reads it.
+ * The first call on each device does one-time set-up there (looks up the scratch address,
+ * the same device probes as fa_fwd); make that first call before any stream capture.
+ * All calls on one device share the one scratch array: two calls that may run at the same
+ * time (different streams or threads, no ordering between them) race and corrupt each
+ * other's results.  Calls ordered on one stream are safe.
+ */
+#define FA_SPLITKV_STATIC_SCRATCH_BYTES (16u * 1024u * 1024u)
+int fa_fwd_splitkv_static(const void *q, const void *k, const void *v, void *out, float *lse,
+                          int B, int Hq, int Hkv, int Nq, int Nk, int d, float scale, int causal,
+                          int num_splits, void *stream);
 
 /* Human-readable text of a status code (static storage; never NULL). */
 const char *fa_status_string(int status);
