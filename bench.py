@@ -163,7 +163,7 @@ def oracle_sample_tflops(w: synth.Workload, target_s: float, heads_cap: int | No
         k = np.ascontiguousarray(x["k"][:, :, g:g + 1])
         v = np.ascontiguousarray(x["v"][:, :, g:g + 1])
         t0 = time.perf_counter()
-        orc.forward(q, k, v, w.scale, w.causal, threads=cores)
+        orc.forward(q, k, v, w.scale, w.causal, threads=cores, window=w.window, dtype=w.dtype)
         t_used += time.perf_counter() - t0
         done_flop += per_head
         heads += 1
@@ -189,7 +189,7 @@ def run_reference(args, w, world, rank):
         k = np.ascontiguousarray(x["k"][:, :, g:g + 1])
         v = np.ascontiguousarray(x["v"][:, :, g:g + 1])
         t0 = time.perf_counter()
-        orc.forward(q, k, v, w.scale, w.causal, threads=cores)
+        orc.forward(q, k, v, w.scale, w.causal, threads=cores, window=w.window, dtype=w.dtype)
         dt = time.perf_counter() - t0
         if step >= args.warmup:
             times.append(dt)
@@ -342,13 +342,14 @@ def run_sweep(args):
     for name in names:
         w = synth.WORKLOADS[name]
         x = synth.make_inputs(w)
-        q, k, v = (torch.from_numpy(x[n].view(np.int16)).view(torch.bfloat16).cuda() for n in ("q", "k", "v"))
+        tdt = torch.float16 if w.dtype == "f16" else torch.bfloat16
+        q, k, v = (torch.from_numpy(x[n].view(np.int16)).view(tdt).cuda() for n in ("q", "k", "v"))
         out = torch.empty_like(q)
         lse = torch.empty((w.B, w.Hq, w.Nq), dtype=torch.float32, device="cuda")
         # inputs smaller than L2 are timed both warm and with an L2 flush before each launch
         flush = torch.empty(int(2 * 126e6) // 4, dtype=torch.float32, device="cuda")
         win = w.window or None
-        splits = fa.splitkv_default_splits(w.B, w.Hq, w.Nq, w.Nk, w.d, torch.cuda.get_device_properties(0).multi_processor_count) if w.splitkv else None
+        splits = fa.splitkv_default_splits(w.B, w.Hq, w.Hkv, w.Nq, w.Nk, w.d, torch.cuda.get_device_properties(0).multi_processor_count) if w.splitkv else None
         ws = torch.empty(max(1, fa.splitkv_workspace_bytes(w.B, w.Hq, w.Nq, w.d, splits)), dtype=torch.uint8, device="cuda") if splits else None
         kw = dict(window=win, num_splits=splits, workspace=ws)
         for _ in range(args.warmup):

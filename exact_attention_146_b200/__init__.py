@@ -30,7 +30,7 @@ FA_ERR_SCRATCH_LIMIT = 9
 SPLITKV_STATIC_SCRATCH_BYTES = 16 * 1024 * 1024
 
 EXPORTED = ("fa_fwd", "fa_fwd_window", "fa_fwd_splitkv", "fa_splitkv_workspace_bytes", "fa_splitkv_default_splits",
-            "fa_fwd_splitkv_static", "fa_status_string", "fa_device_status", "fa_tile_config", "fa_version")
+            "fa_fwd_splitkv_static", "fa_fwd_f16", "fa_status_string", "fa_device_status", "fa_tile_config", "fa_version")
 
 
 class FaError(RuntimeError):
@@ -52,6 +52,8 @@ def lib() -> ctypes.CDLL:
         vp, ci, cf = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
         L.fa_fwd.argtypes = [vp, vp, vp, vp, vp, ci, ci, ci, ci, ci, ci, cf, ci, vp]
         L.fa_fwd.restype = ci
+        L.fa_fwd_f16.argtypes = [vp, vp, vp, vp, vp, ci, ci, ci, ci, ci, ci, cf, ci, vp]
+        L.fa_fwd_f16.restype = ci
         L.fa_fwd_window.argtypes = [vp, vp, vp, vp, vp, ci, ci, ci, ci, ci, ci, cf, ci, vp]
         L.fa_fwd_window.restype = ci
         L.fa_fwd_splitkv.argtypes = [vp, vp, vp, vp, vp, ci, ci, ci, ci, ci, ci, cf, ci, ci, vp, ctypes.c_size_t, vp]
@@ -60,7 +62,7 @@ def lib() -> ctypes.CDLL:
         L.fa_fwd_splitkv_static.restype = ci
         L.fa_splitkv_workspace_bytes.argtypes = [ci, ci, ci, ci, ci]
         L.fa_splitkv_workspace_bytes.restype = ctypes.c_size_t
-        L.fa_splitkv_default_splits.argtypes = [ci, ci, ci, ci, ci, ci]
+        L.fa_splitkv_default_splits.argtypes = [ci, ci, ci, ci, ci, ci, ci]
         L.fa_splitkv_default_splits.restype = ci
         L.fa_status_string.argtypes = [ci]
         L.fa_status_string.restype = ctypes.c_char_p
@@ -104,14 +106,14 @@ def splitkv_workspace_bytes(B: int, Hq: int, Nq: int, d: int, num_splits: int) -
     return int(lib().fa_splitkv_workspace_bytes(int(B), int(Hq), int(Nq), int(d), int(num_splits)))
 
 
-def splitkv_default_splits(B: int, Hq: int, Nq: int, Nk: int, d: int, sm_count: int) -> int:
-    return int(lib().fa_splitkv_default_splits(int(B), int(Hq), int(Nq), int(Nk), int(d), int(sm_count)))
+def splitkv_default_splits(B: int, Hq: int, Hkv: int, Nq: int, Nk: int, d: int, sm_count: int) -> int:
+    return int(lib().fa_splitkv_default_splits(int(B), int(Hq), int(Hkv), int(Nq), int(Nk), int(d), int(sm_count)))
 
 
 def fa_fwd(q, k, v, *, causal: bool = False, scale: float | None = None, out=None, lse=None,
            return_lse: bool = True, stream=None, window: int | None = None,
            num_splits: int | None = None, workspace=None):
-    """Exact attention forward on [B, N, H, d] bf16 CUDA tensors.
+    """Exact attention forward on [B, N, H, d] bf16 (or fp16: fa_fwd_f16) CUDA tensors.
 
     q: [B, Nq, Hq, d]; k, v: [B, Nk, Hkv, d] with Hq % Hkv == 0 (GQA: query head h
     uses KV head h // (Hq // Hkv)).  Returns (out [B, Nq, Hq, d] bf16, lse [B, Hq, Nq]
@@ -122,9 +124,14 @@ def fa_fwd(q, k, v, *, causal: bool = False, scale: float | None = None, out=Non
     splitkv_workspace_bytes; allocated here if None).  Runs asynchronously on `stream`
     (default: torch's current stream)."""
     import torch
+    dt = q.dtype
+    if dt not in (torch.bfloat16, torch.float16):
+        raise ValueError(f"q must be bf16 or fp16, got {dt}")
     for name, t in (("q", q), ("k", k), ("v", v)):
-        if t.dtype != torch.bfloat16 or not t.is_cuda or not t.is_contiguous() or t.dim() != 4:
-            raise ValueError(f"{name} must be a contiguous 4-D bf16 CUDA tensor, got {t.dtype} {tuple(t.shape)}")
+        if t.dtype != dt or not t.is_cuda or not t.is_contiguous() or t.dim() != 4:
+            raise ValueError(f"{name} must be a contiguous 4-D {dt} CUDA tensor, got {t.dtype} {tuple(t.shape)}")
+    if out is not None and out.dtype != dt:
+        raise ValueError(f"out must be {dt}, got {out.dtype}")
     B, Nq, Hq, d = q.shape
     Bk, Nk, Hkv, dk = k.shape
     if v.shape != k.shape or Bk != B or dk != d:
@@ -138,7 +145,12 @@ def fa_fwd(q, k, v, *, causal: bool = False, scale: float | None = None, out=Non
     if not return_lse:
         lse = None
     lse_ptr = lse.data_ptr() if lse is not None else None
-    if num_splits is not None and num_splits > 1:
+    if dt == torch.float16:
+        if window is not None or (num_splits is not None and num_splits > 1):
+            raise ValueError("fp16 inputs take the causal or no mask, without split-KV")
+        rc = lib().fa_fwd_f16(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse_ptr,
+                              B, Hq, Hkv, Nq, Nk, d, float(scale), 1 if causal else 0, _stream_handle(stream))
+    elif num_splits is not None and num_splits > 1:
         if window is not None:
             raise ValueError("split-KV takes the causal or no mask")
         need = splitkv_workspace_bytes(B, Hq, Nq, d, num_splits)

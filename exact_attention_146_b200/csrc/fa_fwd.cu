@@ -21,16 +21,17 @@ using namespace fa;
 
 // Tiling per head dim: TileCfg<d, key rows per tile, query tiles per unit, K/V slots,
 // buffers per Q tile, S buffers per Q tile, P in TMEM columns of its own, exponential
-// pairs per 8 on the FMA pipe>.  d = 256 runs one 128-row query tile, so it has TMEM room
+// pairs per 8 on the FMA pipe, fp16 elements (H) instead of bf16>.  d = 256 runs one 128-row query tile, so it has TMEM room
 // for a second S buffer (S_{j+1} computed while the softmax works on S_j); d <= 64 has
 // room to keep P apart from S, and is where the exponentials dominate.
-using Cfg32 = TileCfg<32, 128, 2, 8, 2, 1, true, 2>;
-using Cfg64 = TileCfg<64, 128, 2, 8, 2, 1, true, 2>;
-using Cfg80 = TileCfg<80, 128, 2, 4, 1, 1>;
-using Cfg96 = TileCfg<96, 128, 2, 4, 1, 1>;
-using Cfg128 = TileCfg<128, 128, 2, 4, 1, 1>;
-using Cfg192 = TileCfg<192, 64, 2, 4, 1, 1>;
-using Cfg256 = TileCfg<256, 64, 1, 4, 1, 2>;
+template <bool H> using Cfg32 = TileCfg<32, 128, 2, 8, 2, 1, true, 2, H>;
+template <bool H> using Cfg64 = TileCfg<64, 128, 2, 8, 2, 1, true, 2, H>;
+template <bool H> using Cfg80 = TileCfg<80, 128, 2, 4, 1, 1, false, 0, H>;
+template <bool H> using Cfg96 = TileCfg<96, 128, 2, 4, 1, 1, false, 0, H>;
+template <bool H> using Cfg128 = TileCfg<128, 128, 2, 4, 1, 1, false, 0, H>;
+template <bool H> using Cfg192 = TileCfg<192, 64, 2, 4, 1, 1, false, 0, H>;
+template <bool H> using Cfg256 = TileCfg<256, 64, 1, 4, 1, 2, false, 0, H>;
+constexpr int kNumCfgSlots = 16;   // 7 head dims x 2 element types
 
 __device__ int g_fa_status;   // per-device kernel status word (0 = OK)
 
@@ -42,8 +43,8 @@ struct DeviceState {
     bool supported = false;
     int num_sms = 0;
     int *status_ptr = nullptr;
-    bool smem_attr_set[8] = {};
-    int regs_ok[8] = {};          // 0 unknown, 1 verified, -1 mismatch
+    bool smem_attr_set[kNumCfgSlots] = {};
+    int regs_ok[kNumCfgSlots] = {};   // 0 unknown, 1 verified, -1 mismatch
 };
 DeviceState g_devices[kMaxDevices];
 std::mutex g_mutex;
@@ -135,16 +136,19 @@ bool overlaps(const void *a, size_t na, const void *b, size_t nb) {
     return a0 < b0 + nb && b0 < a0 + na;
 }
 
-// 4-D view (d, H, N, B) of a [B, N, H, d] bf16 tensor, box (CW, 1, rows, 1).
-int encode_bnhd(CUtensorMap *m, const void *base, int d, int H, int N, int B, int cw, int rows) {
+// 4-D view (d, H, N, B) of a [B, N, H, d] bf16 tensor, box (CW, heads, rows, 1): the box
+// lands in shared memory as heads*rows swizzled rows, row-major over (row, head).
+int encode_bnhd(CUtensorMap *m, const void *base, int d, int H, int N, int B, int cw, int rows, int heads = 1,
+                bool f16 = false) {
     EncodeTiledFn fn = encode_fn();
     if (fn == nullptr) return FA_ERR_CUDA;
     const cuuint64_t dims[4] = {cuuint64_t(d), cuuint64_t(H), cuuint64_t(N), cuuint64_t(B)};
     const cuuint64_t strides[3] = {cuuint64_t(d) * 2, cuuint64_t(H) * d * 2, cuuint64_t(N) * H * d * 2};
-    const cuuint32_t box[4] = {cuuint32_t(cw), 1, cuuint32_t(rows), 1};
+    const cuuint32_t box[4] = {cuuint32_t(cw), cuuint32_t(heads), cuuint32_t(rows), 1};
     const cuuint32_t estr[4] = {1, 1, 1, 1};
     const CUtensorMapSwizzle sw = (cw * 2 == 128) ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
-    const CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(base), dims, strides,
+    const CUresult r = fn(m, f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4,
+                          const_cast<void *>(base), dims, strides,
                           box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS ? FA_OK : FA_ERR_CUDA;
@@ -173,6 +177,15 @@ size_t splitkv_bytes(int B, int Hq, int Nq, int d, int splits) {
     return o + size_t(splits) * size_t(B) * size_t(Hq) * size_t(Nq) * 4;
 }
 
+// GQA packing: with fewer than 128 queries, the n_rep query heads that share a KV head
+// share one unit, their rows stacked in the tile (flat row i * n_rep + r), so a decode-sized
+// Nq does not leave most of each 128-row tile empty.  Needs n_rep to divide 128 (the Q
+// load box is n_rep heads x 128 / n_rep rows).  Each row's arithmetic is unchanged.
+int pack_factor(int Hq, int Hkv, int Nq) {
+    const int n_rep = Hq / Hkv;
+    return (n_rep > 1 && kBlockQ % n_rep == 0 && Nq < kBlockQ) ? n_rep : 1;
+}
+
 template <class C>
 int launch(const Problem &pr, DeviceState &dev, int cfg_slot, cudaStream_t stream) {
     auto kern = fa_fwd_kernel<C>;
@@ -197,12 +210,14 @@ int launch(const Problem &pr, DeviceState &dev, int cfg_slot, cudaStream_t strea
     if (dev.regs_ok[cfg_slot] != 1) return FA_ERR_CUDA;
     CUtensorMap mq, mk, mv;
     int rc;
-    if ((rc = encode_bnhd(&mq, pr.q, C::D, pr.Hq, pr.Nq, pr.B, C::CW, kBlockQ)) != FA_OK) return rc;
-    if ((rc = encode_bnhd(&mk, pr.k, C::D, pr.Hkv, pr.Nk, pr.B, C::CW, C::BC)) != FA_OK) return rc;
-    if ((rc = encode_bnhd(&mv, pr.v, C::D, pr.Hkv, pr.Nk, pr.B, C::CW, C::BC)) != FA_OK) return rc;
+    const int pack = pack_factor(pr.Hq, pr.Hkv, pr.Nq);
+    if ((rc = encode_bnhd(&mq, pr.q, C::D, pr.Hq, pr.Nq, pr.B, C::CW, kBlockQ / pack, pack, C::F16)) != FA_OK)
+        return rc;
+    if ((rc = encode_bnhd(&mk, pr.k, C::D, pr.Hkv, pr.Nk, pr.B, C::CW, C::BC, 1, C::F16)) != FA_OK) return rc;
+    if ((rc = encode_bnhd(&mv, pr.v, C::D, pr.Hkv, pr.Nk, pr.B, C::CW, C::BC, 1, C::F16)) != FA_OK) return rc;
 
     FwdParams p{};
-    p.out = static_cast<__nv_bfloat16 *>(pr.out);
+    p.out = pr.out;
     p.lse = pr.lse;
     p.status = dev.status_ptr;
     p.B = pr.B;
@@ -213,13 +228,14 @@ int launch(const Problem &pr, DeviceState &dev, int cfg_slot, cudaStream_t strea
     p.n_rep = pr.Hq / pr.Hkv;
     p.causal = pr.causal;
     p.window = pr.window;
-    p.nqb = (pr.Nq + C::NQT * kBlockQ - 1) / (C::NQT * kBlockQ);
+    p.pack = pack;
+    p.nqb = (pr.Nq * pack + C::NQT * kBlockQ - 1) / (C::NQT * kBlockQ);
     const int nkv = (pr.Nk + C::BC - 1) / C::BC;
     p.num_splits = pr.num_splits > 1 ? pr.num_splits : 1;
     p.split_tiles = (nkv + p.num_splits - 1) / p.num_splits;
     p.o_part = pr.o_part;
     p.lse_part = pr.lse_part;
-    const long long units = (long long)pr.B * pr.Hq * p.nqb * p.num_splits;
+    const long long units = (long long)pr.B * (pr.Hq / pack) * p.nqb * p.num_splits;
     if (units > 0x7fffffffLL) return FA_ERR_INVALID_ARG;
     p.num_units = int(units);
     p.scale_log2 = pr.scale * 1.4426950408889634f;
@@ -231,23 +247,39 @@ int launch(const Problem &pr, DeviceState &dev, int cfg_slot, cudaStream_t strea
         const long long rows = (long long)pr.B * pr.Nq * pr.Hq;
         const long long want = (rows + 7) / 8;   // 8 rows (warps) per 256-thread block
         const int mgrid = int(want < 8LL * dev.num_sms ? want : 8LL * dev.num_sms);
-        fa_splitkv_merge_kernel<C::D><<<mgrid > 0 ? mgrid : 1, 256, 0, stream>>>(
-            pr.o_part, pr.lse_part, static_cast<__nv_bfloat16 *>(pr.out), pr.lse, pr.B, pr.Hq, pr.Nq, p.num_splits);
+        fa_splitkv_merge_kernel<C::D, C::F16><<<mgrid > 0 ? mgrid : 1, 256, 0, stream>>>(
+            pr.o_part, pr.lse_part, static_cast<uint16_t *>(pr.out), pr.lse, pr.B, pr.Hq, pr.Nq, p.num_splits);
         if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
     }
     return FA_OK;
 }
 
+// Per-head-dim launch for element type H (config slots 0-6 bf16, 8-14 fp16).
+template <bool H>
+int dispatch(const Problem &pr, DeviceState &dev, cudaStream_t st) {
+    constexpr int base = H ? 8 : 0;
+    switch (pr.d) {
+        case 32: return launch<Cfg32<H>>(pr, dev, base + 0, st);
+        case 64: return launch<Cfg64<H>>(pr, dev, base + 1, st);
+        case 80: return launch<Cfg80<H>>(pr, dev, base + 2, st);
+        case 96: return launch<Cfg96<H>>(pr, dev, base + 3, st);
+        case 128: return launch<Cfg128<H>>(pr, dev, base + 4, st);
+        case 192: return launch<Cfg192<H>>(pr, dev, base + 5, st);
+        case 256: return launch<Cfg256<H>>(pr, dev, base + 6, st);
+        default: return FA_ERR_UNSUPPORTED_HEAD_DIM;
+    }
+}
+
 int tile_config(int d, int *bq, int *bk, int *nqt, int *ns) {
     int BC, NQT, NS;
     switch (d) {
-        case 32: BC = Cfg32::BC; NQT = Cfg32::NQT; NS = Cfg32::NS; break;
-        case 64: BC = Cfg64::BC; NQT = Cfg64::NQT; NS = Cfg64::NS; break;
-        case 80: BC = Cfg80::BC; NQT = Cfg80::NQT; NS = Cfg80::NS; break;
-        case 96: BC = Cfg96::BC; NQT = Cfg96::NQT; NS = Cfg96::NS; break;
-        case 128: BC = Cfg128::BC; NQT = Cfg128::NQT; NS = Cfg128::NS; break;
-        case 192: BC = Cfg192::BC; NQT = Cfg192::NQT; NS = Cfg192::NS; break;
-        case 256: BC = Cfg256::BC; NQT = Cfg256::NQT; NS = Cfg256::NS; break;
+        case 32: BC = Cfg32<false>::BC; NQT = Cfg32<false>::NQT; NS = Cfg32<false>::NS; break;
+        case 64: BC = Cfg64<false>::BC; NQT = Cfg64<false>::NQT; NS = Cfg64<false>::NS; break;
+        case 80: BC = Cfg80<false>::BC; NQT = Cfg80<false>::NQT; NS = Cfg80<false>::NS; break;
+        case 96: BC = Cfg96<false>::BC; NQT = Cfg96<false>::NQT; NS = Cfg96<false>::NS; break;
+        case 128: BC = Cfg128<false>::BC; NQT = Cfg128<false>::NQT; NS = Cfg128<false>::NS; break;
+        case 192: BC = Cfg192<false>::BC; NQT = Cfg192<false>::NQT; NS = Cfg192<false>::NS; break;
+        case 256: BC = Cfg256<false>::BC; NQT = Cfg256<false>::NQT; NS = Cfg256<false>::NS; break;
         default: return FA_ERR_UNSUPPORTED_HEAD_DIM;
     }
     if (bq) *bq = kBlockQ;
@@ -299,7 +331,7 @@ namespace {
 // device memory of the current device), so its device-range check is skipped.
 int forward(const void *q, const void *k, const void *v, void *out, float *lse, int B, int Hq, int Hkv,
             int Nq, int Nk, int d, float scale, int causal, int window, int num_splits, void *workspace,
-            size_t workspace_bytes, void *stream, bool library_scratch = false) {
+            size_t workspace_bytes, void *stream, bool library_scratch = false, bool f16 = false) {
     // ---- host-only validation (no CUDA call before this block passes)
     if (B < 0 || Hq <= 0 || Hkv <= 0 || Nq < 0 || Nk < 0) return FA_ERR_INVALID_ARG;
     if (Hq % Hkv != 0) return FA_ERR_INVALID_ARG;
@@ -364,16 +396,7 @@ int forward(const void *q, const void *k, const void *v, void *out, float *lse, 
     }
     const Problem pr{q, k, v, out, lse, B, Hq, Hkv, Nq, Nk, d, scale, causal, window,
                      ws_bytes > 0 ? num_splits : 1, o_part, lse_part};
-    switch (d) {
-        case 32: return launch<Cfg32>(pr, *dev, 0, st);
-        case 64: return launch<Cfg64>(pr, *dev, 1, st);
-        case 80: return launch<Cfg80>(pr, *dev, 2, st);
-        case 96: return launch<Cfg96>(pr, *dev, 3, st);
-        case 128: return launch<Cfg128>(pr, *dev, 4, st);
-        case 192: return launch<Cfg192>(pr, *dev, 5, st);
-        case 256: return launch<Cfg256>(pr, *dev, 6, st);
-        default: return FA_ERR_UNSUPPORTED_HEAD_DIM;
-    }
+    return f16 ? dispatch<true>(pr, *dev, st) : dispatch<false>(pr, *dev, st);
 }
 
 }  // namespace
@@ -390,17 +413,28 @@ size_t fa_splitkv_workspace_bytes(int B, int Hq, int Nq, int d, int num_splits) 
     return splitkv_bytes(B, Hq, Nq, d, num_splits);
 }
 
-int fa_splitkv_default_splits(int B, int Hq, int Nq, int Nk, int d, int sm_count) {
+int fa_splitkv_default_splits(int B, int Hq, int Hkv, int Nq, int Nk, int d, int sm_count) {
     int bq, bk, nqt, ns;
-    if (tile_config(d, &bq, &bk, &nqt, &ns) != FA_OK || B <= 0 || Hq <= 0 || Nq <= 0 || Nk <= 0 || sm_count <= 0)
+    if (tile_config(d, &bq, &bk, &nqt, &ns) != FA_OK || B <= 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0 ||
+        Nq <= 0 || Nk <= 0 || sm_count <= 0)
         return 1;
-    const long long units = (long long)B * Hq * ((Nq + bq * nqt - 1) / (bq * nqt));
+    const int pack = pack_factor(Hq, Hkv, Nq);
+    const long long units = (long long)B * (Hq / pack) * ((Nq * pack + bq * nqt - 1) / (bq * nqt));
     if (units >= sm_count) return 1;
-    const int nkv = (Nk + bk - 1) / bk;
-    long long s = (sm_count + units - 1) / units;   // fill the SMs once
-    if (s > nkv / 4) s = nkv / 4;                    // keep >= 4 key tiles per split
-    if (s > kMaxSplits) s = kMaxSplits;
-    return s < 1 ? 1 : int(s);
+    // Cost of S splits in key-tile steps of the busiest SM: waves x (tiles per split + one
+    // step of per-unit overhead: Q load, pipeline fill, epilogue).  Keep >= 4 key tiles per
+    // split; the smallest S of equal cost wins.
+    const long long nkv = (Nk + bk - 1) / bk;
+    long long best = 1, best_cost = -1;
+    for (long long sp = 1; sp <= kMaxSplits && (sp == 1 || nkv / sp >= 4); ++sp) {
+        const long long waves = (units * sp + sm_count - 1) / sm_count;
+        const long long cost = waves * ((nkv + sp - 1) / sp + 1);
+        if (best_cost < 0 || cost < best_cost) {
+            best = sp;
+            best_cost = cost;
+        }
+    }
+    return int(best);
 }
 
 int fa_fwd_splitkv(const void *q, const void *k, const void *v, void *out, float *lse, int B, int Hq,
@@ -458,6 +492,11 @@ int fa_fwd_splitkv_static(const void *q, const void *k, const void *v, void *out
     }
     return forward(q, k, v, out, lse, B, Hq, Hkv, Nq, Nk, d, scale, causal, 0, num_splits, scratch,
                    sizeof(g_splitkv_scratch), stream, true);
+}
+
+int fa_fwd_f16(const void *q, const void *k, const void *v, void *out, float *lse, int B, int Hq, int Hkv,
+               int Nq, int Nk, int d, float scale, int causal, void *stream) {
+    return forward(q, k, v, out, lse, B, Hq, Hkv, Nq, Nk, d, scale, causal, 0, 1, nullptr, 0, stream, false, true);
 }
 
 int fa_fwd_window(const void *q, const void *k, const void *v, void *out, float *lse, int B, int Hq,

@@ -29,6 +29,7 @@
 
 #include <cstdint>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 
 #include "sm100.cuh"
 
@@ -47,14 +48,16 @@ enum WaitSite : int {
 };
 
 struct FwdParams {
-    __nv_bfloat16 *out;   // [B, Nq, Hq, d]
+    void *out;            // [B, Nq, Hq, d], bf16 or fp16 (the config's element type)
     float *lse;           // [B, Hq, Nq] or nullptr
     int *status;          // device status word
     int B, Hq, Hkv, Nq, Nk;
     int n_rep;            // Hq / Hkv
     int causal;           // 1 for the causal and the sliding-window masks
     int window;           // 0, or the sliding-window width W (keys i+Nk-Nq-W < j <= i+Nk-Nq)
-    int nqb;              // query blocks of NQT*128 rows per (b, hq)
+    int nqb;              // blocks of NQT*128 (flat) rows per (b, head group)
+    int pack;             // query heads per unit (GQA packing): 1, or n_rep when the n_rep heads
+                          // of one KV head stack their rows into the tile (flat row = i*pack + r)
     int num_splits;       // key-range splits per query block (1: no split)
     int split_tiles;      // key tiles per split
     int num_units;        // B * Hq * nqb * num_splits
@@ -64,7 +67,8 @@ struct FwdParams {
 };
 
 // Compile-time tiling for one head dimension.
-template <int D_, int BC_, int NQT_, int NS_, int NQB_ = 1, int SB_ = 1, bool PSEP_ = false, int SOFT_EXP_ = 0>
+template <int D_, int BC_, int NQT_, int NS_, int NQB_ = 1, int SB_ = 1, bool PSEP_ = false, int SOFT_EXP_ = 0,
+          bool F16_ = false>
 struct TileCfg {
     static constexpr int D = D_;        // head dim
     static constexpr int BC = BC_;      // key/value rows per tile
@@ -74,6 +78,7 @@ struct TileCfg {
     static constexpr int SB = SB_;      // S buffers per query tile (2: S_{j+1} computed during softmax j)
     static constexpr bool PSEP = PSEP_; // P in TMEM columns of its own instead of over S
     static constexpr int SOFT_EXP = SOFT_EXP_;   // exponentials on the FMA pipe: pairs per 8
+    static constexpr bool F16 = F16_;   // element type of Q, K, V, P and O: fp16, else bf16
     static constexpr int CW = (D == 32) ? 32 : 64;       // elements per swizzled smem row
     static constexpr int RB = CW * 2;                     // bytes per swizzled row (64 or 128)
     static constexpr int NCH = (D + CW - 1) / CW;         // column chunks of a tile
@@ -117,8 +122,8 @@ struct TileCfg {
     static constexpr int CONTROL_REGS = 72;
     static_assert(!REALLOC_REGS || (SOFTMAX_REGS * 32 * SOFTMAX_WARPS + CONTROL_REGS * 128 <= LAUNCH_REGS * THREADS),
                   "register split exceeds the launch budget");
-    static constexpr uint32_t IDESC_S = sm100::idesc_bf16_f32(kBlockQ, BC, 0, 0);
-    static constexpr uint32_t IDESC_O = sm100::idesc_bf16_f32(kBlockQ, D, 0, 1);
+    static constexpr uint32_t IDESC_S = sm100::idesc_f16kind_f32(kBlockQ, BC, 0, 0, F16);
+    static constexpr uint32_t IDESC_O = sm100::idesc_f16kind_f32(kBlockQ, D, 0, 1, F16);
 
     static_assert(NQT == 1 || NQT == 2, "one or two query tiles per unit");
     static_assert(NQB == 1 || NQB == 2, "one or two buffers per query tile");
@@ -142,7 +147,7 @@ struct TileCfg {
 };
 
 struct UnitInfo {
-    int b, hq, kvh, q0;
+    int b, hq, kvh, q0;   // hq: first query head of the unit; q0: first flat row (i*pack + r)
     int js[2], je[2];   // key tiles [js, je) each query tile visits (empty: js == je)
     int j_lo, j_hi;     // union of the ranges: the K/V tiles the unit loads
     int split;          // which key-range split (0 when not split)
@@ -156,7 +161,8 @@ __device__ __forceinline__ UnitInfo decode_unit(int u, const FwdParams &p) {
     UnitInfo w;
     w.split = u % p.num_splits;
     u /= p.num_splits;
-    const int bh = p.B * p.Hq;
+    const int groups = p.Hq / p.pack;   // head groups (= Hq without packing)
+    const int bh = p.B * groups;
     int qb, r;
     if (p.causal) {
         const int outer = u / bh;
@@ -166,10 +172,11 @@ __device__ __forceinline__ UnitInfo decode_unit(int u, const FwdParams &p) {
         r = u / p.nqb;
         qb = u - r * p.nqb;
     }
-    w.b = r / p.Hq;
-    w.hq = r - w.b * p.Hq;
+    w.b = r / groups;
+    w.hq = (r - w.b * groups) * p.pack;
     w.kvh = w.hq / p.n_rep;
     w.q0 = qb * (C::NQT * kBlockQ);
+    const int flat_rows = p.Nq * p.pack;
     const int nkv = (p.Nk + C::BC - 1) / C::BC;
     const int diag = p.Nk - p.Nq;    // row i sees keys up to i + diag (causal / window)
     w.j_lo = 0x7fffffff;
@@ -177,11 +184,12 @@ __device__ __forceinline__ UnitInfo decode_unit(int u, const FwdParams &p) {
 #pragma unroll
     for (int t = 0; t < 2; ++t) {
         int js = 0, je = 0;
-        const int q_lo = w.q0 + t * kBlockQ;
-        if (t < C::NQT && q_lo < p.Nq) {
+        const int f_lo = w.q0 + t * kBlockQ;
+        if (t < C::NQT && f_lo < flat_rows) {
+            const int q_lo = f_lo / p.pack;   // the tile's first and last query
             je = nkv;
             if (p.causal) {
-                const int q_hi = min(q_lo + kBlockQ - 1, p.Nq - 1);
+                const int q_hi = min(f_lo + kBlockQ - 1, flat_rows - 1) / p.pack;
                 const int lim = q_hi + diag;   // last visible key of the tile's last row
                 je = lim < 0 ? 0 : min(nkv, lim / C::BC + 1);
             }
@@ -280,7 +288,8 @@ __device__ void producer_role(const CUtensorMap *tm_q, const CUtensorMap *tm_k, 
             const uint32_t dst = sbase + C::SMEM_Q + (t * C::NQB + qb) * C::Q_TILE;
 #pragma unroll
             for (int c = 0; c < C::NCH; ++c)
-                sm100::tma_load_4d_elected(dst + c * C::Q_CHUNK, tm_q, fb, c * C::CW, w.hq, w.q0 + t * kBlockQ, w.b);
+                sm100::tma_load_4d_elected(dst + c * C::Q_CHUNK, tm_q, fb, c * C::CW, w.hq,
+                                           (w.q0 + t * kBlockQ) / p.pack, w.b);
         }
         for (int j = w.j_lo; ok && j < w.j_hi; ++j) {
 #pragma unroll
@@ -484,13 +493,13 @@ __device__ void mma_role(const FwdParams &p, uint32_t sbase, uint32_t tmem, cons
 
 // ------------------------------------------------------------------ softmax / epilogue
 
-// p = 2^(s * c_log2 - m) for one row of a score tile, packed to bf16 pairs and stored
+// p = 2^(s * c_log2 - m) for one row of a score tile, packed to bf16 (F16: fp16) pairs and stored
 // to BC/2 TMEM columns at p_taddr (over the S tile itself, or P's own columns); returns
 // the fp32 row sum of p.  On unmasked tiles SOFT_EXP of every 8 pairs take the FMA-pipe
 // exponential to relieve the special-function unit (worth it where the exponentials
 // dominate, i.e. small head dims); masked tiles (which may hold -inf scores) use the
 // hardware ex2 throughout.
-template <int BC, int SOFT_EXP, bool MIXED>
+template <int BC, int SOFT_EXP, bool MIXED, bool F16>
 __device__ __forceinline__ float exp_pack_store(const uint32_t (&s)[BC], float c_log2, float neg_m,
                                                 uint32_t p_taddr) {
     const uint64_t c2 = sm100::pack2(c_log2, c_log2);
@@ -516,7 +525,7 @@ __device__ __forceinline__ float exp_pack_store(const uint32_t (&s)[BC], float c
             else acc0 = sm100::add2(acc0, p2);
             float lo, hi;
             sm100::unpack2(p2, lo, hi);
-            pk[i] = sm100::pack_bf16x2(lo, hi);
+            pk[i] = sm100::pack_x2<F16>(lo, hi);
         }
         sm100::tmem_st32(p_taddr + uint32_t(32 * c), pk);
     }
@@ -545,13 +554,16 @@ __device__ void softmax_role(const FwdParams &p, uint32_t sbase, uint32_t tmem, 
         const UnitInfo w = decode_unit<C>(u, p);
         const int js = w.js[t], je = w.je[t];
         const int nk = je - js;
-        const int q_lo = w.q0 + t * kBlockQ;
-        const int row = q_lo + row_in_tile;
+        const int f_lo = w.q0 + t * kBlockQ;       // flat row f = i * pack + (hq - w.hq)
+        const int q_lo = f_lo / p.pack;            // the tile's first query
+        const int f_row = f_lo + row_in_tile;
+        const int row = f_row / p.pack;            // this thread's query i and head hq
+        const int hq = w.hq + (f_row - row * p.pack);
         const int diag = p.Nk - p.Nq;              // causal: key j visible to row i iff j <= i + diag
         const int row_lim = p.causal ? row + diag : 0x7fffffff;
         // sliding window: keys j > i + diag - W; the tile's first row has the lowest bound
         const int row_lo = p.window > 0 ? row + diag - p.window + 1 : -0x7fffffff;
-        const int tile_lo_hi = p.window > 0 ? q_lo + kBlockQ - 1 + diag - p.window + 1 : -0x7fffffff;
+        const int tile_lo_hi = p.window > 0 ? q_lo + kBlockQ / p.pack - 1 + diag - p.window + 1 : -0x7fffffff;
         float m_ref = -INFINITY;                   // reference max, log2 units (scaled)
         float l = 0.f;                             // running sum of 2^(s*c - m_ref)
 
@@ -600,8 +612,8 @@ __device__ void softmax_role(const FwdParams &p, uint32_t sbase, uint32_t tmem, 
                     need_rescale = true;
                 }
                 const float neg_m = (m_ref == -INFINITY) ? 0.f : -m_ref;
-                row_sum = need_mask ? exp_pack_store<BC, C::SOFT_EXP, false>(s, c_log2, neg_m, p_taddr)
-                                    : exp_pack_store<BC, C::SOFT_EXP, true>(s, c_log2, neg_m, p_taddr);
+                row_sum = need_mask ? exp_pack_store<BC, C::SOFT_EXP, false, C::F16>(s, c_log2, neg_m, p_taddr)
+                                    : exp_pack_store<BC, C::SOFT_EXP, true, C::F16>(s, c_log2, neg_m, p_taddr);
             }
             l = l * alpha + row_sum;
 
@@ -634,9 +646,9 @@ __device__ void softmax_role(const FwdParams &p, uint32_t sbase, uint32_t tmem, 
         {
             const float inv_l = l > 0.f ? 1.f / l : 0.f;
             const bool store = row < p.Nq;
-            const size_t row_off = (size_t(w.b) * p.Nq + size_t(row)) * p.Hq + w.hq;   // [b][row][hq]
+            const size_t row_off = (size_t(w.b) * p.Nq + size_t(row)) * p.Hq + hq;   // [b][row][hq]
             const bool split_mode = p.num_splits > 1;
-            __nv_bfloat16 *orow = p.out + row_off * C::D;
+            uint16_t *orow = static_cast<uint16_t *>(p.out) + row_off * C::D;
             float *prow = split_mode ? p.o_part + (size_t(w.split) * p.B * p.Nq * p.Hq + row_off) * C::D : nullptr;
 #pragma unroll
             for (int c = 0; c < C::O_CHUNKS; ++c) {
@@ -664,7 +676,7 @@ __device__ void softmax_role(const FwdParams &p, uint32_t sbase, uint32_t tmem, 
                 uint32_t pk[16];
 #pragma unroll
                 for (int i = 0; i < 16; ++i)
-                    pk[i] = sm100::pack_bf16x2(__uint_as_float(o[2 * i]) * inv_l, __uint_as_float(o[2 * i + 1]) * inv_l);
+                    pk[i] = sm100::pack_x2<C::F16>(__uint_as_float(o[2 * i]) * inv_l, __uint_as_float(o[2 * i + 1]) * inv_l);
                 if (store) {
 #pragma unroll
                     for (int v4 = 0; v4 < 4; ++v4) {
@@ -678,7 +690,7 @@ __device__ void softmax_role(const FwdParams &p, uint32_t sbase, uint32_t tmem, 
             sm100::tc_fence_before_sync();
             sm100::mbar_arrive(bar(C::B_OEMPTY + t));
             const float lse_row = l > 0.f ? (m_ref + log2f(l)) * 0.6931471805599453f : -INFINITY;
-            const size_t lse_off = (size_t(w.b) * p.Hq + w.hq) * p.Nq + row;
+            const size_t lse_off = (size_t(w.b) * p.Hq + hq) * p.Nq + row;
             if (split_mode) {
                 if (store) p.lse_part[size_t(w.split) * p.B * p.Hq * p.Nq + lse_off] = lse_row;
             } else if (p.lse != nullptr && store) {
@@ -760,9 +772,9 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
 // Split-KV merge: one warp per output row (b, i, hq).  With m = max_s LSE_s, the weights
 // w_s = e^(LSE_s - m) combine the per-split normalised outputs O = sum_s w_s O_s / sum_s w_s,
 // and LSE = m + ln sum_s w_s; a row no split saw (all LSE_s = -inf) gets O = 0, LSE = -inf.
-template <int D>
+template <int D, bool F16>
 __global__ void __launch_bounds__(256) fa_splitkv_merge_kernel(const float *o_part, const float *lse_part,
-                                                               __nv_bfloat16 *out, float *lse, int B, int Hq,
+                                                               uint16_t *out, float *lse, int B, int Hq,
                                                                int Nq, int num_splits) {
     constexpr int PER_LANE = (D + 31) / 32;
     const long rows = long(B) * Nq * Hq;
@@ -798,7 +810,10 @@ __global__ void __launch_bounds__(256) fa_splitkv_merge_kernel(const float *o_pa
 #pragma unroll
         for (int e = 0; e < PER_LANE; ++e) {
             const int col = lane + 32 * e;
-            if (col < D) out[r * D + col] = __float2bfloat16_rn(acc[e] * inv);
+            if (col < D) {
+                if constexpr (F16) out[r * D + col] = __half_as_ushort(__float2half_rn(acc[e] * inv));
+                else out[r * D + col] = __bfloat16_as_ushort(__float2bfloat16_rn(acc[e] * inv));
+            }
         }
         if (lse != nullptr && lane == 0) lse[lse_off] = wsum > 0.f ? m + logf(wsum) : -INFINITY;
     }

@@ -179,12 +179,15 @@ __device__ __forceinline__ void mma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, ui
         : "memory");
 }
 
-// Instruction descriptor of kind::f16 with bf16 A/B and an fp32 accumulator:
-// bits 4-5 D format (1 = f32), 7-9 A format (1 = bf16), 10-12 B format (1 = bf16),
-// 15 A major, 16 B major (0 = K-major, 1 = MN-major), 17-22 N >> 3, 24-28 M >> 4.
-__host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, int a_mn_major, int b_mn_major) {
-    return (1u << 4) | (1u << 7) | (1u << 10) | (uint32_t(a_mn_major) << 15) |
-           (uint32_t(b_mn_major) << 16) | (uint32_t(N >> 3) << 17) | (uint32_t(M >> 4) << 24);
+// Instruction descriptor of kind::f16 with an fp32 accumulator: bits 4-5 D format
+// (1 = f32), 7-9 A format and 10-12 B format (0 = f16, 1 = bf16; A and B always get the
+// same one here), 15 A major, 16 B major (0 = K-major, 1 = MN-major), 17-22 N >> 3,
+// 24-28 M >> 4.
+__host__ __device__ constexpr uint32_t idesc_f16kind_f32(int M, int N, int a_mn_major, int b_mn_major,
+                                                         bool f16_inputs) {
+    return (1u << 4) | ((f16_inputs ? 0u : 1u) << 7) | ((f16_inputs ? 0u : 1u) << 10) |
+           (uint32_t(a_mn_major) << 15) | (uint32_t(b_mn_major) << 16) | (uint32_t(N >> 3) << 17) |
+           (uint32_t(M >> 4) << 24);
 }
 
 // Shared-memory matrix descriptor: start address, leading/stride byte offsets (all
@@ -324,6 +327,19 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     uint32_t w;
     asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(w) : "f"(hi), "f"(lo));
     return w;
+}
+
+// The same with two IEEE fp16 values (round to nearest even).
+__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
+    uint32_t w;
+    asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(w) : "f"(hi), "f"(lo));
+    return w;
+}
+
+template <bool F16>
+__device__ __forceinline__ uint32_t pack_x2(float lo, float hi) {
+    if constexpr (F16) return pack_f16x2(lo, hi);
+    else return pack_bf16x2(lo, hi);
 }
 
 // ------------------------------------------------------------------ packed fp32 pairs

@@ -20,6 +20,10 @@
  * The head dimensions are those listed on the datacanvas.csdn.net head-dim article
  * (32, 64, 96, 128, 192, 256, plus 80 added by the custom-compile workaround).
  *
+ * With fewer than 128 queries and n_rep = Hq / Hkv > 1 dividing 128, the n_rep query heads
+ * of one KV head share a work unit (their rows stacked in one 128-row tile), so decode-sized
+ * Nq keeps the tiles full; the results are the same.
+ *
  * Conventions for every entry point:
  *  - All tensors are dense, row-major (C-contiguous), owned by the caller; the library
  *    allocates no device memory per call and keeps no pointer after it returns.
@@ -79,6 +83,19 @@ int fa_fwd(const void *q, const void *k, const void *v, void *out, float *lse,
            void *stream);
 
 /*
+ * fa_fwd_f16 -- fa_fwd on IEEE fp16 tensors: q, k, v and out are fp16 instead of bf16
+ * (lse stays fp32).  The dtype choice between fp16 and bf16 is the one the
+ * hwcomputing.csdn.net FlashAttention article weighs ("performance tuning", item on data
+ * types: fp16 has the finer mantissa, bf16 the range).  The tensor cores multiply fp16 x
+ * fp16 with fp32 accumulation; P is rounded to fp16 before P V and O to fp16 at the end
+ * (|O| <= max |V|, so O cannot overflow when V is finite).  Arguments, layouts, ownership
+ * and errors as fa_fwd.
+ */
+int fa_fwd_f16(const void *q, const void *k, const void *v, void *out, float *lse,
+               int B, int Hq, int Hkv, int Nq, int Nk, int d, float scale, int causal,
+               void *stream);
+
+/*
  * fa_fwd_window -- exact attention forward with a sliding-window (local) causal mask:
  * query row i sees the `window` keys ending at its causal diagonal,
  *
@@ -109,8 +126,9 @@ int fa_fwd_window(const void *q, const void *k, const void *v, void *out, float 
  *
  * fa_splitkv_workspace_bytes: device bytes the workspace needs (0 for num_splits == 1);
  *   0 also for invalid sizes.
- * fa_splitkv_default_splits: a split count that fills sm_count SMs once (1 when the
- *   plain forward already does), keeping at least four key tiles per slice.
+ * fa_splitkv_default_splits: a split count for sm_count SMs: 1 when the plain forward
+ *   already has a unit per SM, else the count with the fewest key-tile steps on the busiest
+ *   SM (waves x tiles per slice, plus one step per unit), keeping >= 4 key tiles per slice.
  * fa_fwd_splitkv: as fa_fwd (causal in {0, 1}), plus 1 <= num_splits <= 256 and a
  *   caller-owned device workspace of at least fa_splitkv_workspace_bytes bytes, 256-byte
  *   aligned, not overlapping any tensor (FA_ERR_INVALID_ARG / FA_ERR_MISALIGNED /
@@ -119,7 +137,7 @@ int fa_fwd_window(const void *q, const void *k, const void *v, void *out, float 
  *   num_splits == 1 needs no workspace and is fa_fwd.
  */
 size_t fa_splitkv_workspace_bytes(int B, int Hq, int Nq, int d, int num_splits);
-int fa_splitkv_default_splits(int B, int Hq, int Nq, int Nk, int d, int sm_count);
+int fa_splitkv_default_splits(int B, int Hq, int Hkv, int Nq, int Nk, int d, int sm_count);
 int fa_fwd_splitkv(const void *q, const void *k, const void *v, void *out, float *lse,
                    int B, int Hq, int Hkv, int Nq, int Nk, int d, float scale, int causal,
                    int num_splits, void *workspace, size_t workspace_bytes, void *stream);

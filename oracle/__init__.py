@@ -51,13 +51,13 @@ class Oracle:
         lib = ctypes.CDLL(str(path))
         ci, cd, cl = ctypes.c_int, ctypes.c_double, ctypes.c_long
         lib.oracle_attention_fwd.argtypes = [_u16p, _u16p, _u16p, _f64p, _f64p,
-                                             ci, ci, ci, ci, ci, ci, cd, ci, ci, ci]
+                                             ci, ci, ci, ci, ci, ci, cd, ci, ci, ci, ci]
         lib.oracle_attention_fwd.restype = ci
         lib.oracle_attention_probs.argtypes = [_u16p, _u16p, _u16p, _f64p, _f64p, _f64p,
-                                               ci, ci, ci, ci, ci, ci, cd, ci, ci]
+                                               ci, ci, ci, ci, ci, ci, cd, ci, ci, ci]
         lib.oracle_attention_probs.restype = ci
         lib.oracle_attention_rows.argtypes = [_u16p, _u16p, _u16p, _i32p, cl, _f64p, _f64p,
-                                              ci, ci, ci, ci, ci, ci, cd, ci, ci, ci]
+                                              ci, ci, ci, ci, ci, ci, cd, ci, ci, ci, ci]
         lib.oracle_attention_rows.restype = ci
         self.lib = lib
 
@@ -70,32 +70,41 @@ class Oracle:
             raise ValueError(f"shape mismatch q{q.shape} k{k.shape} v{v.shape}")
         return q, k, v, B, Hq, Hkv, Nq, Nk, d
 
-    def forward(self, q, k, v, scale: float, causal: bool, threads: int | None = None, window: int = 0):
-        """O [B,Nq,Hq,d] and LSE [B,Hq,Nq] in fp64 from bf16 bit-pattern inputs
-        (window = W >= 1: sliding window of the W keys ending at the causal diagonal)."""
+    @staticmethod
+    def _elem(dtype: str) -> int:
+        if dtype not in ("bf16", "f16"):
+            raise ValueError(f"dtype must be 'bf16' or 'f16', got {dtype!r}")
+        return 1 if dtype == "f16" else 0
+
+    def forward(self, q, k, v, scale: float, causal: bool, threads: int | None = None, window: int = 0,
+                dtype: str = "bf16"):
+        """O [B,Nq,Hq,d] and LSE [B,Hq,Nq] in fp64 from bf16 (dtype="f16": IEEE fp16)
+        bit-pattern inputs (window = W >= 1: sliding window of the W keys ending at the
+        causal diagonal)."""
         q, k, v, B, Hq, Hkv, Nq, Nk, d = self._dims(q, k, v)
         out = np.zeros((B, Nq, Hq, d), dtype=np.float64)
         lse = np.zeros((B, Hq, Nq), dtype=np.float64)
         rc = self.lib.oracle_attention_fwd(q, k, v, out, lse, B, Hq, Hkv, Nq, Nk, d,
-                                           float(scale), int(bool(causal)), int(window),
+                                           float(scale), int(bool(causal)), int(window), self._elem(dtype),
                                            threads or os.cpu_count() or 1)
         if rc != 0:
             raise RuntimeError(f"oracle_attention_fwd failed: {rc}")
         return out, lse
 
-    def probs(self, q, k, v, scale: float, causal: bool, window: int = 0):
+    def probs(self, q, k, v, scale: float, causal: bool, window: int = 0, dtype: str = "bf16"):
         """(O, LSE, P) with P [B,Hq,Nq,Nk]; for tiny problems."""
         q, k, v, B, Hq, Hkv, Nq, Nk, d = self._dims(q, k, v)
         out = np.zeros((B, Nq, Hq, d), dtype=np.float64)
         lse = np.zeros((B, Hq, Nq), dtype=np.float64)
         P = np.zeros((B, Hq, Nq, Nk), dtype=np.float64)
         rc = self.lib.oracle_attention_probs(q, k, v, out, lse, P, B, Hq, Hkv, Nq, Nk, d,
-                                             float(scale), int(bool(causal)), int(window))
+                                             float(scale), int(bool(causal)), int(window), self._elem(dtype))
         if rc != 0:
             raise RuntimeError(f"oracle_attention_probs failed: {rc}")
         return out, lse, P
 
-    def rows(self, q, k, v, rows, scale: float, causal: bool, threads: int | None = None, window: int = 0):
+    def rows(self, q, k, v, rows, scale: float, causal: bool, threads: int | None = None, window: int = 0,
+             dtype: str = "bf16"):
         """O [n,d] and LSE [n] of the listed (b, hq, i) rows."""
         q, k, v, B, Hq, Hkv, Nq, Nk, d = self._dims(q, k, v)
         rows = np.ascontiguousarray(np.asarray(rows, dtype=np.int32).reshape(-1, 3))
@@ -103,7 +112,7 @@ class Oracle:
         out = np.zeros((n, d), dtype=np.float64)
         lse = np.zeros((n,), dtype=np.float64)
         rc = self.lib.oracle_attention_rows(q, k, v, rows, n, out, lse, B, Hq, Hkv, Nq, Nk, d,
-                                            float(scale), int(bool(causal)), int(window),
+                                            float(scale), int(bool(causal)), int(window), self._elem(dtype),
                                             threads or os.cpu_count() or 1)
         if rc != 0:
             raise RuntimeError(f"oracle_attention_rows failed: {rc}")

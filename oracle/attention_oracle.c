@@ -35,8 +35,9 @@
  *  - a row with no visible key (only possible when Nq > Nk under the causal mask,
  *    or Nk == 0) has O = 0 and LSE = -inf, the limit of an empty sum;
  *  - LSE is the natural-log log-sum-exp of the scaled, masked logits;
- *  - inputs are bf16 bit patterns, widened exactly to fp64; nothing is rounded
- *    in between.
+ *  - inputs are bf16 (or, for the fp16 variant of the "performance tuning" data-type
+ *    item of the same article, IEEE binary16) bit patterns, widened exactly to fp64;
+ *    nothing is rounded in between.
  *
  * Softmax is taken in two passes over the materialised row (row max M_i first,
  * then exp(S_ij - M_i)), the textbook way to keep exp() in range.
@@ -63,13 +64,33 @@ static double bf16_bits_to_double(uint16_t bits) {
     return (double)f;
 }
 
+/* IEEE 754 binary16: 1 sign bit, 5 exponent bits (bias 15), 10 fraction bits;
+ * exponent 0 is subnormal (fraction * 2^-24), exponent 31 is inf/NaN. */
+static double f16_bits_to_double(uint16_t bits) {
+    const int e = (bits >> 10) & 0x1f, frac = bits & 0x3ff;
+    double mag;
+    if (e == 0) mag = ldexp((double)frac, -24);
+    else if (e == 31) mag = frac ? NAN : INFINITY;
+#ifdef ORACLE_PLANT_F16_BIAS
+    else mag = ldexp((double)(1024 + frac), e - 24);
+#else
+    else mag = ldexp((double)(1024 + frac), e - 25);
+#endif
+    return (bits & 0x8000) ? -mag : mag;
+}
+
 typedef struct {
     const uint16_t *q, *k, *v;
     int B, Hq, Hkv, Nq, Nk, d;
     double scale;
     int causal;
     int window;     /* 0: no window; W >= 1: sliding window of W keys (implies causal) */
+    int elem_f16;   /* inputs are fp16 (1) or bf16 (0) bit patterns */
 } problem_t;
+
+static double elem(const problem_t *p, uint16_t bits) {
+    return p->elem_f16 ? f16_bits_to_double(bits) : bf16_bits_to_double(bits);
+}
 
 static int kv_head_of(const problem_t *p, int hq) {
 #ifdef ORACLE_PLANT_GQA_MODULO
@@ -97,16 +118,16 @@ static int key_visible(const problem_t *p, int i, int j) {
 }
 
 static double q_at(const problem_t *p, int b, int i, int h, int c) {
-    return bf16_bits_to_double(p->q[(((size_t)b * p->Nq + i) * p->Hq + h) * p->d + c]);
+    return elem(p, p->q[(((size_t)b * p->Nq + i) * p->Hq + h) * p->d + c]);
 }
 static double k_at(const problem_t *p, int b, int j, int g, int c) {
-    return bf16_bits_to_double(p->k[(((size_t)b * p->Nk + j) * p->Hkv + g) * p->d + c]);
+    return elem(p, p->k[(((size_t)b * p->Nk + j) * p->Hkv + g) * p->d + c]);
 }
 static double v_at(const problem_t *p, int b, int j, int g, int c) {
 #ifdef ORACLE_PLANT_TRANSPOSE_V
     c = p->d - 1 - c;
 #endif
-    return bf16_bits_to_double(p->v[(((size_t)b * p->Nk + j) * p->Hkv + g) * p->d + c]);
+    return elem(p, p->v[(((size_t)b * p->Nk + j) * p->Hkv + g) * p->d + c]);
 }
 
 /*
@@ -233,15 +254,15 @@ static int run_full(const problem_t *p, double *out, double *lse, double *probs,
 
 /*
  * oracle_attention_fwd: the whole forward.
- *   q [B,Nq,Hq,d], k/v [B,Nk,Hkv,d]: bf16 bit patterns (host memory).
+ *   q [B,Nq,Hq,d], k/v [B,Nk,Hkv,d]: bf16 (elem_f16 = 0) or fp16 (1) bit patterns (host memory).
  *   causal in {0,1}; window = 0 (none) or W >= 1 keys (sliding window, causal).
  *   out [B,Nq,Hq,d] fp64, lse [B,Hq,Nq] fp64 (natural log).
  * Returns 0, or a negative code (bad sizes, no memory, thread failure).
  */
 int oracle_attention_fwd(const uint16_t *q, const uint16_t *k, const uint16_t *v,
                          double *out, double *lse, int B, int Hq, int Hkv, int Nq, int Nk,
-                         int d, double scale, int causal, int window, int nthreads) {
-    problem_t p = {q, k, v, B, Hq, Hkv, Nq, Nk, d, scale, causal ? 1 : 0, window};
+                         int d, double scale, int causal, int window, int elem_f16, int nthreads) {
+    problem_t p = {q, k, v, B, Hq, Hkv, Nq, Nk, d, scale, causal ? 1 : 0, window, elem_f16 ? 1 : 0};
     return run_full(&p, out, lse, NULL, nthreads);
 }
 
@@ -251,8 +272,8 @@ int oracle_attention_fwd(const uint16_t *q, const uint16_t *k, const uint16_t *v
  */
 int oracle_attention_probs(const uint16_t *q, const uint16_t *k, const uint16_t *v,
                            double *out, double *lse, double *probs, int B, int Hq, int Hkv,
-                           int Nq, int Nk, int d, double scale, int causal, int window) {
-    problem_t p = {q, k, v, B, Hq, Hkv, Nq, Nk, d, scale, causal ? 1 : 0, window};
+                           int Nq, int Nk, int d, double scale, int causal, int window, int elem_f16) {
+    problem_t p = {q, k, v, B, Hq, Hkv, Nq, Nk, d, scale, causal ? 1 : 0, window, elem_f16 ? 1 : 0};
     return run_full(&p, out, lse, probs, 1);
 }
 
@@ -287,8 +308,8 @@ static void *rows_worker(void *arg) {
 int oracle_attention_rows(const uint16_t *q, const uint16_t *k, const uint16_t *v,
                           const int32_t *rows, long nrows, double *out_rows, double *lse_rows,
                           int B, int Hq, int Hkv, int Nq, int Nk, int d, double scale,
-                          int causal, int window, int nthreads) {
-    problem_t p = {q, k, v, B, Hq, Hkv, Nq, Nk, d, scale, causal ? 1 : 0, window};
+                          int causal, int window, int elem_f16, int nthreads) {
+    problem_t p = {q, k, v, B, Hq, Hkv, Nq, Nk, d, scale, causal ? 1 : 0, window, elem_f16 ? 1 : 0};
     if (!check_problem(&p) || nrows < 0) return ORACLE_EINVAL;
     for (long r = 0; r < nrows; ++r) {
         int b = rows[3 * r], hq = rows[3 * r + 1], i = rows[3 * r + 2];

@@ -118,6 +118,7 @@ class Workload:
     seed: int = 0
     window: int = 0          # sliding window of W keys (0: none; implies causal)
     splitkv: bool = False    # run with the library's default split-KV count (decode shapes)
+    dtype: str = "bf16"      # element type of q, k, v and out: "bf16" or "f16" (IEEE half)
 
     @property
     def scale(self) -> float:
@@ -146,8 +147,23 @@ class Workload:
         return replace(self, **kw)
 
 
+def f32_to_f16_bits(x: np.ndarray) -> np.ndarray:
+    """fp32 -> IEEE half, round to nearest even (numpy's cast), as uint16 bit patterns."""
+    return np.asarray(x, dtype=np.float32).astype(np.float16).view(np.uint16)
+
+
 def make_inputs(w: Workload) -> dict[str, np.ndarray]:
-    """Seeded bf16 bit patterns for q [B,Nq,Hq,d], k and v [B,Nk,Hkv,d]."""
+    """Seeded bf16 (w.dtype "f16": IEEE half) bit patterns for q [B,Nq,Hq,d], k and v
+    [B,Nk,Hkv,d].  The fp16 inputs are the same normal draws rounded to half, with the
+    power-of-two multipliers applied before rounding (exact either way)."""
+    if w.dtype == "f16":
+        shapes = {"q": (w.B, w.Nq, w.Hq, w.d), "k": (w.B, w.Nk, w.Hkv, w.d), "v": (w.B, w.Nk, w.Hkv, w.d)}
+        out = {}
+        for name, shp in shapes.items():
+            z = normal_f64(stream_key(w.seed, w.wid, TENSOR_IDS[name]), int(np.prod(shp)))
+            mult = {"q": w.q_mult, "k": w.k_mult}.get(name, 1.0)
+            out[name] = f32_to_f16_bits(z.astype(np.float32) * np.float32(mult)).reshape(shp)
+        return out
     shapes = {"q": (w.B, w.Nq, w.Hq, w.d), "k": (w.B, w.Nk, w.Hkv, w.d), "v": (w.B, w.Nk, w.Hkv, w.d)}
     out = {}
     for name, shp in shapes.items():
@@ -186,6 +202,9 @@ for _w in [
     _wl("hdim256_b2_n4096_h16", 16, 2, 16, 4096, 256),
     _wl("window4k_long16k_b1_h32_d128", 17, 1, 32, 16384, 128, causal=True, window=4096),
     _wl("decode_b4_hq32_hkv8_nq16_nk32k_d128", 18, 4, 32, 16, 128, Hkv=8, Nk=32768, splitkv=True),
+    _wl("seq4096_b8_h32_d128_f16", 19, 8, 32, 4096, 128, dtype="f16"),
+    _wl("gqa_prefill_b4_n4096_hq32_hkv8_d128_causal_f16", 20, 4, 32, 4096, 128, causal=True, Hkv=8, k_mult=0.5,
+        dtype="f16"),
 ]:
     WORKLOADS[_w.name] = _w
 

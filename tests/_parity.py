@@ -15,8 +15,9 @@ TOL_O_REL_L2 = 5e-3
 TOL_LSE = 1e-3
 
 
-def to_device(bits, torch):
-    return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).cuda()
+def to_device(bits, torch, dtype="bf16"):
+    tdt = torch.float16 if dtype == "f16" else torch.bfloat16
+    return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(tdt).cuda()
 
 
 def bf16_to_f64(t):
@@ -24,11 +25,12 @@ def bf16_to_f64(t):
     return t.float().cpu().numpy().astype(np.float64)
 
 
-def run_cuda(x, scale, causal, with_lse=True, canary=True, window=None, num_splits=None):
-    """fa_fwd through the C ABI; out/lse pre-filled with NaN so unwritten rows show up."""
+def run_cuda(x, scale, causal, with_lse=True, canary=True, window=None, num_splits=None, dtype="bf16"):
+    """fa_fwd (fa_fwd_f16 for dtype "f16") through the C ABI; out/lse pre-filled with NaN
+    so unwritten rows show up."""
     import torch
     import exact_attention_146_b200 as fa
-    q, k, v = (to_device(x[n], torch) for n in ("q", "k", "v"))
+    q, k, v = (to_device(x[n], torch, dtype) for n in ("q", "k", "v"))
     out = torch.full_like(q, float("nan")) if canary else torch.empty_like(q)
     B, Nq, Hq, d = q.shape
     lse = torch.full((B, Hq, Nq), float("nan"), dtype=torch.float32, device="cuda") if with_lse else None
@@ -66,7 +68,7 @@ def workload_splits(w: synth.Workload) -> int | None:
     if not w.splitkv:
         return None
     import exact_attention_146_b200 as fa
-    return fa.splitkv_default_splits(w.B, w.Hq, w.Nq, w.Nk, w.d, 148)
+    return fa.splitkv_default_splits(w.B, w.Hq, w.Hkv, w.Nq, w.Nk, w.d, 148)
 
 
 def sample_rows(w: synth.Workload, n: int, seed: int = 0):

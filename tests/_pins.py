@@ -26,12 +26,14 @@ import synth
 TOL = 1e-12
 
 
-def bits_f64(bits):
+def bits_f64(bits, dtype="bf16"):
+    if dtype == "f16":   # numpy's own IEEE half, widened (exact)
+        return np.asarray(bits, dtype=np.uint16).view(np.float16).astype(np.float64)
     return synth.bf16_bits_to_f32(bits).astype(np.float64)
 
 
-def tiny_inputs(B, Hq, Hkv, Nq, Nk, d, seed, q_mult=1.0):
-    w = synth.Workload("tiny", 1000 + seed, B, Hq, Hkv, Nq, Nk, d, False, q_mult=q_mult, seed=seed)
+def tiny_inputs(B, Hq, Hkv, Nq, Nk, d, seed, q_mult=1.0, dtype="bf16"):
+    w = synth.Workload("tiny", 1000 + seed, B, Hq, Hkv, Nq, Nk, d, False, q_mult=q_mult, seed=seed, dtype=dtype)
     return synth.make_inputs(w)
 
 
@@ -46,10 +48,10 @@ def visible(i, j, Nq, Nk, causal, window=0):
 
 # ---------------------------------------------------------------- brute force
 
-def brute_force_decimal(x, scale, causal, prec=40, window=0):
+def brute_force_decimal(x, scale, causal, prec=40, window=0, dtype="bf16"):
     """O and LSE by the definition in `prec`-digit decimal arithmetic (tiny inputs)."""
     getcontext().prec = prec
-    q, k, v = (bits_f64(x[n]) for n in ("q", "k", "v"))
+    q, k, v = (bits_f64(x[n], dtype) for n in ("q", "k", "v"))
     B, Nq, Hq, d = q.shape
     _, Nk, Hkv, _ = k.shape
     rep = Hq // Hkv
@@ -364,3 +366,42 @@ def pin_window_online_recurrence(orc):
 WINDOW_PINS = [pin_window_brute_force, pin_window_one_key, pin_window_wide_is_causal,
                pin_window_row_is_segment, pin_window_online_recurrence]
 ALL_PINS = ALL_PINS + WINDOW_PINS
+
+
+# ---------------------------------------------------------------- fp16 inputs
+
+def pin_f16_decode_every_pattern(orc):
+    """One key: O = v exactly, so every finite IEEE half pattern placed in v must come back
+    as numpy's float16 value (normals, subnormals, both zeros, both signs)."""
+    pats = np.arange(65536, dtype=np.uint32).astype(np.uint16)
+    pats = pats[((pats >> 10) & 0x1F) != 0x1F]            # drop inf / NaN
+    d = pats.size
+    z = np.zeros((1, 1, 1, d), np.uint16)
+    O, L = orc.forward(z, z, pats.reshape(1, 1, 1, d), 1.0, False, dtype="f16")
+    assert np.array_equal(O[0, 0, 0], pats.view(np.float16).astype(np.float64)), "fp16 decode"
+    assert L[0, 0, 0] == 0.0
+
+
+def pin_f16_known_values(orc):
+    """IEEE binary16 values fixed by the format: 1, -2, the largest finite 65504, the
+    smallest normal 2^-14, the smallest subnormal 2^-24, and 1/3 rounded (1365/4096)."""
+    table = {0x3C00: 1.0, 0xC000: -2.0, 0x7BFF: 65504.0, 0x0400: 2.0 ** -14, 0x0001: 2.0 ** -24,
+             0x3555: 1365 / 4096, 0x8000: -0.0}
+    v = np.array(list(table), dtype=np.uint16).reshape(1, 1, 1, -1)
+    z = np.zeros_like(v)
+    O, _ = orc.forward(z, z, v, 1.0, False, dtype="f16")
+    assert list(O[0, 0, 0]) == list(table.values()), O[0, 0, 0]
+
+
+def pin_f16_brute_force(orc):
+    for (B, Hq, Hkv, Nq, Nk, d, causal, seed) in [(1, 2, 1, 5, 7, 32, False, 60), (1, 4, 2, 6, 4, 64, True, 61)]:
+        x = tiny_inputs(B, Hq, Hkv, Nq, Nk, d, seed, q_mult=8.0, dtype="f16")
+        scale = 1.0 / math.sqrt(d)
+        O, L = orc.forward(x["q"], x["k"], x["v"], scale, causal, dtype="f16")
+        Ob, Lb = brute_force_decimal(x, scale, causal, dtype="f16")
+        assert_close(O, Ob, what="f16 O brute")
+        assert_close(L, Lb, what="f16 LSE brute")
+
+
+F16_PINS = [pin_f16_decode_every_pattern, pin_f16_known_values, pin_f16_brute_force]
+ALL_PINS = ALL_PINS + F16_PINS

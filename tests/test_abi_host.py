@@ -101,11 +101,30 @@ def test_splitkv_workspace_and_default_splits(L):
     o = 3 * 2 * 100 * 4 * 128 * 4
     assert fa.splitkv_workspace_bytes(2, 4, 100, 128, 3) == ((o + 255) // 256) * 256 + 3 * 2 * 4 * 100 * 4
     assert fa.splitkv_workspace_bytes(2, 4, 100, 128, 0) == 0 and fa.splitkv_workspace_bytes(2, 4, 100, 128, 999) == 0
-    assert fa.splitkv_default_splits(8, 32, 4096, 4096, 128, 148) == 1       # already fills the GPU
-    s = fa.splitkv_default_splits(4, 32, 16, 32768, 128, 148)                 # 128 units
-    assert s == 2
-    assert fa.splitkv_default_splits(1, 1, 1, 65536, 128, 148) == 128        # capped by 4 tiles per split
-    assert fa.splitkv_default_splits(1, 1, 1, 300, 64, 148) == 1             # too few key tiles
+    assert fa.splitkv_default_splits(8, 32, 32, 4096, 4096, 128, 148) == 1   # already fills the GPU
+    # GQA-packed decode: 4 x 8 units of 64 rows, 256 key tiles; 9 splits = 2 waves x 29 tiles
+    assert fa.splitkv_default_splits(4, 32, 8, 16, 32768, 128, 148) == 9
+    assert fa.splitkv_default_splits(1, 1, 1, 1, 65536, 128, 148) == 128     # capped by 4 tiles per split
+    assert fa.splitkv_default_splits(1, 1, 1, 1, 300, 64, 148) == 1          # too few key tiles
+    assert fa.splitkv_default_splits(1, 6, 2, 1, 4096, 64, 148) >= 1         # n_rep = 3: not packed
+
+
+def _split_model(B, Hq, Hkv, Nq, Nk, sms, bk=128):
+    """The documented choice: fewest (waves x (tiles per split + 1)), >= 4 tiles per split."""
+    n_rep = Hq // Hkv
+    g = n_rep if (n_rep > 1 and 128 % n_rep == 0 and Nq < 128) else 1
+    units = B * (Hq // g) * -(-(Nq * g) // 256)
+    if units >= sms:
+        return 1
+    nkv = -(-Nk // bk)
+    costs = [(-(-units * s // sms) * (-(-nkv // s) + 1), s) for s in range(1, 257) if s == 1 or nkv // s >= 4]
+    return min(costs)[1]
+
+
+@pytest.mark.parametrize("B,Hq,Hkv,Nq,Nk", [(4, 32, 32, 16, 32768), (1, 8, 1, 1, 8192), (2, 16, 2, 64, 100000),
+                                            (1, 32, 8, 1, 1000), (3, 12, 4, 100, 50000)])
+def test_splitkv_default_splits_model(L, B, Hq, Hkv, Nq, Nk):
+    assert fa.splitkv_default_splits(B, Hq, Hkv, Nq, Nk, 128, 148) == _split_model(B, Hq, Hkv, Nq, Nk, 148)
 
 
 def _splitkv(L, splits=4, ws=FAKE + (5 << 30), ws_bytes=1 << 30, out=FAKE + (3 << 30)):

@@ -37,9 +37,9 @@ def tiny(B, Hq, Hkv, Nq, Nk, d, seed, **kw):
     return synth.make_inputs(w)
 
 
-def check_full(orc, x, scale, causal, what):
-    O, L = _parity.run_cuda(x, scale, causal)
-    Oref, Lref = orc.forward(x["q"], x["k"], x["v"], scale, causal)
+def check_full(orc, x, scale, causal, what, dtype="bf16"):
+    O, L = _parity.run_cuda(x, scale, causal, dtype=dtype)
+    Oref, Lref = orc.forward(x["q"], x["k"], x["v"], scale, causal, dtype=dtype)
     return _parity.compare(O, L, Oref, Lref, what)
 
 
@@ -121,6 +121,69 @@ def test_splitkv(orc, d, Nq, Nk, splits, causal):
     O, L = _parity.run_cuda(x, 1.0 / math.sqrt(d), causal, num_splits=splits)
     Oref, Lref = orc.forward(x["q"], x["k"], x["v"], 1.0 / math.sqrt(d), causal)
     _parity.compare(O, L, Oref, Lref, f"splitkv d={d} Nq={Nq} Nk={Nk} S={splits} causal={causal}")
+
+
+@pytest.mark.parametrize("n_rep", [2, 4, 8, 16, 32])
+@pytest.mark.parametrize("Nq", [1, 5, 16, 33, 127])
+@pytest.mark.parametrize("causal", [False, True])
+def test_gqa_packed_rows(orc, n_rep, Nq, causal):
+    """Nq < 128 with n_rep | 128: the n_rep heads of a KV head share a tile (flat rows
+    i * n_rep + r); two batches and two KV heads exercise the group indexing."""
+    Hkv = 2
+    d = 64 if n_rep >= 16 else 128
+    x = tiny(2, Hkv * n_rep, Hkv, Nq, 700, d, seed=n_rep * 100 + Nq)
+    check_full(orc, x, 1.0 / math.sqrt(d), causal, f"packed n_rep={n_rep} Nq={Nq} causal={causal}")
+
+
+@pytest.mark.parametrize("n_rep,Nq", [(3, 16), (4, 128), (64, 2)])
+def test_gqa_unpacked_and_edge(orc, n_rep, Nq):
+    """n_rep = 3 (does not divide 128) and Nq = 128 run unpacked; n_rep = 64 packs 2 rows per head."""
+    x = tiny(1, n_rep * 2, 2, Nq, 900, 64, seed=n_rep + Nq)
+    check_full(orc, x, 0.125, True, f"n_rep={n_rep} Nq={Nq}")
+
+
+@pytest.mark.parametrize("splits", [3, 9])
+@pytest.mark.parametrize("causal", [False, True])
+def test_gqa_packed_splitkv(orc, splits, causal):
+    x = tiny(2, 32, 8, 16, 5000, 128, seed=splits + 40)
+    O, L = _parity.run_cuda(x, 0.088, causal, num_splits=splits)
+    Oref, Lref = orc.forward(x["q"], x["k"], x["v"], 0.088, causal)
+    _parity.compare(O, L, Oref, Lref, f"packed split-KV S={splits} causal={causal}")
+
+
+@pytest.mark.parametrize("W", [1, 100, 1000])
+def test_gqa_packed_window(orc, W):
+    x = tiny(1, 16, 2, 40, 1200, 128, seed=W)
+    O, L = _parity.run_cuda(x, 0.088, True, window=W)
+    Oref, Lref = orc.forward(x["q"], x["k"], x["v"], 0.088, True, window=W)
+    _parity.compare(O, L, Oref, Lref, f"packed window W={W}")
+
+
+@pytest.mark.parametrize("d", HEAD_DIMS)
+@pytest.mark.parametrize("N", [17, 300])
+@pytest.mark.parametrize("causal", [False, True])
+def test_f16_small_shapes(orc, d, N, causal):
+    """fp16 inputs (fa_fwd_f16) against the oracle reading the same half bit patterns."""
+    x = tiny(1, 2, 1, N, N, d, seed=N + d + 7, dtype="f16")
+    check_full(orc, x, 1.0 / math.sqrt(d), causal, f"f16 d={d} N={N} causal={causal}", dtype="f16")
+
+
+@pytest.mark.parametrize("case", [(2, 8, 2, 200, 700, 128, True), (1, 32, 8, 16, 3000, 128, False),
+                                  (1, 4, 4, 1, 1, 64, False), (2, 6, 3, 130, 129, 96, True)])
+def test_f16_gqa_ragged(orc, case):
+    B, Hq, Hkv, Nq, Nk, d, causal = case
+    x = tiny(B, Hq, Hkv, Nq, Nk, d, seed=Nq + Nk, q_mult=8.0, dtype="f16")
+    check_full(orc, x, 1.0 / math.sqrt(d), causal, f"f16 {case}", dtype="f16")
+
+
+def test_f16_is_not_read_as_bf16(orc):
+    """The same bits read as bf16 give a different answer: fa_fwd_f16 must match the fp16
+    reading, not the bf16 one."""
+    x = tiny(1, 2, 1, 64, 64, 64, seed=3, dtype="f16")
+    O, L = _parity.run_cuda(x, 0.125, False, dtype="f16")
+    Of, _ = orc.forward(x["q"], x["k"], x["v"], 0.125, False, dtype="f16")
+    Ob, _ = orc.forward(x["q"], x["k"], x["v"], 0.125, False, dtype="bf16")
+    assert np.abs(O - Of).max() <= _parity.TOL_O_MAX < np.abs(O - Ob).max()
 
 
 def test_splitkv_matches_plain_forward():
@@ -221,7 +284,7 @@ LARGE_SAMPLED = [n for n in synth.WORKLOADS if n not in SMALL_FULL]
 def test_workload_full(orc, name):
     w = synth.WORKLOADS[name]
     x = synth.make_inputs(w)
-    res = check_full(orc, x, w.scale, w.causal, name)
+    res = check_full(orc, x, w.scale, w.causal, name, dtype=w.dtype)
     print(name, res)
 
 
@@ -231,10 +294,11 @@ def test_workload_sampled_rows(orc, name):
     oracle one by one, and every output row checked to be written and finite."""
     w = synth.WORKLOADS[name]
     x = synth.make_inputs(w)
-    O, L = _parity.run_cuda(x, w.scale, w.causal, window=w.window or None, num_splits=_parity.workload_splits(w))
+    O, L = _parity.run_cuda(x, w.scale, w.causal, window=w.window or None, num_splits=_parity.workload_splits(w),
+                            dtype=w.dtype)
     assert np.isfinite(O).all() and np.isfinite(L).all()
     rows = _parity.sample_rows(w, 192, seed=w.wid)
-    Oref, Lref = orc.rows(x["q"], x["k"], x["v"], rows, w.scale, w.causal, window=w.window)
+    Oref, Lref = orc.rows(x["q"], x["k"], x["v"], rows, w.scale, w.causal, window=w.window, dtype=w.dtype)
     Os = O[rows[:, 0], rows[:, 2], rows[:, 1], :]
     Ls = L[rows[:, 0], rows[:, 1], rows[:, 2]]
     res = _parity.compare(Os, Ls, Oref, Lref, name)
