@@ -59,6 +59,9 @@ class Oracle:
         lib.oracle_attention_rows.argtypes = [_u16p, _u16p, _u16p, _i32p, cl, _f64p, _f64p,
                                               ci, ci, ci, ci, ci, ci, cd, ci, ci, ci, ci]
         lib.oracle_attention_rows.restype = ci
+        lib.oracle_attention_bwd.argtypes = [_u16p, _u16p, _u16p, _u16p, _f64p, _f64p, _f64p,
+                                             ci, ci, ci, ci, ci, ci, cd, ci, ci, ci, ci]
+        lib.oracle_attention_bwd.restype = ci
         self.lib = lib
 
     @staticmethod
@@ -117,6 +120,25 @@ class Oracle:
         if rc != 0:
             raise RuntimeError(f"oracle_attention_rows failed: {rc}")
         return out, lse
+
+
+    def backward(self, q, k, v, dout, scale: float, causal: bool, threads: int | None = None, window: int = 0,
+                 dtype: str = "bf16"):
+        """(dQ [B,Nq,Hq,d], dK [B,Nk,Hkv,d], dV [B,Nk,Hkv,d]) in fp64: the gradient of
+        sum(O * dO) for bit-pattern inputs q, k, v, dout of element type `dtype`."""
+        q, k, v, B, Hq, Hkv, Nq, Nk, d = self._dims(q, k, v)
+        dout = np.ascontiguousarray(dout, dtype=np.uint16)
+        if dout.shape != q.shape:
+            raise ValueError(f"dout shape {dout.shape} != q shape {q.shape}")
+        dq = np.zeros((B, Nq, Hq, d), dtype=np.float64)
+        dk = np.zeros((B, Nk, Hkv, d), dtype=np.float64)
+        dv = np.zeros((B, Nk, Hkv, d), dtype=np.float64)
+        rc = self.lib.oracle_attention_bwd(q, k, v, dout, dq, dk, dv, B, Hq, Hkv, Nq, Nk, d, float(scale),
+                                           int(bool(causal)), int(window), self._elem(dtype),
+                                           threads or os.cpu_count() or 1)
+        if rc != 0:
+            raise RuntimeError(f"oracle_attention_bwd failed: {rc}")
+        return dq, dk, dv
 
 
 _default: Oracle | None = None

@@ -42,6 +42,15 @@
  * Softmax is taken in two passes over the materialised row (row max M_i first,
  * then exp(S_ij - M_i)), the textbook way to keep exp() in range.
  *
+ * The backward pass (oracle_attention_bwd) is the gradient of L = sum O (.) dO through
+ * the same definition: the pages ask for it by recomputation from Q, K, V (hwcomputing
+ * article, "performance tuning"; kaiwu.csdn.net page on the FlashAttention principle,
+ * section 2.3 on recomputing S and P in the backward pass).  With P the probability
+ * matrix of the forward, the chain rule through O = P V and the row softmax gives
+ *     dV = P^T dO,  dP = dO V^T,  dS_ij = P_ij (dP_ij - sum_k P_ik dP_ik),
+ *     dQ = scale dS K,  dK = scale dS^T Q,
+ * with dK and dV of a KV head summed over the query heads that share it (GQA).
+ *
  * Compile-time ORACLE_PLANT_* macros build deliberately wrong variants; the test
  * suite uses them to show that its pins catch each kind of mistake.  A normal build
  * defines none of them.
@@ -326,6 +335,113 @@ int oracle_attention_rows(const uint16_t *q, const uint16_t *k, const uint16_t *
         jobs[t] = (rows_job_t){&p, rows, nrows * t / nt, nrows * (t + 1) / nt, out_rows, lse_rows, 0};
         if (nt == 1) { rows_worker(&jobs[t]); continue; }
         if (pthread_create(&tid[t], NULL, rows_worker, &jobs[t]) != 0) { rc = ORACLE_ETHREAD; break; }
+        ++started;
+    }
+    for (int t = 0; t < started; ++t) pthread_join(tid[t], NULL);
+    for (int t = 0; t < nt && rc == ORACLE_OK; ++t) if (jobs[t].rc) rc = jobs[t].rc;
+    free(tid);
+    free(jobs);
+    return rc;
+}
+
+/* ---- backward: gradients of L = sum_{b,i,h,c} O[b,i,h,c] dO[b,i,h,c] ---- */
+
+typedef struct {
+    const problem_t *p;
+    const uint16_t *dout;     /* dO bit patterns, [B,Nq,Hq,d] */
+    double *dq, *dk, *dv;     /* [B,Nq,Hq,d], [B,Nk,Hkv,d], [B,Nk,Hkv,d] */
+    int t, nt;                /* this worker takes (b, g) pairs t, t + nt, ... */
+    int rc;
+} bwd_job_t;
+
+static double do_at(const bwd_job_t *jb, int b, int i, int h, int c) {
+    const problem_t *p = jb->p;
+    return elem(p, jb->dout[(((size_t)b * p->Nq + i) * p->Hq + h) * p->d + c]);
+}
+
+static void *bwd_worker(void *arg) {
+    bwd_job_t *jb = (bwd_job_t *)arg;
+    const problem_t *p = jb->p;
+    const int Nk = p->Nk, d = p->d, n_rep = p->Hq / p->Hkv;
+    const size_t nk = Nk > 0 ? (size_t)Nk : 1;
+    double *prow = (double *)malloc(sizeof(double) * nk);
+    double *dprow = (double *)malloc(sizeof(double) * nk);
+    double *orow = (double *)malloc(sizeof(double) * (size_t)d);
+    if (!prow || !dprow || !orow) { free(prow); free(dprow); free(orow); jb->rc = ORACLE_ENOMEM; return NULL; }
+    for (long pair = jb->t; pair < (long)p->B * p->Hkv; pair += jb->nt) {
+        const int b = (int)(pair / p->Hkv), g = (int)(pair % p->Hkv);
+        for (int r = 0; r < n_rep; ++r) {
+            const int hq = g * n_rep + r;    /* the query heads that read KV head g */
+            if (kv_head_of(p, hq) != g) continue;
+            for (int i = 0; i < p->Nq; ++i) {
+                double lse;
+                attention_row(p, b, hq, i, prow, orow, &lse);   /* prow = P_i. */
+                /* dP_ij = dO_i . V_j ; D_i = sum_j P_ij dP_ij */
+                double D = 0.0;
+                for (int j = 0; j < Nk; ++j) {
+                    double acc = 0.0;
+                    for (int c = 0; c < d; ++c) acc += do_at(jb, b, i, hq, c) * v_at(p, b, j, g, c);
+                    dprow[j] = acc;
+                    D += prow[j] * acc;
+                }
+                double *dqi = jb->dq + (((size_t)b * p->Nq + i) * p->Hq + hq) * d;
+                for (int j = 0; j < Nk; ++j) {
+                    const double pij = prow[j];
+                    if (pij == 0.0) continue;
+#ifdef ORACLE_PLANT_BWD_NO_D
+                    const double dsij = pij * dprow[j];
+#else
+                    const double dsij = pij * (dprow[j] - D);
+#endif
+#ifdef ORACLE_PLANT_BWD_DQ_NO_SCALE
+                    const double sq = 1.0;
+#else
+                    const double sq = p->scale;
+#endif
+                    double *dkj = jb->dk + (((size_t)b * Nk + j) * p->Hkv + g) * d;
+                    double *dvj = jb->dv + (((size_t)b * Nk + j) * p->Hkv + g) * d;
+                    for (int c = 0; c < d; ++c) {
+                        dqi[c] += sq * dsij * k_at(p, b, j, g, c);
+                        dkj[c] += p->scale * dsij * q_at(p, b, i, hq, c);
+#ifdef ORACLE_PLANT_BWD_DV_NO_P
+                        dvj[c] += do_at(jb, b, i, hq, c);
+#else
+                        dvj[c] += pij * do_at(jb, b, i, hq, c);
+#endif
+                    }
+                }
+            }
+        }
+    }
+    free(prow); free(dprow); free(orow);
+    return NULL;
+}
+
+/*
+ * oracle_attention_bwd: dQ, dK, dV of L = sum O (.) dO.
+ *   q/k/v as oracle_attention_fwd; dout [B,Nq,Hq,d] bit patterns of the same element type.
+ *   dq [B,Nq,Hq,d], dk/dv [B,Nk,Hkv,d] fp64, overwritten.
+ */
+int oracle_attention_bwd(const uint16_t *q, const uint16_t *k, const uint16_t *v, const uint16_t *dout,
+                         double *dq, double *dk, double *dv, int B, int Hq, int Hkv, int Nq, int Nk,
+                         int d, double scale, int causal, int window, int elem_f16, int nthreads) {
+    problem_t p = {q, k, v, B, Hq, Hkv, Nq, Nk, d, scale, causal ? 1 : 0, window, elem_f16 ? 1 : 0};
+    if (!check_problem(&p)) return ORACLE_EINVAL;
+    memset(dq, 0, sizeof(double) * (size_t)B * Nq * Hq * d);
+    memset(dk, 0, sizeof(double) * (size_t)B * Nk * Hkv * d);
+    memset(dv, 0, sizeof(double) * (size_t)B * Nk * Hkv * d);
+    if (nthreads < 1) nthreads = 1;
+    const long pairs = (long)B * Hkv;
+    if (pairs == 0 || Nq == 0 || Nk == 0) return ORACLE_OK;
+    int nt = (long)nthreads < pairs ? nthreads : (int)pairs;
+    pthread_t *tid = (pthread_t *)malloc(sizeof(pthread_t) * (size_t)nt);
+    bwd_job_t *jobs = (bwd_job_t *)malloc(sizeof(bwd_job_t) * (size_t)nt);
+    if (!tid || !jobs) { free(tid); free(jobs); return ORACLE_ENOMEM; }
+    int started = 0, rc = ORACLE_OK;
+    for (int t = 0; t < nt; ++t) {
+        jobs[t] = (bwd_job_t){&p, dout, dq, dk, dv, t, nt, 0};
+        if (nt == 1) { bwd_worker(&jobs[t]); continue; }
+        if (pthread_create(&tid[t], NULL, bwd_worker, &jobs[t]) != 0) { rc = ORACLE_ETHREAD; break; }
         ++started;
     }
     for (int t = 0; t < started; ++t) pthread_join(tid[t], NULL);

@@ -34,7 +34,7 @@ GOLDEN_GAMMA = np.uint64(0x9E3779B97F4A7C15)
 _M1 = np.uint64(0xBF58476D1CE4E5B9)
 _M2 = np.uint64(0x94D049BB133111EB)
 
-TENSOR_IDS = {"q": 1, "k": 2, "v": 3}
+TENSOR_IDS = {"q": 1, "k": 2, "v": 3, "do": 4}
 
 
 def _mix(z: np.ndarray) -> np.ndarray:
@@ -175,6 +175,15 @@ def make_inputs(w: Workload) -> dict[str, np.ndarray]:
             bits = scale_bf16_bits_pow2(bits, mult)
         out[name] = bits.reshape(shp)
     return out
+
+
+def make_grad_output(w: Workload) -> np.ndarray:
+    """Seeded upstream gradient dO [B,Nq,Hq,d] for the backward pass: N(0,1) draws from
+    their own stream, rounded to the workload's element type like the inputs."""
+    shp = (w.B, w.Nq, w.Hq, w.d)
+    z = normal_f64(stream_key(w.seed, w.wid, TENSOR_IDS["do"]), int(np.prod(shp))).astype(np.float32)
+    bits = f32_to_f16_bits(z) if w.dtype == "f16" else f32_to_bf16_bits(z)
+    return bits.reshape(shp)
 
 
 def _wl(name, wid, B, H, N, d, causal=False, Hkv=None, Nk=None, **kw):

@@ -405,3 +405,129 @@ def pin_f16_brute_force(orc):
 
 F16_PINS = [pin_f16_decode_every_pattern, pin_f16_known_values, pin_f16_brute_force]
 ALL_PINS = ALL_PINS + F16_PINS
+
+
+# ---------------------------------------------------------------- backward pass
+
+def _dec(a):
+    return np.array([Decimal(float(t)) for t in np.asarray(a, dtype=np.float64).ravel()], dtype=object).reshape(np.shape(a))
+
+
+def decimal_loss(q, k, v, do, scale, causal, window=0):
+    """L = sum O (.) dO by the definition, in Decimal arithmetic (object arrays)."""
+    B, Nq, Hq, d = q.shape
+    _, Nk, Hkv, _ = k.shape
+    rep = Hq // Hkv
+    sc = Decimal(float(scale))
+    total = Decimal(0)
+    for b in range(B):
+        for h in range(Hq):
+            g = h // rep
+            for i in range(Nq):
+                es = []
+                for j in range(Nk):
+                    if visible(i, j, Nq, Nk, causal, window):
+                        es.append((j, (sc * sum(q[b, i, h, c] * k[b, j, g, c] for c in range(d))).exp()))
+                Z = sum(e for _, e in es)
+                if not es:
+                    continue
+                for c in range(d):
+                    total += sum(e * v[b, j, g, c] for j, e in es) / Z * do[b, i, h, c]
+    return total
+
+
+def finite_difference_grads(x, do_bits, scale, causal, window=0, h="1e-15"):
+    """Central differences of decimal_loss with respect to every element of q, k, v."""
+    getcontext().prec = 60
+    arrs = {n: _dec(bits_f64(x[n])) for n in ("q", "k", "v")}
+    do = _dec(bits_f64(do_bits))
+    hh = Decimal(h)
+    grads = {}
+    for name in ("q", "k", "v"):
+        a = arrs[name]
+        g = np.zeros(a.shape)
+        for idx in np.ndindex(a.shape):
+            x0 = a[idx]
+            a[idx] = x0 + hh
+            lp = decimal_loss(arrs["q"], arrs["k"], arrs["v"], do, scale, causal, window)
+            a[idx] = x0 - hh
+            lm = decimal_loss(arrs["q"], arrs["k"], arrs["v"], do, scale, causal, window)
+            a[idx] = x0
+            g[idx] = float((lp - lm) / (2 * hh))
+        grads[name] = g
+    return grads["q"], grads["k"], grads["v"]
+
+
+def _bwd_inputs(B, Hq, Hkv, Nq, Nk, d, seed, dtype="bf16"):
+    w = synth.Workload("tinybwd", 2000 + seed, B, Hq, Hkv, Nq, Nk, d, False, seed=seed, dtype=dtype)
+    return synth.make_inputs(w), synth.make_grad_output(w)
+
+
+BWD_FD_CASES = [
+    # B, Hq, Hkv, Nq, Nk, d, causal, window, seed
+    (1, 2, 1, 3, 4, 3, False, 0, 70),
+    (1, 2, 2, 4, 3, 2, True, 0, 71),     # Nq > Nk: row 0 sees no key
+    (1, 1, 1, 5, 5, 2, True, 2, 72),     # sliding window
+]
+
+
+def pin_bwd_finite_difference(orc):
+    """The oracle's dQ, dK, dV equal central differences of the loss sum O (.) dO taken in
+    60-digit decimal arithmetic straight from the forward definition."""
+    for (B, Hq, Hkv, Nq, Nk, d, causal, W, seed) in BWD_FD_CASES:
+        x, do = _bwd_inputs(B, Hq, Hkv, Nq, Nk, d, seed)
+        scale = 0.7
+        dq, dk, dv = orc.backward(x["q"], x["k"], x["v"], do, scale, causal, window=W)
+        fq, fk, fv = finite_difference_grads(x, do, scale, causal, window=W)
+        assert_close(dq, fq, tol=1e-9, what=f"dQ fd {seed}")
+        assert_close(dk, fk, tol=1e-9, what=f"dK fd {seed}")
+        assert_close(dv, fv, tol=1e-9, what=f"dV fd {seed}")
+
+
+def pin_bwd_one_key(orc):
+    """Nk = 1: P = 1 for every row, so dS = 0 (dQ = dK = 0) and dV = sum of dO over the
+    rows and query heads of the group."""
+    x, do = _bwd_inputs(2, 4, 2, 5, 1, 16, seed=73)
+    dq, dk, dv = orc.backward(x["q"], x["k"], x["v"], do, 0.25, False)
+    assert np.abs(dq).max() < TOL and np.abs(dk).max() < TOL
+    dof = bits_f64(do)
+    for b in range(2):
+        for g in range(2):
+            assert_close(dv[b, 0, g], dof[b, :, 2 * g:2 * g + 2].sum(axis=(0, 1)), what="dV one key")
+
+
+def pin_bwd_dk_sums_to_zero(orc):
+    """Each softmax row is invariant to adding one vector to every key, so the key
+    gradients of a head sum to zero (sum_j dS_ij = 0 per row)."""
+    for causal in (False, True):
+        x, do = _bwd_inputs(1, 4, 2, 7, 9, 16, seed=74)
+        _, dk, _ = orc.backward(x["q"], x["k"], x["v"], do, 0.3, causal)
+        assert np.abs(dk.sum(axis=1)).max() < 1e-12 * max(1.0, np.abs(dk).max() * 9)
+
+
+def pin_bwd_gqa_is_summed_mha(orc):
+    """GQA gradients: dQ equals MHA with K, V repeated per query head; dK, dV of a KV head
+    are the sums over its query heads of the MHA ones."""
+    x, do = _bwd_inputs(1, 6, 2, 5, 7, 8, seed=75)
+    dq, dk, dv = orc.backward(x["q"], x["k"], x["v"], do, 0.4, True)
+    kr = np.repeat(x["k"], 3, axis=2)
+    vr = np.repeat(x["v"], 3, axis=2)
+    dq2, dk2, dv2 = orc.backward(x["q"], kr, vr, do, 0.4, True)
+    assert_close(dq, dq2, what="GQA dQ")
+    assert_close(dk, dk2.reshape(1, 7, 2, 3, 8).sum(axis=3), what="GQA dK")
+    assert_close(dv, dv2.reshape(1, 7, 2, 3, 8).sum(axis=3), what="GQA dV")
+
+
+def pin_bwd_causal_first_row(orc):
+    """Causal, Nq = Nk: row 0 sees only key 0, so its dQ is zero; the last key is seen
+    only by the last row, so its dV is P_last,last * dO_last."""
+    x, do = _bwd_inputs(1, 1, 1, 6, 6, 8, seed=76)
+    dq, dk, dv = orc.backward(x["q"], x["k"], x["v"], do, 0.5, True)
+    assert np.abs(dq[0, 0, 0]).max() < TOL
+    _, _, P = orc.probs(x["q"], x["k"], x["v"], 0.5, True)
+    assert_close(dv[0, 5, 0], P[0, 0, 5, 5] * bits_f64(do)[0, 5, 0], what="last key dV")
+
+
+BWD_PINS = [pin_bwd_finite_difference, pin_bwd_one_key, pin_bwd_dk_sums_to_zero, pin_bwd_gqa_is_summed_mha,
+            pin_bwd_causal_first_row]
+ALL_PINS = ALL_PINS + BWD_PINS
