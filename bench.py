@@ -350,6 +350,61 @@ def run_ours(args, w, world, rank, local):
     return 0
 
 
+BWD_DEFAULT = ("seq4096_b8_h32_d128,seq1024_b8_h32_d128,gqa_prefill_b4_n4096_hq32_hkv8_d128_causal,"
+               "long16k_b1_h32_d128_causal,hdim64_b2_n4096_h16")
+
+
+def run_bwd_sweep(args):
+    """Backward pass (fa_bwd) on workloads of the table, one JSON line each (device time,
+    1 GPU).  FLOPs: five matrix products of the forward's size, 2.5x the forward count."""
+    import torch
+    import exact_attention_146_b200 as fa
+    torch.cuda.set_device(0)
+    pk = peaks()
+    names = (args.sweep_only or BWD_DEFAULT).split(",")
+    for name in names:
+        w = synth.WORKLOADS[name]
+        if w.d not in (64, 128) or w.dtype != "bf16" or w.window or w.splitkv:
+            continue
+        x = synth.make_inputs(w)
+        q, k, v = (torch.from_numpy(x[n].view(np.int16)).view(torch.bfloat16).cuda() for n in ("q", "k", "v"))
+        do = torch.from_numpy(synth.make_grad_output(w).view(np.int16)).view(torch.bfloat16).cuda()
+        out, lse = fa.fa_fwd(q, k, v, causal=w.causal, scale=w.scale)
+        dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+        ws = torch.empty(max(1, fa.bwd_workspace_bytes(w.B, w.Hq, w.Nq, w.d)), dtype=torch.uint8, device="cuda")
+        flush = torch.empty(int(2 * 126e6) // 4, dtype=torch.float32, device="cuda")
+
+        def call():
+            fa.fa_bwd(q, k, v, out, do, lse, causal=w.causal, scale=w.scale, dq=dq, dk=dk, dv=dv, workspace=ws)
+
+        for _ in range(args.warmup):
+            call()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        for _ in range(args.steps):
+            call()
+        b.record()
+        torch.cuda.synchronize()
+        ms_warm = a.elapsed_time(b) / args.steps
+        times = []
+        for _ in range(min(args.steps, 10)):
+            flush.zero_()
+            a.record()
+            call()
+            b.record()
+            torch.cuda.synchronize()
+            times.append(a.elapsed_time(b))
+        ms_cold = sorted(times)[len(times) // 2]
+        st, _ = fa.device_status()
+        flops = 2.5 * w.flops
+        print(json.dumps({"workload": name, "pass": "backward", "ms_warm": ms_warm, "ms_l2_flushed": ms_cold,
+                          "tflops": flops / (ms_cold * 1e-3) / 1e12,
+                          "pct_peak": 100 * flops / (ms_cold * 1e-3) / 1e12 / pk["bf16_tflops"],
+                          "launches_per_call": 3, "status": st}), flush=True)
+    return 0
+
+
 def run_sweep(args):
     """Every workload of the table, one JSON line each (device time only, 1 GPU)."""
     import torch
@@ -415,12 +470,15 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-clocks", action="store_true")
     ap.add_argument("--sweep", action="store_true", help="time every workload of the table (1 GPU)")
-    ap.add_argument("--sweep-only", default="", help="comma-separated workload names for --sweep")
+    ap.add_argument("--sweep-only", default="", help="comma-separated workload names for --sweep / --bwd-sweep")
+    ap.add_argument("--bwd-sweep", action="store_true", help="time the backward pass on workloads of the table")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     if args.sweep:
         return run_sweep(args)
+    if args.bwd_sweep:
+        return run_bwd_sweep(args)
     w = synth.WORKLOADS[args.workload]
     world, rank, local = dist_setup(args.gpus)
     if args.impl == "reference":

@@ -167,6 +167,39 @@ int fa_fwd_splitkv_static(const void *q, const void *k, const void *v, void *out
                           int B, int Hq, int Hkv, int Nq, int Nk, int d, float scale, int causal,
                           int num_splits, void *stream);
 
+/*
+ * fa_bwd -- exact attention backward: the gradients dQ, dK, dV of L = sum O (.) dO, with
+ * S and P recomputed from Q, K, V and the forward's LSE instead of being stored (the
+ * kaiwu.csdn.net FlashAttention principle page, section 2.3; the hwcomputing.csdn.net
+ * FlashAttention article, "performance tuning"):
+ *
+ *     P = exp(scale Q K^T - LSE)  (masked),   dV = P^T dO,   dP = dO V^T,
+ *     dS = P (.) (dP - D) with D_i = dO_i . O_i,   dQ = scale dS K,   dK = scale dS^T Q,
+ *
+ * dK and dV of a KV head summed over the query heads that share it (GQA).
+ *
+ *   q, out, dout [B, Nq, Hq, d] bf16, read only (out and lse from fa_fwd on the same q, k, v,
+ *                scale and mask)
+ *   k, v         [B, Nk, Hkv, d] bf16, read only
+ *   lse          [B, Hq, Nq] fp32 (natural log), read only
+ *   dq           [B, Nq, Hq, d] bf16, written;  dk, dv [B, Nk, Hkv, d] bf16, written
+ *   d in {64, 128} (FA_ERR_UNSUPPORTED_HEAD_DIM otherwise); causal in {0, 1}; the other
+ *   sizes and the scale as fa_fwd
+ *   workspace    caller-owned device scratch of at least fa_bwd_workspace_bytes bytes,
+ *                256-byte aligned (fp32 dQ accumulator and D); no initial contents are
+ *                needed (the call zeroes what it accumulates into); contents undefined
+ *                afterwards; two calls must not share one concurrently.
+ *
+ * Three kernels run on `stream`: D and the zeroed accumulator, the main kernel (one unit per
+ * (batch, KV head, 128-key tile); dQ accumulated with fp32 reductions), and dQ = bf16(scale
+ * acc).  Errors as fa_fwd; the outputs must not overlap any input, each other or the
+ * workspace (FA_ERR_OVERLAP).  With Nq == 0 or Nk == 0 the existing gradients are zero.
+ */
+size_t fa_bwd_workspace_bytes(int B, int Hq, int Nq, int d);
+int fa_bwd(const void *q, const void *k, const void *v, const void *out, const void *dout, const float *lse,
+           void *dq, void *dk, void *dv, int B, int Hq, int Hkv, int Nq, int Nk, int d, float scale, int causal,
+           void *workspace, size_t workspace_bytes, void *stream);
+
 /* Human-readable text of a status code (static storage; never NULL). */
 const char *fa_status_string(int status);
 

@@ -142,6 +142,25 @@ def test_splitkv_validation(L):
     assert _splitkv(L) in (fa.FA_ERR_UNSUPPORTED_DEVICE, fa.FA_ERR_NOT_DEVICE_MEMORY)
 
 
+def _bwd(L, d=128, ws=FAKE + (12 << 30), ws_bytes=1 << 30, dq=FAKE + (5 << 30), causal=0, lse=FAKE + (4 << 30)):
+    return L.fa_bwd(FAKE, FAKE + (1 << 30), FAKE + (2 << 30), FAKE + (3 << 30), FAKE + (6 << 30), lse, dq,
+                    FAKE + (7 << 30), FAKE + (8 << 30), 1, 2, 1, 64, 64, d, 0.125, causal, ws, ws_bytes, None)
+
+
+def test_bwd_validation(L):
+    assert fa.bwd_workspace_bytes(2, 4, 100, 128) == ((2 * 100 * 4 * 128 * 4 + 255) // 256) * 256 + 2 * 4 * 100 * 4
+    assert _bwd(L, d=96) == fa.FA_ERR_UNSUPPORTED_HEAD_DIM
+    assert _bwd(L, causal=2) == fa.FA_ERR_INVALID_ARG
+    assert _bwd(L, lse=None) == fa.FA_ERR_INVALID_ARG
+    assert _bwd(L, ws=None) == fa.FA_ERR_INVALID_ARG
+    assert _bwd(L, ws_bytes=10) == fa.FA_ERR_INVALID_ARG
+    assert _bwd(L, ws=FAKE + (12 << 30) + 16) == fa.FA_ERR_MISALIGNED
+    assert _bwd(L, dq=FAKE + (5 << 30) + 2) == fa.FA_ERR_MISALIGNED
+    assert _bwd(L, dq=FAKE) == fa.FA_ERR_OVERLAP                       # dq over q
+    assert _bwd(L, ws=FAKE + (7 << 30)) == fa.FA_ERR_OVERLAP           # workspace over dk
+    assert _bwd(L) in (fa.FA_ERR_UNSUPPORTED_DEVICE, fa.FA_ERR_NOT_DEVICE_MEMORY)
+
+
 def test_empty_problems_are_noops(L):
     # no output rows: nothing to validate against the device, nothing launched
     assert call(L, B=0, q=None, k=None, v=None, out=None, lse=None) == fa.FA_OK
