@@ -418,20 +418,22 @@ __device__ void dw_role(const BwdParams &p, uint32_t sbase, uint32_t tmem, const
             if (!warp_wait(bar(C::B_DQ_FULL), n_step & 1u, ctl, kSiteDqFull)) return;
             sm100::tc_fence_after_sync();
             float *dst = p.dq_acc + ((size_t(w.b) * p.Nq + size_t(q)) * p.Hq + hq) * C::D;
-#pragma unroll 1
-            for (int c = 0; c < C::D / 32; ++c) {
-                uint32_t v[32];
-                sm100::tmem_ld32_sync(tmem + lane_off + uint32_t(C::COL_A + 32 * c), v);
-                if (q < p.Nq) {
+            // the whole dQ row into registers first, so region A is free for the next
+            // step's S^T while the reductions run
+            uint32_t v[C::D];
 #pragma unroll
-                    for (int m = 0; m < 8; ++m)
-                        atomicAdd(reinterpret_cast<float4 *>(dst + 32 * c + 4 * m),
-                                  make_float4(__uint_as_float(v[4 * m]), __uint_as_float(v[4 * m + 1]),
-                                              __uint_as_float(v[4 * m + 2]), __uint_as_float(v[4 * m + 3])));
-                }
-            }
+            for (int c = 0; c < C::D / 32; ++c)
+                sm100::tmem_ld32_sync(tmem + lane_off + uint32_t(C::COL_A + 32 * c),
+                                      *reinterpret_cast<uint32_t(*)[32]>(v + 32 * c));
             sm100::tc_fence_before_sync();
             sm100::mbar_arrive(bar(C::B_DQ_EMPTY));
+            if (q < p.Nq) {
+#pragma unroll
+                for (int m = 0; m < C::D / 4; ++m)
+                    atomicAdd(reinterpret_cast<float4 *>(dst + 4 * m),
+                              make_float4(__uint_as_float(v[4 * m]), __uint_as_float(v[4 * m + 1]),
+                                          __uint_as_float(v[4 * m + 2]), __uint_as_float(v[4 * m + 3])));
+            }
         }
         if (!warp_wait(bar(C::B_ACC_FULL), n_unit & 1u, ctl, kSiteAccFull)) return;
         sm100::tc_fence_after_sync();
