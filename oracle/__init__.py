@@ -24,6 +24,7 @@ LIB_PATH = _HERE / "liboracle.so"
 _u16p = np.ctypeslib.ndpointer(dtype=np.uint16, flags="C_CONTIGUOUS")
 _f64p = np.ctypeslib.ndpointer(dtype=np.float64, flags="C_CONTIGUOUS")
 _i32p = np.ctypeslib.ndpointer(dtype=np.int32, flags="C_CONTIGUOUS")
+_u8p = np.ctypeslib.ndpointer(dtype=np.uint8, flags="C_CONTIGUOUS")
 
 
 def build(out: Path | None = None, defines: tuple[str, ...] = ()) -> Path:
@@ -62,6 +63,12 @@ class Oracle:
         lib.oracle_attention_bwd.argtypes = [_u16p, _u16p, _u16p, _u16p, _f64p, _f64p, _f64p,
                                              ci, ci, ci, ci, ci, ci, cd, ci, ci, ci, ci]
         lib.oracle_attention_bwd.restype = ci
+        lib.oracle_attention_fwd_fp8.argtypes = [_u8p, _u8p, _u8p, _f64p, _f64p, ci, ci, ci, ci, ci, ci,
+                                                 cd, cd, cd, cd, ci, ci, ci]
+        lib.oracle_attention_fwd_fp8.restype = ci
+        lib.oracle_attention_rows_fp8.argtypes = [_u8p, _u8p, _u8p, _i32p, cl, _f64p, _f64p, ci, ci, ci, ci, ci, ci,
+                                                  cd, cd, cd, cd, ci, ci, ci]
+        lib.oracle_attention_rows_fp8.restype = ci
         self.lib = lib
 
     @staticmethod
@@ -121,6 +128,41 @@ class Oracle:
             raise RuntimeError(f"oracle_attention_rows failed: {rc}")
         return out, lse
 
+
+    def forward_fp8(self, q8, k8, v8, scale: float, causal: bool, descale=(1.0, 1.0, 1.0), threads: int | None = None,
+                    window: int = 0):
+        """O, LSE in fp64 for OCP E4M3 byte inputs with dequantisation factors
+        descale = (dq, dk, dv): Q = dq * q8, K = dk * k8, V = dv * v8."""
+        q8, k8, v8 = (np.ascontiguousarray(x, dtype=np.uint8) for x in (q8, k8, v8))
+        B, Nq, Hq, d = q8.shape
+        Bk, Nk, Hkv, dk_ = k8.shape
+        if v8.shape != k8.shape or Bk != B or dk_ != d:
+            raise ValueError(f"shape mismatch q{q8.shape} k{k8.shape} v{v8.shape}")
+        out = np.zeros((B, Nq, Hq, d), dtype=np.float64)
+        lse = np.zeros((B, Hq, Nq), dtype=np.float64)
+        rc = self.lib.oracle_attention_fwd_fp8(q8, k8, v8, out, lse, B, Hq, Hkv, Nq, Nk, d, float(scale),
+                                               float(descale[0]), float(descale[1]), float(descale[2]),
+                                               int(bool(causal)), int(window), threads or os.cpu_count() or 1)
+        if rc != 0:
+            raise RuntimeError(f"oracle_attention_fwd_fp8 failed: {rc}")
+        return out, lse
+
+    def rows_fp8(self, q8, k8, v8, rows, scale: float, causal: bool, descale=(1.0, 1.0, 1.0),
+                 threads: int | None = None, window: int = 0):
+        """O [n,d] and LSE [n] of the listed (b, hq, i) rows for E4M3 inputs."""
+        q8, k8, v8 = (np.ascontiguousarray(x, dtype=np.uint8) for x in (q8, k8, v8))
+        B, Nq, Hq, d = q8.shape
+        Nk, Hkv = k8.shape[1], k8.shape[2]
+        rows = np.ascontiguousarray(np.asarray(rows, dtype=np.int32).reshape(-1, 3))
+        n = rows.shape[0]
+        out = np.zeros((n, d), dtype=np.float64)
+        lse = np.zeros((n,), dtype=np.float64)
+        rc = self.lib.oracle_attention_rows_fp8(q8, k8, v8, rows, n, out, lse, B, Hq, Hkv, Nq, Nk, d, float(scale),
+                                                float(descale[0]), float(descale[1]), float(descale[2]),
+                                                int(bool(causal)), int(window), threads or os.cpu_count() or 1)
+        if rc != 0:
+            raise RuntimeError(f"oracle_attention_rows_fp8 failed: {rc}")
+        return out, lse
 
     def backward(self, q, k, v, dout, scale: float, causal: bool, threads: int | None = None, window: int = 0,
                  dtype: str = "bf16"):

@@ -37,7 +37,10 @@
  *  - LSE is the natural-log log-sum-exp of the scaled, masked logits;
  *  - inputs are bf16 (or, for the fp16 variant of the "performance tuning" data-type
  *    item of the same article, IEEE binary16) bit patterns, widened exactly to fp64;
- *    nothing is rounded in between.
+ *    nothing is rounded in between;
+ *  - FP8 inputs (the FlashAttention-3 FP8 forward of the datacanvas.csdn.net head-dim
+ *    page) are OCP E4M3 bytes with one dequantisation factor per tensor: Q = dq * q8,
+ *    K = dk * k8, V = dv * v8, after which the definition is unchanged.
  *
  * Softmax is taken in two passes over the materialised row (row max M_i first,
  * then exp(S_ij - M_i)), the textbook way to keep exp() in range.
@@ -73,6 +76,21 @@ static double bf16_bits_to_double(uint16_t bits) {
     return (double)f;
 }
 
+/* OCP FP8 E4M3: 1 sign bit, 4 exponent bits (bias 7), 3 fraction bits; exponent 0 is
+ * subnormal (fraction * 2^-9); S.1111.111 is NaN; there is no infinity (max 448). */
+static double e4m3_bits_to_double(uint8_t bits) {
+    const int e = (bits >> 3) & 0xf, frac = bits & 0x7;
+    double mag;
+    if (e == 0xf && frac == 0x7) return NAN;
+    if (e == 0) mag = ldexp((double)frac, -9);
+#ifdef ORACLE_PLANT_E4M3_BIAS
+    else mag = ldexp((double)(8 + frac), e - 11);
+#else
+    else mag = ldexp((double)(8 + frac), e - 10);
+#endif
+    return (bits & 0x80) ? -mag : mag;
+}
+
 /* IEEE 754 binary16: 1 sign bit, 5 exponent bits (bias 15), 10 fraction bits;
  * exponent 0 is subnormal (fraction * 2^-24), exponent 31 is inf/NaN. */
 static double f16_bits_to_double(uint16_t bits) {
@@ -95,6 +113,8 @@ typedef struct {
     int causal;
     int window;     /* 0: no window; W >= 1: sliding window of W keys (implies causal) */
     int elem_f16;   /* inputs are fp16 (1) or bf16 (0) bit patterns */
+    const uint8_t *q8, *k8, *v8;   /* non-NULL: E4M3 inputs (q, k, v unused) */
+    double dq, dk, dv;             /* dequantisation factors of the E4M3 inputs */
 } problem_t;
 
 static double elem(const problem_t *p, uint16_t bits) {
@@ -127,16 +147,19 @@ static int key_visible(const problem_t *p, int i, int j) {
 }
 
 static double q_at(const problem_t *p, int b, int i, int h, int c) {
-    return elem(p, p->q[(((size_t)b * p->Nq + i) * p->Hq + h) * p->d + c]);
+    const size_t at = (((size_t)b * p->Nq + i) * p->Hq + h) * p->d + c;
+    return p->q8 ? p->dq * e4m3_bits_to_double(p->q8[at]) : elem(p, p->q[at]);
 }
 static double k_at(const problem_t *p, int b, int j, int g, int c) {
-    return elem(p, p->k[(((size_t)b * p->Nk + j) * p->Hkv + g) * p->d + c]);
+    const size_t at = (((size_t)b * p->Nk + j) * p->Hkv + g) * p->d + c;
+    return p->k8 ? p->dk * e4m3_bits_to_double(p->k8[at]) : elem(p, p->k[at]);
 }
 static double v_at(const problem_t *p, int b, int j, int g, int c) {
 #ifdef ORACLE_PLANT_TRANSPOSE_V
     c = p->d - 1 - c;
 #endif
-    return elem(p, p->v[(((size_t)b * p->Nk + j) * p->Hkv + g) * p->d + c]);
+    const size_t at = (((size_t)b * p->Nk + j) * p->Hkv + g) * p->d + c;
+    return p->v8 ? p->dv * e4m3_bits_to_double(p->v8[at]) : elem(p, p->v[at]);
 }
 
 /*
@@ -271,7 +294,7 @@ static int run_full(const problem_t *p, double *out, double *lse, double *probs,
 int oracle_attention_fwd(const uint16_t *q, const uint16_t *k, const uint16_t *v,
                          double *out, double *lse, int B, int Hq, int Hkv, int Nq, int Nk,
                          int d, double scale, int causal, int window, int elem_f16, int nthreads) {
-    problem_t p = {q, k, v, B, Hq, Hkv, Nq, Nk, d, scale, causal ? 1 : 0, window, elem_f16 ? 1 : 0};
+    problem_t p = {q, k, v, B, Hq, Hkv, Nq, Nk, d, scale, causal ? 1 : 0, window, elem_f16 ? 1 : 0, NULL, NULL, NULL, 1.0, 1.0, 1.0};
     return run_full(&p, out, lse, NULL, nthreads);
 }
 
@@ -282,7 +305,7 @@ int oracle_attention_fwd(const uint16_t *q, const uint16_t *k, const uint16_t *v
 int oracle_attention_probs(const uint16_t *q, const uint16_t *k, const uint16_t *v,
                            double *out, double *lse, double *probs, int B, int Hq, int Hkv,
                            int Nq, int Nk, int d, double scale, int causal, int window, int elem_f16) {
-    problem_t p = {q, k, v, B, Hq, Hkv, Nq, Nk, d, scale, causal ? 1 : 0, window, elem_f16 ? 1 : 0};
+    problem_t p = {q, k, v, B, Hq, Hkv, Nq, Nk, d, scale, causal ? 1 : 0, window, elem_f16 ? 1 : 0, NULL, NULL, NULL, 1.0, 1.0, 1.0};
     return run_full(&p, out, lse, probs, 1);
 }
 
@@ -310,15 +333,11 @@ static void *rows_worker(void *arg) {
     return NULL;
 }
 
-/*
- * oracle_attention_rows: O and LSE of the listed rows only.
- *   rows: nrows triples (b, hq, i), each in range; out_rows [nrows, d]; lse_rows [nrows].
- */
-int oracle_attention_rows(const uint16_t *q, const uint16_t *k, const uint16_t *v,
-                          const int32_t *rows, long nrows, double *out_rows, double *lse_rows,
-                          int B, int Hq, int Hkv, int Nq, int Nk, int d, double scale,
-                          int causal, int window, int elem_f16, int nthreads) {
-    problem_t p = {q, k, v, B, Hq, Hkv, Nq, Nk, d, scale, causal ? 1 : 0, window, elem_f16 ? 1 : 0};
+/* O and LSE of the listed rows only (shared by the bit-pattern and E4M3 entry points). */
+static int run_rows(const problem_t *pp, const int32_t *rows, long nrows, double *out_rows, double *lse_rows,
+                    int nthreads) {
+    const problem_t p = *pp;
+    const int B = p.B, Hq = p.Hq, Nq = p.Nq;
     if (!check_problem(&p) || nrows < 0) return ORACLE_EINVAL;
     for (long r = 0; r < nrows; ++r) {
         int b = rows[3 * r], hq = rows[3 * r + 1], i = rows[3 * r + 2];
@@ -342,6 +361,29 @@ int oracle_attention_rows(const uint16_t *q, const uint16_t *k, const uint16_t *
     free(tid);
     free(jobs);
     return rc;
+}
+
+/*
+ * oracle_attention_rows: O and LSE of the listed rows only.
+ *   rows: nrows triples (b, hq, i), each in range; out_rows [nrows, d]; lse_rows [nrows].
+ */
+int oracle_attention_rows(const uint16_t *q, const uint16_t *k, const uint16_t *v,
+                          const int32_t *rows, long nrows, double *out_rows, double *lse_rows,
+                          int B, int Hq, int Hkv, int Nq, int Nk, int d, double scale,
+                          int causal, int window, int elem_f16, int nthreads) {
+    problem_t p = {q, k, v, B, Hq, Hkv, Nq, Nk, d, scale, causal ? 1 : 0, window, elem_f16 ? 1 : 0,
+                   NULL, NULL, NULL, 1.0, 1.0, 1.0};
+    return run_rows(&p, rows, nrows, out_rows, lse_rows, nthreads);
+}
+
+/* oracle_attention_rows_fp8: the same for E4M3 inputs with dequantisation factors. */
+int oracle_attention_rows_fp8(const uint8_t *q8, const uint8_t *k8, const uint8_t *v8, const int32_t *rows,
+                              long nrows, double *out_rows, double *lse_rows, int B, int Hq, int Hkv, int Nq, int Nk,
+                              int d, double scale, double dq, double dk, double dv, int causal, int window,
+                              int nthreads) {
+    problem_t p = {NULL, NULL, NULL, B, Hq, Hkv, Nq, Nk, d, scale, causal ? 1 : 0, window, 0, q8, k8, v8, dq, dk, dv};
+    if (!q8 || !k8 || !v8) return ORACLE_EINVAL;
+    return run_rows(&p, rows, nrows, out_rows, lse_rows, nthreads);
 }
 
 /* ---- backward: gradients of L = sum_{b,i,h,c} O[b,i,h,c] dO[b,i,h,c] ---- */
@@ -425,7 +467,7 @@ static void *bwd_worker(void *arg) {
 int oracle_attention_bwd(const uint16_t *q, const uint16_t *k, const uint16_t *v, const uint16_t *dout,
                          double *dq, double *dk, double *dv, int B, int Hq, int Hkv, int Nq, int Nk,
                          int d, double scale, int causal, int window, int elem_f16, int nthreads) {
-    problem_t p = {q, k, v, B, Hq, Hkv, Nq, Nk, d, scale, causal ? 1 : 0, window, elem_f16 ? 1 : 0};
+    problem_t p = {q, k, v, B, Hq, Hkv, Nq, Nk, d, scale, causal ? 1 : 0, window, elem_f16 ? 1 : 0, NULL, NULL, NULL, 1.0, 1.0, 1.0};
     if (!check_problem(&p)) return ORACLE_EINVAL;
     memset(dq, 0, sizeof(double) * (size_t)B * Nq * Hq * d);
     memset(dk, 0, sizeof(double) * (size_t)B * Nk * Hkv * d);
@@ -449,4 +491,17 @@ int oracle_attention_bwd(const uint16_t *q, const uint16_t *k, const uint16_t *v
     free(tid);
     free(jobs);
     return rc;
+}
+
+/*
+ * oracle_attention_fwd_fp8 / oracle_attention_rows_fp8: the same forward (all rows, or
+ * listed rows) for E4M3 inputs q8, k8, v8 (one byte per element, layouts as above) with
+ * dequantisation factors dq, dk, dv: Q = dq * q8 and so on.
+ */
+int oracle_attention_fwd_fp8(const uint8_t *q8, const uint8_t *k8, const uint8_t *v8, double *out, double *lse,
+                             int B, int Hq, int Hkv, int Nq, int Nk, int d, double scale, double dq, double dk,
+                             double dv, int causal, int window, int nthreads) {
+    problem_t p = {NULL, NULL, NULL, B, Hq, Hkv, Nq, Nk, d, scale, causal ? 1 : 0, window, 0, q8, k8, v8, dq, dk, dv};
+    if (!q8 || !k8 || !v8 || !isfinite(dq) || !isfinite(dk) || !isfinite(dv)) return ORACLE_EINVAL;
+    return run_full(&p, out, lse, NULL, nthreads);
 }

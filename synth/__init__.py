@@ -118,7 +118,7 @@ class Workload:
     seed: int = 0
     window: int = 0          # sliding window of W keys (0: none; implies causal)
     splitkv: bool = False    # run with the library's default split-KV count (decode shapes)
-    dtype: str = "bf16"      # element type of q, k, v and out: "bf16" or "f16" (IEEE half)
+    dtype: str = "bf16"      # element type of q, k, v: "bf16", "f16" (IEEE half) or "e4m3" (OCP FP8; out bf16)
 
     @property
     def scale(self) -> float:
@@ -138,10 +138,11 @@ class Workload:
 
     @property
     def io_bytes(self) -> int:
-        """Algorithmic HBM bytes: Q, K, V read once, O written once (bf16), LSE fp32."""
+        """Algorithmic HBM bytes: Q, K, V read once, O written once (2-byte), LSE fp32."""
         q = self.B * self.Nq * self.Hq * self.d
         kv = self.B * self.Nk * self.Hkv * self.d
-        return 2 * (2 * q + 2 * kv) + 4 * self.B * self.Hq * self.Nq
+        es = 1 if self.dtype == "e4m3" else 2     # input element bytes; O is 2-byte either way
+        return es * (q + 2 * kv) + 2 * q + 4 * self.B * self.Hq * self.Nq
 
     def with_(self, **kw) -> "Workload":
         return replace(self, **kw)
@@ -152,10 +153,25 @@ def f32_to_f16_bits(x: np.ndarray) -> np.ndarray:
     return np.asarray(x, dtype=np.float32).astype(np.float16).view(np.uint16)
 
 
+def f32_to_e4m3_bits(x: np.ndarray) -> np.ndarray:
+    """fp32 -> OCP FP8 E4M3 (round to nearest even, torch's cast), as uint8 bytes."""
+    import torch
+    t = torch.from_numpy(np.ascontiguousarray(x, dtype=np.float32))
+    return t.to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+
+
 def make_inputs(w: Workload) -> dict[str, np.ndarray]:
     """Seeded bf16 (w.dtype "f16": IEEE half) bit patterns for q [B,Nq,Hq,d], k and v
     [B,Nk,Hkv,d].  The fp16 inputs are the same normal draws rounded to half, with the
     power-of-two multipliers applied before rounding (exact either way)."""
+    if w.dtype == "e4m3":   # FP8 bytes of the same draws (times the multipliers); |x| << 448
+        shapes = {"q": (w.B, w.Nq, w.Hq, w.d), "k": (w.B, w.Nk, w.Hkv, w.d), "v": (w.B, w.Nk, w.Hkv, w.d)}
+        out = {}
+        for name, shp in shapes.items():
+            z = normal_f64(stream_key(w.seed, w.wid, TENSOR_IDS[name]), int(np.prod(shp)))
+            mult = {"q": w.q_mult, "k": w.k_mult}.get(name, 1.0)
+            out[name] = f32_to_e4m3_bits(z.astype(np.float32) * np.float32(mult)).reshape(shp)
+        return out
     if w.dtype == "f16":
         shapes = {"q": (w.B, w.Nq, w.Hq, w.d), "k": (w.B, w.Nk, w.Hkv, w.d), "v": (w.B, w.Nk, w.Hkv, w.d)}
         out = {}

@@ -48,10 +48,20 @@ def visible(i, j, Nq, Nk, causal, window=0):
 
 # ---------------------------------------------------------------- brute force
 
+def e4m3_f64(bits):
+    """OCP E4M3 bytes widened by torch's own float8_e4m3fn type (exact)."""
+    import torch
+    return torch.from_numpy(np.ascontiguousarray(bits, dtype=np.uint8)).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+
+
 def brute_force_decimal(x, scale, causal, prec=40, window=0, dtype="bf16"):
     """O and LSE by the definition in `prec`-digit decimal arithmetic (tiny inputs)."""
+    return brute_force_values(*(bits_f64(x[n], dtype) for n in ("q", "k", "v")), scale, causal, prec, window)
+
+
+def brute_force_values(q, k, v, scale, causal, prec=40, window=0):
+    """The same on already-decoded float64 arrays q, k, v."""
     getcontext().prec = prec
-    q, k, v = (bits_f64(x[n], dtype) for n in ("q", "k", "v"))
     B, Nq, Hq, d = q.shape
     _, Nk, Hkv, _ = k.shape
     rep = Hq // Hkv
@@ -531,3 +541,60 @@ def pin_bwd_causal_first_row(orc):
 BWD_PINS = [pin_bwd_finite_difference, pin_bwd_one_key, pin_bwd_dk_sums_to_zero, pin_bwd_gqa_is_summed_mha,
             pin_bwd_causal_first_row]
 ALL_PINS = ALL_PINS + BWD_PINS
+
+
+# ---------------------------------------------------------------- FP8 (E4M3) inputs
+
+def _fp8_inputs(B, Hq, Hkv, Nq, Nk, d, seed, q_mult=1.0):
+    w = synth.Workload("tinyfp8", 4000 + seed, B, Hq, Hkv, Nq, Nk, d, False, q_mult=q_mult, seed=seed, dtype="e4m3")
+    return synth.make_inputs(w)
+
+
+def pin_e4m3_decode_every_pattern(orc):
+    """One key: O = dv * v8 exactly, so every non-NaN E4M3 byte placed in v comes back as
+    torch's float8_e4m3fn value (normals, subnormals, both zeros, both signs)."""
+    pats = np.arange(256, dtype=np.uint8)
+    pats = pats[(pats & 0x7F) != 0x7F]
+    z = np.zeros((1, 1, 1, pats.size), np.uint8)
+    O, L = orc.forward_fp8(z, z, pats.reshape(1, 1, 1, -1), 1.0, False)
+    assert np.array_equal(O[0, 0, 0], e4m3_f64(pats)), "e4m3 decode"
+    O2, _ = orc.forward_fp8(z, z, pats.reshape(1, 1, 1, -1), 1.0, False, descale=(1.0, 1.0, 0.375))
+    assert np.array_equal(O2[0, 0, 0], 0.375 * e4m3_f64(pats)), "dv applied to V"
+    assert L[0, 0, 0] == 0.0
+
+
+def pin_e4m3_known_values(orc):
+    """E4M3 values fixed by the format: 1, -1, the largest finite 448, the smallest normal
+    2^-6, the smallest subnormal 2^-9, 1.125 (one fraction step above 1)."""
+    table = {0x38: 1.0, 0xB8: -1.0, 0x7E: 448.0, 0x08: 2.0 ** -6, 0x01: 2.0 ** -9, 0x39: 1.125}
+    v = np.array(list(table), dtype=np.uint8).reshape(1, 1, 1, -1)
+    z = np.zeros_like(v)
+    O, _ = orc.forward_fp8(z, z, v, 1.0, False)
+    assert list(O[0, 0, 0]) == list(table.values()), O[0, 0, 0]
+
+
+def pin_fp8_brute_force_with_descales(orc):
+    """Decimal brute force on Q = dq q8, K = dk k8, V = dv v8 (torch-decoded bytes)."""
+    for (B, Hq, Hkv, Nq, Nk, d, causal, seed, ds) in [(1, 2, 1, 5, 6, 32, False, 80, (0.5, 2.0, 0.25)),
+                                                       (1, 2, 2, 6, 4, 16, True, 81, (0.125, 1.0, 3.0))]:
+        x = _fp8_inputs(B, Hq, Hkv, Nq, Nk, d, seed, q_mult=4.0)
+        scale = 1.0 / math.sqrt(d)
+        O, L = orc.forward_fp8(x["q"], x["k"], x["v"], scale, causal, descale=ds)
+        qf, kf, vf = (c * e4m3_f64(x[n]) for c, n in zip(ds, ("q", "k", "v")))
+        Ob, Lb = brute_force_values(qf, kf, vf, scale, causal)
+        assert_close(O, Ob, what="fp8 O brute")
+        assert_close(L, Lb, what="fp8 LSE brute")
+
+
+def pin_fp8_rows_match_full(orc):
+    x = _fp8_inputs(2, 4, 2, 9, 13, 32, seed=82)
+    O, L = orc.forward_fp8(x["q"], x["k"], x["v"], 0.2, True, descale=(0.5, 0.5, 2.0))
+    rows = np.array([(0, 0, 0), (1, 3, 8), (0, 2, 4), (1, 1, 2)], dtype=np.int32)
+    Or, Lr = orc.rows_fp8(x["q"], x["k"], x["v"], rows, 0.2, True, descale=(0.5, 0.5, 2.0))
+    for n, (b, h, i) in enumerate(rows):
+        assert np.array_equal(Or[n], O[b, i, h]) and Lr[n] == L[b, h, i]
+
+
+FP8_PINS = [pin_e4m3_decode_every_pattern, pin_e4m3_known_values, pin_fp8_brute_force_with_descales,
+            pin_fp8_rows_match_full]
+ALL_PINS = ALL_PINS + FP8_PINS

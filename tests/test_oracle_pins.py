@@ -71,7 +71,7 @@ def test_invalid_sizes_rejected(orc):
 MUTANTS = ["ORACLE_PLANT_NO_SCALE", "ORACLE_PLANT_GQA_MODULO", "ORACLE_PLANT_CAUSAL_STRICT",
            "ORACLE_PLANT_TRANSPOSE_V", "ORACLE_PLANT_LSE_NO_MAX", "ORACLE_PLANT_NO_NORMALIZE",
            "ORACLE_PLANT_WINDOW_OFF_BY_ONE", "ORACLE_PLANT_F16_BIAS", "ORACLE_PLANT_BWD_NO_D",
-           "ORACLE_PLANT_BWD_DQ_NO_SCALE", "ORACLE_PLANT_BWD_DV_NO_P"]
+           "ORACLE_PLANT_BWD_DQ_NO_SCALE", "ORACLE_PLANT_BWD_DV_NO_P", "ORACLE_PLANT_E4M3_BIAS"]
 
 
 @pytest.mark.parametrize("mutant", MUTANTS)
@@ -79,7 +79,7 @@ def test_pins_catch_planted_mistake(mutant):
     """Each planted mistake (dropped scale, modulo GQA mapping, diagonal masked,
     transposed V index, LSE without the max, missing normalisation, window one key too
     wide, fp16 exponent bias off by one, backward without the D term, dQ without the
-    scale, dV without the P weights) fails a pin."""
+    scale, dV without the P weights, E4M3 exponent bias off by one) fails a pin."""
     with tempfile.TemporaryDirectory() as td:
         lib = oracle.build(Path(td) / f"lib_{mutant}.so", defines=(mutant,))
         bad = oracle.Oracle(lib)
