@@ -48,6 +48,15 @@ def peaks():
     return dict(FALLBACK_PEAKS)
 
 
+def tensor_peak(pk, w):
+    """(TFLOP/s, source) of the tensor roofline for a workload's dtype: the measured bf16
+    figure (fp16 has the same nominal rate); E4M3 takes it x 2, the nominal dense fp8/bf16
+    ratio (4.5 / 2.25 PFLOP/s)."""
+    if w.dtype == "e4m3":
+        return 2.0 * pk["bf16_tflops"], f"{pk['source']} bf16 dense (burst) x 2 (nominal fp8/bf16 ratio)"
+    return pk["bf16_tflops"], f"{pk['source']} bf16 dense (burst)"
+
+
 def kernel_source_hash() -> str:
     h = hashlib.sha256()
     for f in sorted((ROOT / "exact_attention_146_b200" / "csrc").glob("*")):
@@ -209,6 +218,23 @@ def run_reference(args, w, world, rank):
     return 0
 
 
+def device_inputs(torch, x, w, pin=False):
+    """q, k, v of a workload as torch tensors: bf16 / fp16 bits, or E4M3 bytes (uint8)."""
+    if w.dtype == "e4m3":
+        ts = {n: torch.from_numpy(np.ascontiguousarray(x[n])) for n in ("q", "k", "v")}
+    else:
+        tdt = torch.float16 if w.dtype == "f16" else torch.bfloat16
+        ts = {n: torch.from_numpy(x[n].view(np.int16)).view(tdt) for n in ("q", "k", "v")}
+    return {n: (t.pin_memory() if pin else t) for n, t in ts.items()}
+
+
+def forward_call(fa, w, q, k, v, out, lse, **kw):
+    """The entry point a workload runs through (fa_fwd_fp8 for E4M3 inputs)."""
+    if w.dtype == "e4m3":
+        return fa.fa_fwd_fp8(q, k, v, causal=w.causal, scale=w.scale, out=out, lse=lse)
+    return fa.fa_fwd(q, k, v, causal=w.causal, scale=w.scale, out=out, lse=lse, **kw)
+
+
 def run_ours(args, w, world, rank, local):
     import torch
     import exact_attention_146_b200 as fa
@@ -226,10 +252,9 @@ def run_ours(args, w, world, rank, local):
     # per-rank replica of the workload on its own seeded data (weak scaling)
     wr = rank_workload(w, rank)
     x = synth.make_inputs(wr)
-    tdt = torch.float16 if w.dtype == "f16" else torch.bfloat16
-    host = {n: torch.from_numpy(x[n].view(np.int16)).view(tdt).pin_memory() for n in ("q", "k", "v")}
+    host = device_inputs(torch, x, w, pin=True)
     q, k, v = (host[n].to(dev, non_blocking=True) for n in ("q", "k", "v"))
-    out = torch.empty_like(q)
+    out = torch.empty(q.shape, dtype=torch.bfloat16 if w.dtype == "e4m3" else q.dtype, device=dev)
     lse = torch.empty((w.B, w.Hq, w.Nq), dtype=torch.float32, device=dev)
     # split-KV workloads: the library's default split count, workspace allocated once here
     splits = (fa.splitkv_default_splits(w.B, w.Hq, w.Hkv, w.Nq, w.Nk, w.d,
@@ -242,7 +267,7 @@ def run_ours(args, w, world, rank, local):
     torch.cuda.synchronize()
 
     def step():
-        fa.fa_fwd(q, k, v, causal=w.causal, scale=w.scale, out=out, lse=lse, **call_kw)
+        forward_call(fa, w, q, k, v, out, lse, **call_kw)
 
     for _ in range(args.warmup):
         step()
@@ -287,9 +312,9 @@ def run_ours(args, w, world, rank, local):
                     "tflops": achieved}
     else:
         # fp16 takes the bf16 figure: the nominal dense fp16 and bf16 tensor rates are equal
-        roofline = {"bound": "tensor", "achieved": achieved, "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
-                    "frac": achieved / pk["bf16_tflops"], "traffic": profiled_traffic(w.name),
-                    "peak_source": f"{pk['source']} bf16 dense (burst)",
+        tp, tsrc = tensor_peak(pk, w)
+        roofline = {"bound": "tensor", "achieved": achieved, "peak": tp, "unit": "TFLOP/s",
+                    "frac": achieved / tp, "traffic": profiled_traffic(w.name), "peak_source": tsrc,
                     "algorithmic_bytes": w.io_bytes, "hbm_gbs": gbs}
 
     # end to end through the public API: pinned host inputs in, O and LSE back to host
@@ -303,7 +328,7 @@ def run_ours(args, w, world, rank, local):
             q.copy_(host["q"], non_blocking=True)
             k.copy_(host["k"], non_blocking=True)
             v.copy_(host["v"], non_blocking=True)
-            fa.fa_fwd(q, k, v, causal=w.causal, scale=w.scale, out=out, lse=lse, **call_kw)
+            forward_call(fa, w, q, k, v, out, lse, **call_kw)
             out_h.copy_(out, non_blocking=True)
             lse_h.copy_(lse, non_blocking=True)
 
@@ -318,7 +343,7 @@ def run_ours(args, w, world, rank, local):
         f1.record(stream)
         torch.cuda.synchronize()
         ms_e2e = max_over_ranks(f0.elapsed_time(f1) / n_e2e, pg, dev)
-        h2d = sum(host[n].numel() * 2 for n in ("q", "k", "v"))
+        h2d = sum(host[n].numel() * host[n].element_size() for n in ("q", "k", "v"))
         d2h = out.numel() * 2 + lse.numel() * 4
         e2e = {"value": weak_scaling_tflops(w, world, ms_e2e), "unit": "TFLOP/s", "ms_per_step": ms_e2e,
                "steps": n_e2e, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
@@ -415,9 +440,9 @@ def run_sweep(args):
     for name in names:
         w = synth.WORKLOADS[name]
         x = synth.make_inputs(w)
-        tdt = torch.float16 if w.dtype == "f16" else torch.bfloat16
-        q, k, v = (torch.from_numpy(x[n].view(np.int16)).view(tdt).cuda() for n in ("q", "k", "v"))
-        out = torch.empty_like(q)
+        ti = device_inputs(torch, x, w)
+        q, k, v = (ti[n].cuda() for n in ("q", "k", "v"))
+        out = torch.empty(q.shape, dtype=torch.bfloat16 if w.dtype == "e4m3" else q.dtype, device="cuda")
         lse = torch.empty((w.B, w.Hq, w.Nq), dtype=torch.float32, device="cuda")
         # inputs smaller than L2 are timed both warm and with an L2 flush before each launch
         flush = torch.empty(int(2 * 126e6) // 4, dtype=torch.float32, device="cuda")
@@ -426,12 +451,12 @@ def run_sweep(args):
         ws = torch.empty(max(1, fa.splitkv_workspace_bytes(w.B, w.Hq, w.Nq, w.d, splits)), dtype=torch.uint8, device="cuda") if splits else None
         kw = dict(window=win, num_splits=splits, workspace=ws)
         for _ in range(args.warmup):
-            fa.fa_fwd(q, k, v, causal=w.causal, scale=w.scale, out=out, lse=lse, **kw)
+            forward_call(fa, w, q, k, v, out, lse, **kw)
         torch.cuda.synchronize()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record()
         for _ in range(args.steps):
-            fa.fa_fwd(q, k, v, causal=w.causal, scale=w.scale, out=out, lse=lse, **kw)
+            forward_call(fa, w, q, k, v, out, lse, **kw)
         e1.record()
         torch.cuda.synchronize()
         ms_warm = e0.elapsed_time(e1) / args.steps
@@ -440,16 +465,16 @@ def run_sweep(args):
             flush.zero_()
             a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             a.record()
-            fa.fa_fwd(q, k, v, causal=w.causal, scale=w.scale, out=out, lse=lse, **kw)
+            forward_call(fa, w, q, k, v, out, lse, **kw)
             b.record()
             torch.cuda.synchronize()
             cold.append(a.elapsed_time(b))
         ms_cold = statistics.median(cold)
         st, word = fa.device_status()
-        roof_ms = max(w.flops / (pk["bf16_tflops"] * 1e12), w.io_bytes / (pk["hbm_gbs"] * 1e9)) * 1e3
+        roof_ms = max(w.flops / (tensor_peak(pk, w)[0] * 1e12), w.io_bytes / (pk["hbm_gbs"] * 1e9)) * 1e3
         print(json.dumps({
             "workload": name, "ms_warm": ms_warm, "ms_l2_flushed": ms_cold,
-            "splits": splits, "tflops": w.flops / (ms_cold * 1e-3) / 1e12, "pct_peak": 100 * w.flops / (ms_cold * 1e-3) / 1e12 / pk["bf16_tflops"],
+            "splits": splits, "tflops": w.flops / (ms_cold * 1e-3) / 1e12, "pct_peak": 100 * w.flops / (ms_cold * 1e-3) / 1e12 / tensor_peak(pk, w)[0],
             "hbm_gbs": w.io_bytes / (ms_cold * 1e-3) / 1e9, "roofline_ms": roof_ms,
             "roofline_frac": roof_ms / ms_cold, "status": st}), flush=True)
         del q, k, v, out, lse, flush

@@ -30,7 +30,7 @@ FA_ERR_SCRATCH_LIMIT = 9
 SPLITKV_STATIC_SCRATCH_BYTES = 16 * 1024 * 1024
 
 EXPORTED = ("fa_fwd", "fa_fwd_window", "fa_fwd_splitkv", "fa_splitkv_workspace_bytes", "fa_splitkv_default_splits",
-            "fa_fwd_splitkv_static", "fa_fwd_f16", "fa_bwd", "fa_bwd_workspace_bytes", "fa_status_string", "fa_device_status", "fa_tile_config", "fa_version")
+            "fa_fwd_splitkv_static", "fa_fwd_f16", "fa_fwd_fp8", "fa_bwd", "fa_bwd_workspace_bytes", "fa_status_string", "fa_device_status", "fa_tile_config", "fa_version")
 
 
 class FaError(RuntimeError):
@@ -54,6 +54,8 @@ def lib() -> ctypes.CDLL:
         L.fa_fwd.restype = ci
         L.fa_fwd_f16.argtypes = [vp, vp, vp, vp, vp, ci, ci, ci, ci, ci, ci, cf, ci, vp]
         L.fa_fwd_f16.restype = ci
+        L.fa_fwd_fp8.argtypes = [vp, vp, vp, vp, vp, ci, ci, ci, ci, ci, ci, cf, cf, cf, cf, ci, vp]
+        L.fa_fwd_fp8.restype = ci
         L.fa_fwd_window.argtypes = [vp, vp, vp, vp, vp, ci, ci, ci, ci, ci, ci, cf, ci, vp]
         L.fa_fwd_window.restype = ci
         L.fa_fwd_splitkv.argtypes = [vp, vp, vp, vp, vp, ci, ci, ci, ci, ci, ci, cf, ci, ci, vp, ctypes.c_size_t, vp]
@@ -172,6 +174,38 @@ def fa_fwd(q, k, v, *, causal: bool = False, scale: float | None = None, out=Non
                         B, Hq, Hkv, Nq, Nk, d, scale, 1 if causal else 0, _stream_handle(stream))
     if rc != FA_OK:
         raise FaError(rc)
+    return out, lse
+
+
+def fa_fwd_fp8(q8, k8, v8, *, descale=(1.0, 1.0, 1.0), causal: bool = False, scale: float | None = None, out=None,
+               lse=None, return_lse: bool = True, stream=None):
+    """FP8 forward (fa_fwd_fp8): q8, k8, v8 are [B, N, H, d] uint8 CUDA tensors of OCP E4M3
+    bytes (or torch.float8_e4m3fn), dequantised by descale = (dq, dk, dv); out is bf16."""
+    import torch
+    ts = []
+    for name, t in (("q", q8), ("k", k8), ("v", v8)):
+        if t.dtype == torch.float8_e4m3fn:
+            t = t.view(torch.uint8)
+        if t.dtype != torch.uint8 or not t.is_cuda or not t.is_contiguous() or t.dim() != 4:
+            raise ValueError(f"{name} must be a contiguous 4-D E4M3 (uint8) CUDA tensor, got {t.dtype} {tuple(t.shape)}")
+        ts.append(t)
+    q8, k8, v8 = ts
+    B, Nq, Hq, d = q8.shape
+    Nk, Hkv = k8.shape[1], k8.shape[2]
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if out is None:
+        out = torch.empty((B, Nq, Hq, d), dtype=torch.bfloat16, device=q8.device)
+    if return_lse and lse is None:
+        lse = torch.empty((B, Hq, Nq), dtype=torch.float32, device=q8.device)
+    if not return_lse:
+        lse = None
+    rc = lib().fa_fwd_fp8(q8.data_ptr(), k8.data_ptr(), v8.data_ptr(), out.data_ptr(),
+                          lse.data_ptr() if lse is not None else None, B, Hq, Hkv, Nq, Nk, d, float(scale),
+                          float(descale[0]), float(descale[1]), float(descale[2]), 1 if causal else 0,
+                          _stream_handle(stream))
+    if rc != FA_OK:
+        raise FaError(rc, "fa_fwd_fp8")
     return out, lse
 
 

@@ -32,8 +32,11 @@ template <bool H> using Cfg96 = TileCfg<96, 128, 2, 4, 1, 1, false, 0, H>;
 template <bool H> using Cfg128 = TileCfg<128, 128, 2, 4, 1, 1, false, 0, H>;
 template <bool H> using Cfg192 = TileCfg<192, 64, 2, 4, 1, 1, false, 0, H>;
 template <bool H> using Cfg256 = TileCfg<256, 64, 1, 4, 1, 2, false, 0, H>;
-constexpr int kNumCfgSlots = 18;   // forward: 7 head dims x 2 element types; backward: 2 head dims
+// FP8 (E4M3) inputs, d = 128: 16 KB tiles, so eight K/V slots
+using Cfg128F8 = TileCfg<128, 128, 2, 8, 1, 1, false, 0, false, true>;
+constexpr int kNumCfgSlots = 19;   // forward: 7 head dims x 2 element types; backward: 2 head dims; FP8
 constexpr int kBwdSlot0 = 16;      // backward d = 64, 128 use slots 16, 17
+constexpr int kFp8Slot = 18;
 
 __device__ int g_fa_status;   // per-device kernel status word (0 = OK)
 
@@ -140,17 +143,21 @@ bool overlaps(const void *a, size_t na, const void *b, size_t nb) {
 
 // 4-D view (d, H, N, B) of a [B, N, H, d] bf16 tensor, box (CW, heads, rows, 1): the box
 // lands in shared memory as heads*rows swizzled rows, row-major over (row, head).
+// elem: 0 bf16, 1 fp16, 2 E4M3 bytes.
 int encode_bnhd(CUtensorMap *m, const void *base, int d, int H, int N, int B, int cw, int rows, int heads = 1,
-                bool f16 = false) {
+                int elem = 0) {
     EncodeTiledFn fn = encode_fn();
     if (fn == nullptr) return FA_ERR_CUDA;
     const cuuint64_t dims[4] = {cuuint64_t(d), cuuint64_t(H), cuuint64_t(N), cuuint64_t(B)};
-    const cuuint64_t strides[3] = {cuuint64_t(d) * 2, cuuint64_t(H) * d * 2, cuuint64_t(N) * H * d * 2};
+    const cuuint64_t es = elem == 2 ? 1 : 2;
+    const cuuint64_t strides[3] = {cuuint64_t(d) * es, cuuint64_t(H) * d * es, cuuint64_t(N) * H * d * es};
     const cuuint32_t box[4] = {cuuint32_t(cw), cuuint32_t(heads), cuuint32_t(rows), 1};
     const cuuint32_t estr[4] = {1, 1, 1, 1};
-    const CUtensorMapSwizzle sw = (cw * 2 == 128) ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
-    const CUresult r = fn(m, f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4,
-                          const_cast<void *>(base), dims, strides,
+    const CUtensorMapSwizzle sw = (cw * es == 128) ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
+    const CUtensorMapDataType dt = elem == 2   ? CU_TENSOR_MAP_DATA_TYPE_UINT8
+                                   : elem == 1 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16
+                                               : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+    const CUresult r = fn(m, dt, 4, const_cast<void *>(base), dims, strides,
                           box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS ? FA_OK : FA_ERR_CUDA;
@@ -167,6 +174,7 @@ struct Problem {
     int num_splits;     // 1: plain forward; > 1: split-KV into the workspace, then merge
     float *o_part;      // workspace: fp32 partial O [split][B][Nq][Hq][d]
     float *lse_part;    // workspace: partial LSE [split][B][Hq][Nq]
+    float o_scale;      // FP8: V dequantisation factor (1 otherwise)
 };
 
 // Workspace layout of the split-KV forward: partial O, then (256-byte aligned) partial LSE.
@@ -213,10 +221,11 @@ int launch(const Problem &pr, DeviceState &dev, int cfg_slot, cudaStream_t strea
     CUtensorMap mq, mk, mv;
     int rc;
     const int pack = pack_factor(pr.Hq, pr.Hkv, pr.Nq);
-    if ((rc = encode_bnhd(&mq, pr.q, C::D, pr.Hq, pr.Nq, pr.B, C::CW, kBlockQ / pack, pack, C::F16)) != FA_OK)
+    constexpr int elem = C::FP8 ? 2 : (C::F16 ? 1 : 0);
+    if ((rc = encode_bnhd(&mq, pr.q, C::D, pr.Hq, pr.Nq, pr.B, C::CW, kBlockQ / pack, pack, elem)) != FA_OK)
         return rc;
-    if ((rc = encode_bnhd(&mk, pr.k, C::D, pr.Hkv, pr.Nk, pr.B, C::CW, C::BC, 1, C::F16)) != FA_OK) return rc;
-    if ((rc = encode_bnhd(&mv, pr.v, C::D, pr.Hkv, pr.Nk, pr.B, C::CW, C::BC, 1, C::F16)) != FA_OK) return rc;
+    if ((rc = encode_bnhd(&mk, pr.k, C::D, pr.Hkv, pr.Nk, pr.B, C::CW, C::BC, 1, elem)) != FA_OK) return rc;
+    if ((rc = encode_bnhd(&mv, pr.v, C::D, pr.Hkv, pr.Nk, pr.B, C::CW, C::BC, 1, elem)) != FA_OK) return rc;
 
     FwdParams p{};
     p.out = pr.out;
@@ -241,6 +250,7 @@ int launch(const Problem &pr, DeviceState &dev, int cfg_slot, cudaStream_t strea
     if (units > 0x7fffffffLL) return FA_ERR_INVALID_ARG;
     p.num_units = int(units);
     p.scale_log2 = pr.scale * 1.4426950408889634f;
+    p.o_scale = pr.o_scale;
 
     const int grid = int(units < dev.num_sms ? units : dev.num_sms);
     fa_fwd_kernel<C><<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(mq, mk, mv, p);
@@ -333,7 +343,7 @@ namespace {
 // device memory of the current device), so its device-range check is skipped.
 int forward(const void *q, const void *k, const void *v, void *out, float *lse, int B, int Hq, int Hkv,
             int Nq, int Nk, int d, float scale, int causal, int window, int num_splits, void *workspace,
-            size_t workspace_bytes, void *stream, bool library_scratch = false, bool f16 = false) {
+            size_t workspace_bytes, void *stream, bool library_scratch = false, int elem = 0, float o_scale = 1.f) {
     // ---- host-only validation (no CUDA call before this block passes)
     if (B < 0 || Hq <= 0 || Hkv <= 0 || Nq < 0 || Nk < 0) return FA_ERR_INVALID_ARG;
     if (Hq % Hkv != 0) return FA_ERR_INVALID_ARG;
@@ -342,8 +352,12 @@ int forward(const void *q, const void *k, const void *v, void *out, float *lse, 
     if (num_splits < 1 || num_splits > kMaxSplits) return FA_ERR_INVALID_ARG;
     if (!std::isfinite(scale) || !(scale > 0.f)) return FA_ERR_INVALID_ARG;
     if (tile_config(d, nullptr, nullptr, nullptr, nullptr) != FA_OK) return FA_ERR_UNSUPPORTED_HEAD_DIM;
-    const size_t q_bytes = size_t(B) * size_t(Nq) * size_t(Hq) * size_t(d) * 2;
-    const size_t kv_bytes = size_t(B) * size_t(Nk) * size_t(Hkv) * size_t(d) * 2;
+    if (elem == 2 && d != 128) return FA_ERR_UNSUPPORTED_HEAD_DIM;
+    if (!std::isfinite(o_scale) || !(o_scale > 0.f)) return FA_ERR_INVALID_ARG;
+    const size_t es = elem == 2 ? 1 : 2;   // input element bytes; out is 2-byte
+    const size_t q_bytes = size_t(B) * size_t(Nq) * size_t(Hq) * size_t(d) * es;
+    const size_t out_bytes = size_t(B) * size_t(Nq) * size_t(Hq) * size_t(d) * 2;
+    const size_t kv_bytes = size_t(B) * size_t(Nk) * size_t(Hkv) * size_t(d) * es;
     const size_t lse_bytes = size_t(B) * size_t(Hq) * size_t(Nq) * 4;
     if (q_bytes == 0) return FA_OK;   // B == 0 or Nq == 0: no output rows
     if (q == nullptr || out == nullptr) return FA_ERR_INVALID_ARG;
@@ -351,17 +365,17 @@ int forward(const void *q, const void *k, const void *v, void *out, float *lse, 
     auto mis = [](const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) != 0; };
     if (mis(q, 16) || mis(out, 16) || (kv_bytes > 0 && (mis(k, 16) || mis(v, 16))) || (lse && mis(lse, 4)))
         return FA_ERR_MISALIGNED;
-    if (overlaps(out, q_bytes, q, q_bytes) || overlaps(out, q_bytes, k, kv_bytes) ||
-        overlaps(out, q_bytes, v, kv_bytes) || overlaps(lse, lse_bytes, q, q_bytes) ||
+    if (overlaps(out, out_bytes, q, q_bytes) || overlaps(out, out_bytes, k, kv_bytes) ||
+        overlaps(out, out_bytes, v, kv_bytes) || overlaps(lse, lse_bytes, q, q_bytes) ||
         overlaps(lse, lse_bytes, k, kv_bytes) || overlaps(lse, lse_bytes, v, kv_bytes) ||
-        overlaps(lse, lse_bytes, out, q_bytes))
+        overlaps(lse, lse_bytes, out, out_bytes))
         return FA_ERR_OVERLAP;
     const size_t ws_bytes = (Nk > 0) ? splitkv_bytes(B, Hq, Nq, d, num_splits) : 0;
     if (ws_bytes > 0) {
         if (workspace == nullptr || workspace_bytes < ws_bytes) return FA_ERR_INVALID_ARG;
         if (mis(workspace, 256)) return FA_ERR_MISALIGNED;
         if (overlaps(workspace, ws_bytes, q, q_bytes) || overlaps(workspace, ws_bytes, k, kv_bytes) ||
-            overlaps(workspace, ws_bytes, v, kv_bytes) || overlaps(workspace, ws_bytes, out, q_bytes) ||
+            overlaps(workspace, ws_bytes, v, kv_bytes) || overlaps(workspace, ws_bytes, out, out_bytes) ||
             overlaps(workspace, ws_bytes, lse, lse_bytes))
             return FA_ERR_OVERLAP;
     }
@@ -372,7 +386,7 @@ int forward(const void *q, const void *k, const void *v, void *out, float *lse, 
     int rc = current_device(&dev, &dev_id);
     if (rc != FA_OK) return rc;
     if ((rc = check_device_range(q, q_bytes, dev_id)) != FA_OK) return rc;
-    if ((rc = check_device_range(out, q_bytes, dev_id)) != FA_OK) return rc;
+    if ((rc = check_device_range(out, out_bytes, dev_id)) != FA_OK) return rc;
     if (kv_bytes > 0) {
         if ((rc = check_device_range(k, kv_bytes, dev_id)) != FA_OK) return rc;
         if ((rc = check_device_range(v, kv_bytes, dev_id)) != FA_OK) return rc;
@@ -383,7 +397,7 @@ int forward(const void *q, const void *k, const void *v, void *out, float *lse, 
 
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     if (Nk == 0) {
-        const size_t n16 = q_bytes / 16;
+        const size_t n16 = out_bytes / 16;
         const int grid = int(std::min<size_t>((n16 + 255) / 256, size_t(dev->num_sms) * 8));
         fa_no_keys_kernel<<<grid > 0 ? grid : 1, 256, 0, st>>>(static_cast<uint4 *>(out), n16, lse,
                                                              lse ? size_t(B) * Hq * Nq : 0);
@@ -397,8 +411,9 @@ int forward(const void *q, const void *k, const void *v, void *out, float *lse, 
                                              ((splitkv_o_bytes(B, Hq, Nq, d, num_splits) + 255) & ~size_t(255)));
     }
     const Problem pr{q, k, v, out, lse, B, Hq, Hkv, Nq, Nk, d, scale, causal, window,
-                     ws_bytes > 0 ? num_splits : 1, o_part, lse_part};
-    return f16 ? dispatch<true>(pr, *dev, st) : dispatch<false>(pr, *dev, st);
+                     ws_bytes > 0 ? num_splits : 1, o_part, lse_part, o_scale};
+    if (elem == 2) return launch<Cfg128F8>(pr, *dev, kFp8Slot, st);
+    return elem == 1 ? dispatch<true>(pr, *dev, st) : dispatch<false>(pr, *dev, st);
 }
 
 }  // namespace
@@ -498,7 +513,18 @@ int fa_fwd_splitkv_static(const void *q, const void *k, const void *v, void *out
 
 int fa_fwd_f16(const void *q, const void *k, const void *v, void *out, float *lse, int B, int Hq, int Hkv,
                int Nq, int Nk, int d, float scale, int causal, void *stream) {
-    return forward(q, k, v, out, lse, B, Hq, Hkv, Nq, Nk, d, scale, causal, 0, 1, nullptr, 0, stream, false, true);
+    return forward(q, k, v, out, lse, B, Hq, Hkv, Nq, Nk, d, scale, causal, 0, 1, nullptr, 0, stream, false, 1);
+}
+
+int fa_fwd_fp8(const void *q, const void *k, const void *v, void *out, float *lse, int B, int Hq, int Hkv,
+               int Nq, int Nk, int d, float scale, float descale_q, float descale_k, float descale_v, int causal,
+               void *stream) {
+    if (!std::isfinite(descale_q) || !(descale_q > 0.f) || !std::isfinite(descale_k) || !(descale_k > 0.f))
+        return FA_ERR_INVALID_ARG;
+    const float s = scale * descale_q * descale_k;   // logits of the dequantised Q, K
+    if (!std::isfinite(scale) || !(scale > 0.f) || !std::isfinite(s) || !(s > 0.f)) return FA_ERR_INVALID_ARG;
+    return forward(q, k, v, out, lse, B, Hq, Hkv, Nq, Nk, d, s, causal, 0, 1, nullptr, 0, stream, false, 2,
+                   descale_v);
 }
 
 int fa_fwd_window(const void *q, const void *k, const void *v, void *out, float *lse, int B, int Hq,

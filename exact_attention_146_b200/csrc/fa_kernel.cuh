@@ -63,12 +63,13 @@ struct FwdParams {
     int num_units;        // B * Hq * nqb * num_splits
     float *o_part;        // num_splits > 1: fp32 partial O [split][B][Nq][Hq][d], normalised
     float *lse_part;      // num_splits > 1: partial LSE [split][B][Hq][Nq]
-    float scale_log2;     // scale * log2(e)
+    float scale_log2;     // scale * log2(e) (FP8: times the Q and K dequantisation factors)
+    float o_scale;        // FP8: the V dequantisation factor, applied to O with 1 / l
 };
 
 // Compile-time tiling for one head dimension.
 template <int D_, int BC_, int NQT_, int NS_, int NQB_ = 1, int SB_ = 1, bool PSEP_ = false, int SOFT_EXP_ = 0,
-          bool F16_ = false>
+          bool F16_ = false, bool FP8_ = false>
 struct TileCfg {
     static constexpr int D = D_;        // head dim
     static constexpr int BC = BC_;      // key/value rows per tile
@@ -79,8 +80,12 @@ struct TileCfg {
     static constexpr bool PSEP = PSEP_; // P in TMEM columns of its own instead of over S
     static constexpr int SOFT_EXP = SOFT_EXP_;   // exponentials on the FMA pipe: pairs per 8
     static constexpr bool F16 = F16_;   // element type of Q, K, V, P and O: fp16, else bf16
-    static constexpr int CW = (D == 32) ? 32 : 64;       // elements per swizzled smem row
-    static constexpr int RB = CW * 2;                     // bytes per swizzled row (64 or 128)
+    static constexpr bool FP8 = FP8_;   // Q, K, V and P in OCP E4M3 (kind::f8f6f4); O stays bf16
+    static constexpr int ES = FP8 ? 1 : 2;                // bytes per Q/K/V/P element
+    static constexpr int RB = (D * ES >= 128) ? 128 : 64; // bytes per swizzled smem row
+    static constexpr int CW = RB / ES;                    // elements per swizzled smem row
+    static constexpr int KSTEP = 32 / ES;                 // K elements per MMA (32 bytes)
+    static constexpr int PCOLS = BC * ES / 4;             // TMEM columns of one row of P
     static constexpr int NCH = (D + CW - 1) / CW;         // column chunks of a tile
     static constexpr int Q_CHUNK = kBlockQ * RB;
     static constexpr int KV_CHUNK = BC * RB;
@@ -122,15 +127,17 @@ struct TileCfg {
     static constexpr int CONTROL_REGS = 72;
     static_assert(!REALLOC_REGS || (SOFTMAX_REGS * 32 * SOFTMAX_WARPS + CONTROL_REGS * 128 <= LAUNCH_REGS * THREADS),
                   "register split exceeds the launch budget");
-    static constexpr uint32_t IDESC_S = sm100::idesc_f16kind_f32(kBlockQ, BC, 0, 0, F16);
-    static constexpr uint32_t IDESC_O = sm100::idesc_f16kind_f32(kBlockQ, D, 0, 1, F16);
+    // format code 0 is F16 under kind::f16 and E4M3 under kind::f8f6f4
+    static constexpr uint32_t IDESC_S = sm100::idesc_f16kind_f32(kBlockQ, BC, 0, 0, F16 || FP8);
+    static constexpr uint32_t IDESC_O = sm100::idesc_f16kind_f32(kBlockQ, D, 0, 1, F16 || FP8);
 
     static_assert(NQT == 1 || NQT == 2, "one or two query tiles per unit");
     static_assert(NQB == 1 || NQB == 2, "one or two buffers per query tile");
     static_assert(SB == 1 || SB == 2, "one or two S buffers per query tile");
     static_assert(D % 16 == 0 && D >= 32 && D <= 256, "MMA N and K granularity");
     static_assert(BC % 64 == 0 && BC <= 256, "key tile: whole 32-column TMEM chunks of P");
-    static_assert(P_COL0 + (PSEP ? NQT * BC / 2 : 0) <= TMEM_COLS, "TMEM budget");
+    static_assert(P_COL0 + (PSEP ? NQT * PCOLS : 0) <= TMEM_COLS, "TMEM budget");
+    static_assert(!FP8 || (!F16 && !PSEP && SOFT_EXP == 0 && BC % 128 == 0), "FP8 tiling");
     static_assert(SMEM_BYTES <= 232448, "shared memory budget");
     // Barrier indices (Q barriers indexed t * NQB + buffer, S/P barriers t * SB + buffer).
     // Every barrier is waited on densely (each completion in order) by its waiter, except
@@ -335,11 +342,14 @@ __device__ __forceinline__ void issue_qk(uint32_t sbase, uint32_t tmem, int t, i
     const uint64_t b0 = sm100::opaque(sm100::smem_desc(sbase + C::SMEM_KV + slot * C::KV_TILE, 16, C::SBO, C::LAYOUT));
     const uint32_t d_tmem = tmem + uint32_t((t * C::SB + sbuf) * C::BC);
 #pragma unroll
-    for (int kk = 0; kk < C::D / 16; ++kk) {
+    for (int kk = 0; kk < C::D / C::KSTEP; ++kk) {
         constexpr int kCW = C::CW;
-        const uint32_t a_off = uint32_t(((kk * 16) / kCW) * C::Q_CHUNK + ((kk * 16) % kCW) * 2);
-        const uint32_t b_off = uint32_t(((kk * 16) / kCW) * C::KV_CHUNK + ((kk * 16) % kCW) * 2);
-        sm100::mma_bf16_ss_elected(d_tmem, a0 + (a_off >> 4), b0 + (b_off >> 4), C::IDESC_S, kk > 0 ? 1u : 0u);
+        const uint32_t a_off = uint32_t(((kk * C::KSTEP) / kCW) * C::Q_CHUNK + ((kk * C::KSTEP) % kCW) * C::ES);
+        const uint32_t b_off = uint32_t(((kk * C::KSTEP) / kCW) * C::KV_CHUNK + ((kk * C::KSTEP) % kCW) * C::ES);
+        if constexpr (C::FP8)
+            sm100::mma_f8_ss_elected(d_tmem, a0 + (a_off >> 4), b0 + (b_off >> 4), C::IDESC_S, kk > 0 ? 1u : 0u);
+        else
+            sm100::mma_bf16_ss_elected(d_tmem, a0 + (a_off >> 4), b0 + (b_off >> 4), C::IDESC_S, kk > 0 ? 1u : 0u);
     }
 }
 
@@ -349,12 +359,18 @@ __device__ __forceinline__ void issue_pv(uint32_t sbase, uint32_t tmem, int t, i
     // 64-element column chunks C::KV_CHUNK bytes apart (leading byte offset).  P is the
     // A operand, read from TMEM (16 bf16 = 8 columns per MMA).
     const uint64_t b0 = sm100::opaque(sm100::smem_desc(sbase + C::SMEM_KV + slot * C::KV_TILE, C::KV_CHUNK, C::SBO, C::LAYOUT));
-    const uint32_t a_tmem = tmem + uint32_t(C::PSEP ? C::P_COL0 + t * (C::BC / 2) : (t * C::SB + sbuf) * C::BC);
+    const uint32_t a_tmem = tmem + uint32_t(C::PSEP ? C::P_COL0 + t * C::PCOLS : (t * C::SB + sbuf) * C::BC);
     const uint32_t d_tmem = tmem + uint32_t(C::O_COL0 + t * C::OST);
+    // one MMA takes KSTEP keys: 32 bytes of each P row = 8 TMEM columns, KSTEP rows of V
 #pragma unroll
-    for (int kk = 0; kk < C::BC / 16; ++kk)
-        sm100::mma_bf16_ts_elected(d_tmem, a_tmem + uint32_t(kk * 8), b0 + uint64_t((kk * 16 * C::RB) >> 4), C::IDESC_O,
-                           (accumulate || kk > 0) ? 1u : 0u);
+    for (int kk = 0; kk < C::BC / C::KSTEP; ++kk) {
+        if constexpr (C::FP8)
+            sm100::mma_f8_ts_elected(d_tmem, a_tmem + uint32_t(kk * 8), b0 + uint64_t((kk * C::KSTEP * C::RB) >> 4),
+                                     C::IDESC_O, (accumulate || kk > 0) ? 1u : 0u);
+        else
+            sm100::mma_bf16_ts_elected(d_tmem, a_tmem + uint32_t(kk * 8), b0 + uint64_t((kk * 16 * C::RB) >> 4),
+                                       C::IDESC_O, (accumulate || kk > 0) ? 1u : 0u);
+    }
 }
 
 template <class C>
@@ -499,6 +515,39 @@ __device__ void mma_role(const FwdParams &p, uint32_t sbase, uint32_t tmem, cons
 // exponential to relieve the special-function unit (worth it where the exponentials
 // dominate, i.e. small head dims); masked tiles (which may hold -inf scores) use the
 // hardware ex2 throughout.
+// FP8 P: four exponentials per 32-bit TMEM column (E4M3 bytes), 128 keys per store of
+// 32 columns; the row sum is taken over the unrounded fp32 values, like the LSE.
+template <int BC>
+__device__ __forceinline__ float exp_pack_store_e4m3(const uint32_t (&s)[BC], float c_log2, float neg_m,
+                                                     uint32_t p_taddr) {
+    const uint64_t c2 = sm100::pack2(c_log2, c_log2);
+    const uint64_t nm2 = sm100::pack2(neg_m, neg_m);
+    uint64_t acc0 = sm100::pack2(0.f, 0.f), acc1 = acc0;
+#pragma unroll
+    for (int c = 0; c < BC / 128; ++c) {
+        uint32_t pk[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+            const int e = 128 * c + 4 * i;
+            const uint64_t x01 = sm100::fma2(sm100::pack2(__uint_as_float(s[e]), __uint_as_float(s[e + 1])), c2, nm2);
+            const uint64_t x23 = sm100::fma2(sm100::pack2(__uint_as_float(s[e + 2]), __uint_as_float(s[e + 3])), c2, nm2);
+            float a, b, cc, d;
+            sm100::unpack2(x01, a, b);
+            sm100::unpack2(x23, cc, d);
+            const float p0 = sm100::ex2_approx(a), p1 = sm100::ex2_approx(b);
+            const float p2 = sm100::ex2_approx(cc), p3 = sm100::ex2_approx(d);
+            acc0 = sm100::add2(acc0, sm100::pack2(p0, p1));
+            acc1 = sm100::add2(acc1, sm100::pack2(p2, p3));
+            pk[i] = sm100::pack_e4m3x4(p0, p1, p2, p3);
+        }
+        sm100::tmem_st32(p_taddr + uint32_t(32 * c), pk);
+    }
+    float a0, a1, b0, b1;
+    sm100::unpack2(acc0, a0, a1);
+    sm100::unpack2(acc1, b0, b1);
+    return (a0 + a1) + (b0 + b1);
+}
+
 template <int BC, int SOFT_EXP, bool MIXED, bool F16>
 __device__ __forceinline__ float exp_pack_store(const uint32_t (&s)[BC], float c_log2, float neg_m,
                                                 uint32_t p_taddr) {
@@ -545,7 +594,7 @@ __device__ void softmax_role(const FwdParams &p, uint32_t sbase, uint32_t tmem, 
     const int row_in_tile = quarter * 32 + lane;
     const uint32_t lane_off = uint32_t(quarter * 32) << 16;
     const uint32_t s_taddr0 = tmem + lane_off + uint32_t(t * C::SB * BC);   // S buffer 0 of this tile
-    const uint32_t p_taddr_sep = tmem + lane_off + uint32_t(C::P_COL0 + t * (BC / 2));
+    const uint32_t p_taddr_sep = tmem + lane_off + uint32_t(C::P_COL0 + t * C::PCOLS);
     const uint32_t o_taddr = tmem + lane_off + uint32_t(C::O_COL0 + t * C::OST);
     const float c_log2 = p.scale_log2;
     uint32_t scnt = 0, ocnt = 0, ofin = 0;
@@ -612,8 +661,11 @@ __device__ void softmax_role(const FwdParams &p, uint32_t sbase, uint32_t tmem, 
                     need_rescale = true;
                 }
                 const float neg_m = (m_ref == -INFINITY) ? 0.f : -m_ref;
-                row_sum = need_mask ? exp_pack_store<BC, C::SOFT_EXP, false, C::F16>(s, c_log2, neg_m, p_taddr)
-                                    : exp_pack_store<BC, C::SOFT_EXP, true, C::F16>(s, c_log2, neg_m, p_taddr);
+                if constexpr (C::FP8)
+                    row_sum = exp_pack_store_e4m3<BC>(s, c_log2, neg_m, p_taddr);
+                else
+                    row_sum = need_mask ? exp_pack_store<BC, C::SOFT_EXP, false, C::F16>(s, c_log2, neg_m, p_taddr)
+                                        : exp_pack_store<BC, C::SOFT_EXP, true, C::F16>(s, c_log2, neg_m, p_taddr);
             }
             l = l * alpha + row_sum;
 
@@ -644,7 +696,8 @@ __device__ void softmax_role(const FwdParams &p, uint32_t sbase, uint32_t tmem, 
         }
         ocnt += uint32_t(nk);
         {
-            const float inv_l = l > 0.f ? 1.f / l : 0.f;
+            float inv_l = l > 0.f ? 1.f / l : 0.f;
+            if constexpr (C::FP8) inv_l *= p.o_scale;
             const bool store = row < p.Nq;
             const size_t row_off = (size_t(w.b) * p.Nq + size_t(row)) * p.Hq + hq;   // [b][row][hq]
             const bool split_mode = p.num_splits > 1;

@@ -96,6 +96,20 @@ int fa_fwd_f16(const void *q, const void *k, const void *v, void *out, float *ls
                void *stream);
 
 /*
+ * fa_fwd_fp8 -- fa_fwd on FP8 inputs: q, k, v are OCP E4M3 bytes with one dequantisation
+ * factor per tensor (Q = descale_q * q8, K = descale_k * k8, V = descale_v * v8), the FP8
+ * forward the datacanvas.csdn.net head-dim page attributes to FlashAttention-3.  The tensor
+ * cores multiply E4M3 x E4M3 (kind::f8f6f4) with fp32 accumulation; P is rounded to E4M3
+ * (relative error <= 2^-4) before P V; out is bf16 [B, Nq, Hq, d], lse fp32 as in fa_fwd
+ * (the LSE of the dequantised logits).  d must be 128 (FA_ERR_UNSUPPORTED_HEAD_DIM
+ * otherwise); the descales must be finite and > 0.  Layouts, ownership and the other
+ * errors as fa_fwd (q, k, v one byte per element, 16-byte aligned).
+ */
+int fa_fwd_fp8(const void *q, const void *k, const void *v, void *out, float *lse,
+               int B, int Hq, int Hkv, int Nq, int Nk, int d, float scale,
+               float descale_q, float descale_k, float descale_v, int causal, void *stream);
+
+/*
  * fa_fwd_window -- exact attention forward with a sliding-window (local) causal mask:
  * query row i sees the `window` keys ending at its causal diagonal,
  *

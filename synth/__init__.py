@@ -230,6 +230,7 @@ for _w in [
     _wl("seq4096_b8_h32_d128_f16", 19, 8, 32, 4096, 128, dtype="f16"),
     _wl("gqa_prefill_b4_n4096_hq32_hkv8_d128_causal_f16", 20, 4, 32, 4096, 128, causal=True, Hkv=8, k_mult=0.5,
         dtype="f16"),
+    _wl("seq4096_b8_h32_d128_fp8", 21, 8, 32, 4096, 128, dtype="e4m3"),
 ]:
     WORKLOADS[_w.name] = _w
 

@@ -39,8 +39,16 @@ def tiny(B, Hq, Hkv, Nq, Nk, d, seed, **kw):
 
 def check_full(orc, x, scale, causal, what, dtype="bf16"):
     O, L = _parity.run_cuda(x, scale, causal, dtype=dtype)
+    if dtype == "e4m3":
+        Oref, Lref = orc.forward_fp8(x["q"], x["k"], x["v"], scale, causal)
+        return _parity.compare_fp8(O, L, Oref, Lref, float(np.abs(_pins_e4m3(x["v"])).max()), what)
     Oref, Lref = orc.forward(x["q"], x["k"], x["v"], scale, causal, dtype=dtype)
     return _parity.compare(O, L, Oref, Lref, what)
+
+
+def _pins_e4m3(bits):
+    from tests._pins import e4m3_f64
+    return e4m3_f64(bits)
 
 
 @pytest.mark.parametrize("d", HEAD_DIMS)
@@ -186,6 +194,27 @@ def test_f16_is_not_read_as_bf16(orc):
     assert np.abs(O - Of).max() <= _parity.TOL_O_MAX < np.abs(O - Ob).max()
 
 
+@pytest.mark.parametrize("N", [1, 17, 128, 129, 300, 600])
+@pytest.mark.parametrize("causal", [False, True])
+def test_fp8_small_shapes(orc, N, causal):
+    """E4M3 inputs (fa_fwd_fp8, d = 128) against the oracle reading the same bytes."""
+    x = tiny(1, 2, 1, N, N, 128, seed=N + 11, dtype="e4m3")
+    check_full(orc, x, 1.0 / math.sqrt(128), causal, f"fp8 N={N} causal={causal}", dtype="e4m3")
+
+
+@pytest.mark.parametrize("case", [(2, 8, 2, 200, 700, True, (0.5, 2.0, 0.25)), (1, 32, 8, 16, 3000, False, (1.0, 1.0, 4.0)),
+                                  (2, 6, 3, 130, 129, True, (0.125, 0.75, 1.5)), (1, 4, 4, 1000, 1000, False, (2.0, 2.0, 0.5))])
+def test_fp8_gqa_descales(orc, case):
+    """GQA, ragged lengths, GQA-packed decode rows and non-unit dequantisation factors."""
+    B, Hq, Hkv, Nq, Nk, causal, ds = case
+    x = tiny(B, Hq, Hkv, Nq, Nk, 128, seed=Nq + Nk, q_mult=4.0, dtype="e4m3")
+    scale = 1.0 / math.sqrt(128)
+    O, L = _parity.run_cuda_fp8(x, scale, causal, descale=ds)
+    Oref, Lref = orc.forward_fp8(x["q"], x["k"], x["v"], scale, causal, descale=ds)
+    vmax = ds[2] * float(np.abs(_pins_e4m3(x["v"])).max())
+    _parity.compare_fp8(O, L, Oref, Lref, vmax, f"fp8 {case}")
+
+
 def test_splitkv_matches_plain_forward():
     x = tiny(2, 8, 2, 64, 4096, 128, seed=99)
     O1, L1 = _parity.run_cuda(x, 0.08, False)
@@ -294,6 +323,14 @@ def test_workload_sampled_rows(orc, name):
     oracle one by one, and every output row checked to be written and finite."""
     w = synth.WORKLOADS[name]
     x = synth.make_inputs(w)
+    if w.dtype == "e4m3":
+        O, L = _parity.run_cuda_fp8(x, w.scale, w.causal)
+        rows = _parity.sample_rows(w, 64)
+        Oref, Lref = orc.rows_fp8(x["q"], x["k"], x["v"], rows, w.scale, w.causal)
+        Og = np.stack([O[b, i, h] for (b, h, i) in rows])
+        Lg = np.array([L[b, h, i] for (b, h, i) in rows])
+        _parity.compare_fp8(Og, Lg, Oref, Lref, float(np.abs(_pins_e4m3(x["v"])).max()), name)
+        return
     O, L = _parity.run_cuda(x, w.scale, w.causal, window=w.window or None, num_splits=_parity.workload_splits(w),
                             dtype=w.dtype)
     assert np.isfinite(O).all() and np.isfinite(L).all()
