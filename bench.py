@@ -57,10 +57,15 @@ def tensor_peak(pk, w):
     return pk["bf16_tflops"], f"{pk['source']} bf16 dense (burst)"
 
 
+FORWARD_SOURCES = ("fa_fwd.cu", "fa_host.h", "fa_kernel.cuh", "sm100.cuh")
+
+
 def kernel_source_hash() -> str:
+    """Hash of the sources the forward kernel and its launch are built from (the backward's
+    own files are left out, so they can change without invalidating forward profiles)."""
     h = hashlib.sha256()
-    for f in sorted((ROOT / "exact_attention_146_b200" / "csrc").glob("*")):
-        h.update(f.read_bytes())
+    for name in FORWARD_SOURCES:
+        h.update((ROOT / "exact_attention_146_b200" / "csrc" / name).read_bytes())
     return h.hexdigest()[:16]
 
 

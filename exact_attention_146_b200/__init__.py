@@ -30,7 +30,7 @@ FA_ERR_SCRATCH_LIMIT = 9
 SPLITKV_STATIC_SCRATCH_BYTES = 16 * 1024 * 1024
 
 EXPORTED = ("fa_fwd", "fa_fwd_window", "fa_fwd_splitkv", "fa_splitkv_workspace_bytes", "fa_splitkv_default_splits",
-            "fa_fwd_splitkv_static", "fa_fwd_f16", "fa_fwd_fp8", "fa_bwd", "fa_bwd_workspace_bytes", "fa_status_string", "fa_device_status", "fa_tile_config", "fa_version")
+            "fa_fwd_splitkv_static", "fa_fwd_f16", "fa_fwd_fp8", "fa_fwd_partial", "fa_merge_partials", "fa_bwd", "fa_bwd_workspace_bytes", "fa_status_string", "fa_device_status", "fa_tile_config", "fa_version")
 
 
 class FaError(RuntimeError):
@@ -56,6 +56,10 @@ def lib() -> ctypes.CDLL:
         L.fa_fwd_f16.restype = ci
         L.fa_fwd_fp8.argtypes = [vp, vp, vp, vp, vp, ci, ci, ci, ci, ci, ci, cf, cf, cf, cf, ci, vp]
         L.fa_fwd_fp8.restype = ci
+        L.fa_fwd_partial.argtypes = [vp, vp, vp, vp, vp, ci, ci, ci, ci, ci, ci, cf, ci, ci, ci, vp]
+        L.fa_fwd_partial.restype = ci
+        L.fa_merge_partials.argtypes = [vp, vp, ci, vp, vp, ci, ci, ci, ci, vp]
+        L.fa_merge_partials.restype = ci
         L.fa_fwd_window.argtypes = [vp, vp, vp, vp, vp, ci, ci, ci, ci, ci, ci, cf, ci, vp]
         L.fa_fwd_window.restype = ci
         L.fa_fwd_splitkv.argtypes = [vp, vp, vp, vp, vp, ci, ci, ci, ci, ci, ci, cf, ci, ci, vp, ctypes.c_size_t, vp]
@@ -206,6 +210,45 @@ def fa_fwd_fp8(q8, k8, v8, *, descale=(1.0, 1.0, 1.0), causal: bool = False, sca
                           _stream_handle(stream))
     if rc != FA_OK:
         raise FaError(rc, "fa_fwd_fp8")
+    return out, lse
+
+
+def fa_fwd_partial(q, k, v, *, key_offset: int, nk_total: int, causal: bool = False, scale: float | None = None,
+                   o_part=None, lse_part=None, stream=None):
+    """Partial forward over a key shard (fa_fwd_partial): q [B, Nq, Hq, d] bf16, k/v the
+    shard [B, Nk, Hkv, d] bf16 holding global keys key_offset .. key_offset + Nk - 1 of
+    nk_total.  Returns (o_part [B, Nq, Hq, d] fp32 normalised over the shard, lse_part
+    [B, Hq, Nq] fp32)."""
+    import torch
+    B, Nq, Hq, d = q.shape
+    Nk, Hkv = k.shape[1], k.shape[2]
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if o_part is None:
+        o_part = torch.empty((B, Nq, Hq, d), dtype=torch.float32, device=q.device)
+    if lse_part is None:
+        lse_part = torch.empty((B, Hq, Nq), dtype=torch.float32, device=q.device)
+    rc = lib().fa_fwd_partial(q.data_ptr(), k.data_ptr(), v.data_ptr(), o_part.data_ptr(), lse_part.data_ptr(),
+                              B, Hq, Hkv, Nq, Nk, d, float(scale), 1 if causal else 0, int(key_offset),
+                              int(nk_total), _stream_handle(stream))
+    if rc != FA_OK:
+        raise FaError(rc, "fa_fwd_partial")
+    return o_part, lse_part
+
+
+def fa_merge_partials(o_parts, lse_parts, *, out=None, lse=None, stream=None):
+    """Merge R stacked partials (fa_merge_partials): o_parts [R, B, Nq, Hq, d] fp32,
+    lse_parts [R, B, Hq, Nq] fp32 -> (out [B, Nq, Hq, d] bf16, lse [B, Hq, Nq] fp32)."""
+    import torch
+    R, B, Nq, Hq, d = o_parts.shape
+    if out is None:
+        out = torch.empty((B, Nq, Hq, d), dtype=torch.bfloat16, device=o_parts.device)
+    if lse is None:
+        lse = torch.empty((B, Hq, Nq), dtype=torch.float32, device=o_parts.device)
+    rc = lib().fa_merge_partials(o_parts.data_ptr(), lse_parts.data_ptr(), R, out.data_ptr(), lse.data_ptr(),
+                                 B, Hq, Nq, d, _stream_handle(stream))
+    if rc != FA_OK:
+        raise FaError(rc, "fa_merge_partials")
     return out, lse
 
 

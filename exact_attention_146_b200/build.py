@@ -17,13 +17,13 @@ ROOT = PKG.parent
 CSRC = PKG / "csrc"
 INCLUDE = ROOT / "include"
 LIB = PKG / "libfa.so"
-SOURCES = [CSRC / "fa_fwd.cu"]
-DEPS = SOURCES + sorted(CSRC.glob("*.cuh")) + sorted(INCLUDE.glob("*.h"))
+SOURCES = [CSRC / "fa_fwd.cu", CSRC / "fa_bwd.cu"]
+DEPS = SOURCES + sorted(CSRC.glob("*.cuh")) + sorted(CSRC.glob("*.h")) + sorted(INCLUDE.glob("*.h"))
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",
     "-O3", "-lineinfo", "-std=c++17",
-    "-Xcompiler", "-fPIC", "-shared",
+    "-Xcompiler", "-fPIC",
     "-Xptxas", "-v",
 ]
 
@@ -46,13 +46,32 @@ def build(force: bool = False, verbose: bool = False) -> Path:
     if not force and up_to_date():
         return LIB
     tmp = LIB.with_name(LIB.name + f".tmp{os.getpid()}")
-    cmd = [nvcc(), *NVCC_FLAGS, f"-I{INCLUDE}", f"-I{CSRC}", *map(str, SOURCES), "-o", str(tmp)]
-    res = subprocess.run(cmd, capture_output=True, text=True)
-    if res.returncode != 0:
-        sys.stderr.write(res.stdout + res.stderr)
-        raise RuntimeError("nvcc failed building libfa.so")
-    if verbose:
-        sys.stderr.write(res.stderr)
+    # translation units compile in parallel to objects, then link into the shared library
+    objs = [LIB.with_name(f"{src.stem}.{os.getpid()}.o") for src in SOURCES]
+    procs = [subprocess.Popen([nvcc(), *NVCC_FLAGS, f"-I{INCLUDE}", f"-I{CSRC}", "-c", str(src), "-o", str(o)],
+                              stdout=subprocess.PIPE, stderr=subprocess.PIPE, text=True)
+             for src, o in zip(SOURCES, objs)]
+    try:
+        failed = False
+        for pr in procs:
+            out, err = pr.communicate()
+            if pr.returncode != 0:
+                sys.stderr.write(out + err)
+                failed = True
+            elif verbose:
+                sys.stderr.write(err)
+        if failed:
+            raise RuntimeError("nvcc failed building libfa.so")
+        link = [nvcc(), "-gencode", "arch=compute_100a,code=sm_100a", "-shared", *map(str, objs),
+                "-o", str(tmp)]
+        res = subprocess.run(link, capture_output=True, text=True)
+        if res.returncode != 0:
+            sys.stderr.write(res.stdout + res.stderr)
+            raise RuntimeError("nvcc failed linking libfa.so")
+    finally:
+        for o in objs:
+            if o.exists():
+                o.unlink()
     os.replace(tmp, LIB)
     return LIB
 

@@ -1,0 +1,172 @@
+// fa_bwd.cu -- the C ABI of the backward pass (declared in include/fa.h): argument
+// validation, workspace layout, tensor maps and the three launches (D and the zeroed dQ
+// accumulator, the main kernel of fa_bwd_kernel.cuh, dQ = bf16(scale * acc)).
+#include <algorithm>
+#include <cmath>
+#include <cstdint>
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "fa.h"
+#include "fa_bwd_kernel.cuh"
+#include "fa_host.h"
+
+// ------------------------------------------------------------------ backward
+
+namespace {
+
+using namespace fa_host;
+
+using BwdCfg64 = fa::bwd::BwdCfg<64>;
+using BwdCfg128 = fa::bwd::BwdCfg<128>;
+
+// Workspace of the backward: the fp32 dQ accumulator [B, Nq, Hq, d], then (256-byte
+// aligned) D = rowsum(dO * O) [B, Hq, Nq].
+size_t bwd_acc_bytes(int B, int Hq, int Nq, int d) {
+    return (size_t(B) * size_t(Nq) * size_t(Hq) * size_t(d) * 4 + 255) & ~size_t(255);
+}
+size_t bwd_bytes(int B, int Hq, int Nq, int d) {
+    return bwd_acc_bytes(B, Hq, Nq, d) + size_t(B) * size_t(Hq) * size_t(Nq) * 4;
+}
+
+template <class C>
+int launch_bwd(const void *q, const void *k, const void *v, const void *out, const void *dout, const float *lse,
+               void *dq, void *dk, void *dv, int B, int Hq, int Hkv, int Nq, int Nk, float scale, int causal,
+               float *dq_acc, float *delta, DeviceState &dev, int slot, cudaStream_t st) {
+    auto kern = fa::bwd::fa_bwd_kernel<C>;
+    if (!dev.smem_attr_set[slot]) {
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) != cudaSuccess) {
+            cudaGetLastError();
+            return FA_ERR_CUDA;
+        }
+        dev.smem_attr_set[slot] = true;
+    }
+    CUtensorMap mq, mk, mv, mdo;
+    int rc;
+    if ((rc = encode_bnhd(&mq, q, C::D, Hq, Nq, B, C::CW, fa::bwd::kRows)) != FA_OK) return rc;
+    if ((rc = encode_bnhd(&mdo, dout, C::D, Hq, Nq, B, C::CW, fa::bwd::kRows)) != FA_OK) return rc;
+    if ((rc = encode_bnhd(&mk, k, C::D, Hkv, Nk, B, C::CW, fa::bwd::kRows)) != FA_OK) return rc;
+    if ((rc = encode_bnhd(&mv, v, C::D, Hkv, Nk, B, C::CW, fa::bwd::kRows)) != FA_OK) return rc;
+
+    // D and the zeroed accumulator
+    const long long rows = (long long)B * Nq * Hq;
+    const long long want = (rows + 7) / 8;
+    const int pgrid = int(want < 8LL * dev.num_sms ? want : 8LL * dev.num_sms);
+    fa::bwd::fa_bwd_pre_kernel<C::D><<<pgrid > 0 ? pgrid : 1, 256, 0, st>>>(
+        static_cast<const uint16_t *>(out), static_cast<const uint16_t *>(dout), delta, dq_acc, B, Hq, Nq);
+    if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
+
+    fa::bwd::BwdParams p{};
+    p.lse = lse;
+    p.delta = delta;
+    p.dq_acc = dq_acc;
+    p.dk = static_cast<uint16_t *>(dk);
+    p.dv = static_cast<uint16_t *>(dv);
+    p.status = dev.status_ptr;
+    p.B = B;
+    p.Hq = Hq;
+    p.Hkv = Hkv;
+    p.Nq = Nq;
+    p.Nk = Nk;
+    p.n_rep = Hq / Hkv;
+    p.causal = causal;
+    p.nkt = (Nk + fa::bwd::kRows - 1) / fa::bwd::kRows;
+    p.nqt = (Nq + fa::bwd::kRows - 1) / fa::bwd::kRows;
+    const long long units = (long long)B * Hkv * p.nkt;
+    if (units > 0x7fffffffLL) return FA_ERR_INVALID_ARG;
+    p.num_units = int(units);
+    p.scale = scale;
+    p.scale_log2 = scale * 1.4426950408889634f;
+    const int grid = int(units < dev.num_sms ? units : dev.num_sms);
+    kern<<<grid, C::THREADS, C::SMEM_BYTES, st>>>(mq, mk, mv, mdo, p);
+    if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
+
+    const size_t n4 = size_t(rows) * C::D / 4;
+    const int qgrid = int(std::min<size_t>((n4 + 255) / 256, size_t(dev.num_sms) * 8));
+    fa::bwd::fa_bwd_post_kernel<<<qgrid > 0 ? qgrid : 1, 256, 0, st>>>(reinterpret_cast<const float4 *>(dq_acc),
+                                                                      static_cast<uint2 *>(dq), n4, scale);
+    return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t fa_bwd_workspace_bytes(int B, int Hq, int Nq, int d) {
+    if (B < 0 || Hq < 0 || Nq < 0 || d <= 0) return 0;
+    return bwd_bytes(B, Hq, Nq, d);
+}
+
+int fa_bwd(const void *q, const void *k, const void *v, const void *out, const void *dout, const float *lse,
+           void *dq, void *dk, void *dv, int B, int Hq, int Hkv, int Nq, int Nk, int d, float scale, int causal,
+           void *workspace, size_t workspace_bytes, void *stream) {
+    // ---- host-only validation
+    if (B < 0 || Hq <= 0 || Hkv <= 0 || Nq < 0 || Nk < 0) return FA_ERR_INVALID_ARG;
+    if (Hq % Hkv != 0) return FA_ERR_INVALID_ARG;
+    if (causal != 0 && causal != 1) return FA_ERR_INVALID_ARG;
+    if (!std::isfinite(scale) || !(scale > 0.f)) return FA_ERR_INVALID_ARG;
+    if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED_HEAD_DIM;
+    const size_t q_bytes = size_t(B) * size_t(Nq) * size_t(Hq) * size_t(d) * 2;
+    const size_t kv_bytes = size_t(B) * size_t(Nk) * size_t(Hkv) * size_t(d) * 2;
+    const size_t lse_bytes = size_t(B) * size_t(Hq) * size_t(Nq) * 4;
+    if (q_bytes == 0 && kv_bytes == 0) return FA_OK;
+    if (q_bytes > 0 && (q == nullptr || out == nullptr || dout == nullptr || lse == nullptr || dq == nullptr))
+        return FA_ERR_INVALID_ARG;
+    if (kv_bytes > 0 && (k == nullptr || v == nullptr || dk == nullptr || dv == nullptr)) return FA_ERR_INVALID_ARG;
+    auto mis = [](const void *p, uintptr_t a) { return p != nullptr && (reinterpret_cast<uintptr_t>(p) % a) != 0; };
+    if (mis(q, 16) || mis(k, 16) || mis(v, 16) || mis(out, 16) || mis(dout, 16) || mis(dq, 16) || mis(dk, 16) ||
+        mis(dv, 16) || mis(lse, 4))
+        return FA_ERR_MISALIGNED;
+    // outputs must not overlap any input or each other
+    const void *ins[6] = {q, k, v, out, dout, lse};
+    const size_t in_bytes[6] = {q_bytes, kv_bytes, kv_bytes, q_bytes, q_bytes, lse_bytes};
+    void *outs[3] = {dq, dk, dv};
+    const size_t out_bytes[3] = {q_bytes, kv_bytes, kv_bytes};
+    for (int o = 0; o < 3; ++o) {
+        for (int i = 0; i < 6; ++i)
+            if (overlaps(outs[o], out_bytes[o], ins[i], in_bytes[i])) return FA_ERR_OVERLAP;
+        for (int o2 = o + 1; o2 < 3; ++o2)
+            if (overlaps(outs[o], out_bytes[o], outs[o2], out_bytes[o2])) return FA_ERR_OVERLAP;
+    }
+    const bool work = q_bytes > 0 && kv_bytes > 0;
+    const size_t ws_bytes = work ? bwd_bytes(B, Hq, Nq, d) : 0;
+    if (work) {
+        if (workspace == nullptr || workspace_bytes < ws_bytes) return FA_ERR_INVALID_ARG;
+        if (mis(workspace, 256)) return FA_ERR_MISALIGNED;
+        for (int i = 0; i < 6; ++i)
+            if (overlaps(workspace, ws_bytes, ins[i], in_bytes[i])) return FA_ERR_OVERLAP;
+        for (int o = 0; o < 3; ++o)
+            if (overlaps(workspace, ws_bytes, outs[o], out_bytes[o])) return FA_ERR_OVERLAP;
+    }
+
+    // ---- device checks
+    DeviceState *dev = nullptr;
+    int dev_id = -1;
+    int rc = current_device(&dev, &dev_id);
+    if (rc != FA_OK) return rc;
+    for (int i = 0; i < 6; ++i)
+        if (in_bytes[i] > 0 && (rc = check_device_range(ins[i], in_bytes[i], dev_id)) != FA_OK) return rc;
+    for (int o = 0; o < 3; ++o)
+        if (out_bytes[o] > 0 && (rc = check_device_range(outs[o], out_bytes[o], dev_id)) != FA_OK) return rc;
+    if (work && (rc = check_device_range(workspace, ws_bytes, dev_id)) != FA_OK) return rc;
+
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (!work) {   // no query rows or no keys: every gradient that exists is zero
+        for (int o = 0; o < 3; ++o) {
+            if (out_bytes[o] == 0) continue;
+            if (zero_fill(outs[o], out_bytes[o], nullptr, 0, dev->num_sms, st) != FA_OK) return FA_ERR_CUDA;
+        }
+        return FA_OK;
+    }
+    float *dq_acc = static_cast<float *>(workspace);
+    float *delta = reinterpret_cast<float *>(static_cast<char *>(workspace) + bwd_acc_bytes(B, Hq, Nq, d));
+    if (d == 64)
+        return launch_bwd<BwdCfg64>(q, k, v, out, dout, lse, dq, dk, dv, B, Hq, Hkv, Nq, Nk, scale, causal, dq_acc,
+                                    delta, *dev, kBwdSlot0, st);
+    return launch_bwd<BwdCfg128>(q, k, v, out, dout, lse, dq, dk, dv, B, Hq, Hkv, Nq, Nk, scale, causal, dq_acc, delta,
+                                 *dev, kBwdSlot0 + 1, st);
+}
+
+}  // extern "C"
+

@@ -13,44 +13,17 @@
 #include <cuda_runtime.h>
 
 #include "fa.h"
-#include "fa_bwd_kernel.cuh"
+#include "fa_host.h"
 #include "fa_kernel.cuh"
 
-namespace {
+// ------------------------------------------------------------------ host helpers (fa_host.h)
 
-using namespace fa;
+namespace fa_host {
 
-// Tiling per head dim: TileCfg<d, key rows per tile, query tiles per unit, K/V slots,
-// buffers per Q tile, S buffers per Q tile, P in TMEM columns of its own, exponential
-// pairs per 8 on the FMA pipe, fp16 elements (H) instead of bf16>.  d = 256 runs one 128-row query tile, so it has TMEM room
-// for a second S buffer (S_{j+1} computed while the softmax works on S_j); d <= 64 has
-// room to keep P apart from S, and is where the exponentials dominate.
-template <bool H> using Cfg32 = TileCfg<32, 128, 2, 8, 2, 1, true, 2, H>;
-template <bool H> using Cfg64 = TileCfg<64, 128, 2, 8, 2, 1, true, 2, H>;
-template <bool H> using Cfg80 = TileCfg<80, 128, 2, 4, 1, 1, false, 0, H>;
-template <bool H> using Cfg96 = TileCfg<96, 128, 2, 4, 1, 1, false, 0, H>;
-template <bool H> using Cfg128 = TileCfg<128, 128, 2, 4, 1, 1, false, 0, H>;
-template <bool H> using Cfg192 = TileCfg<192, 64, 2, 4, 1, 1, false, 0, H>;
-template <bool H> using Cfg256 = TileCfg<256, 64, 1, 4, 1, 2, false, 0, H>;
-// FP8 (E4M3) inputs, d = 128: 16 KB tiles, so eight K/V slots
-using Cfg128F8 = TileCfg<128, 128, 2, 8, 1, 1, false, 0, false, true>;
-constexpr int kNumCfgSlots = 19;   // forward: 7 head dims x 2 element types; backward: 2 head dims; FP8
-constexpr int kBwdSlot0 = 16;      // backward d = 64, 128 use slots 16, 17
-constexpr int kFp8Slot = 18;
+using fa::fa_no_keys_kernel;
 
 __device__ int g_fa_status;   // per-device kernel status word (0 = OK)
 
-constexpr int kMaxDevices = 64;
-constexpr int kMaxSplits = 256;
-
-struct DeviceState {
-    bool probed = false;
-    bool supported = false;
-    int num_sms = 0;
-    int *status_ptr = nullptr;
-    bool smem_attr_set[kNumCfgSlots] = {};
-    int regs_ok[kNumCfgSlots] = {};   // 0 unknown, 1 verified, -1 mismatch
-};
 DeviceState g_devices[kMaxDevices];
 std::mutex g_mutex;
 
@@ -60,7 +33,7 @@ using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_
                                    CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 using AddressRangeFn = CUresult (*)(CUdeviceptr *, size_t *, CUdeviceptr);
 
-void *driver_fn(const char *name) {
+static void *driver_fn(const char *name) {
     void *fn = nullptr;
     cudaDriverEntryPointQueryResult q{};
     if (cudaGetDriverEntryPoint(name, &fn, cudaEnableDefault, &q) != cudaSuccess ||
@@ -69,12 +42,12 @@ void *driver_fn(const char *name) {
     return fn;
 }
 
-EncodeTiledFn encode_fn() {
+static EncodeTiledFn encode_fn() {
     static EncodeTiledFn fn = reinterpret_cast<EncodeTiledFn>(driver_fn("cuTensorMapEncodeTiled"));
     return fn;
 }
 
-AddressRangeFn address_range_fn() {
+static AddressRangeFn address_range_fn() {
     static AddressRangeFn fn = reinterpret_cast<AddressRangeFn>(driver_fn("cuMemGetAddressRange"));
     return fn;
 }
@@ -144,8 +117,8 @@ bool overlaps(const void *a, size_t na, const void *b, size_t nb) {
 // 4-D view (d, H, N, B) of a [B, N, H, d] bf16 tensor, box (CW, heads, rows, 1): the box
 // lands in shared memory as heads*rows swizzled rows, row-major over (row, head).
 // elem: 0 bf16, 1 fp16, 2 E4M3 bytes.
-int encode_bnhd(CUtensorMap *m, const void *base, int d, int H, int N, int B, int cw, int rows, int heads = 1,
-                int elem = 0) {
+int encode_bnhd(CUtensorMap *m, const void *base, int d, int H, int N, int B, int cw, int rows, int heads,
+                int elem) {
     EncodeTiledFn fn = encode_fn();
     if (fn == nullptr) return FA_ERR_CUDA;
     const cuuint64_t dims[4] = {cuuint64_t(d), cuuint64_t(H), cuuint64_t(N), cuuint64_t(B)};
@@ -163,6 +136,34 @@ int encode_bnhd(CUtensorMap *m, const void *base, int d, int H, int N, int B, in
     return r == CUDA_SUCCESS ? FA_OK : FA_ERR_CUDA;
 }
 
+int zero_fill(void *dst, size_t bytes, float *lse, size_t n_lse, int num_sms, cudaStream_t st) {
+    const size_t n16 = bytes / 16;
+    const int grid = int(std::min<size_t>((std::max(n16, n_lse) + 255) / 256, size_t(num_sms) * 8));
+    fa_no_keys_kernel<<<grid > 0 ? grid : 1, 256, 0, st>>>(static_cast<uint4 *>(dst), n16, lse, n_lse);
+    return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+}  // namespace fa_host
+
+namespace {
+
+using namespace fa;
+using namespace fa_host;
+
+// Tiling per head dim: TileCfg<d, key rows per tile, query tiles per unit, K/V slots,
+// buffers per Q tile, S buffers per Q tile, P in TMEM columns of its own, exponential
+// pairs per 8 on the FMA pipe, fp16 elements (H) instead of bf16>.  d = 256 runs one 128-row query tile, so it has TMEM room
+// for a second S buffer (S_{j+1} computed while the softmax works on S_j); d <= 64 has
+// room to keep P apart from S, and is where the exponentials dominate.
+template <bool H> using Cfg32 = TileCfg<32, 128, 2, 8, 2, 1, true, 2, H>;
+template <bool H> using Cfg64 = TileCfg<64, 128, 2, 8, 2, 1, true, 2, H>;
+template <bool H> using Cfg80 = TileCfg<80, 128, 2, 4, 1, 1, false, 0, H>;
+template <bool H> using Cfg96 = TileCfg<96, 128, 2, 4, 1, 1, false, 0, H>;
+template <bool H> using Cfg128 = TileCfg<128, 128, 2, 4, 1, 1, false, 0, H>;
+template <bool H> using Cfg192 = TileCfg<192, 64, 2, 4, 1, 1, false, 0, H>;
+template <bool H> using Cfg256 = TileCfg<256, 64, 1, 4, 1, 2, false, 0, H>;
+// FP8 (E4M3) inputs, d = 128: 16 KB tiles, so eight K/V slots
+using Cfg128F8 = TileCfg<128, 128, 2, 8, 1, 1, false, 0, false, true>;
 struct Problem {
     const void *q, *k, *v;
     void *out;
@@ -175,6 +176,8 @@ struct Problem {
     float *o_part;      // workspace: fp32 partial O [split][B][Nq][Hq][d]
     float *lse_part;    // workspace: partial LSE [split][B][Hq][Nq]
     float o_scale;      // FP8: V dequantisation factor (1 otherwise)
+    int diag;           // causal diagonal offset (Nk - Nq unless a key shard)
+    int partial;        // write the shard partial (fp32 O, LSE) to o_part / lse_part
 };
 
 // Workspace layout of the split-KV forward: partial O, then (256-byte aligned) partial LSE.
@@ -251,11 +254,13 @@ int launch(const Problem &pr, DeviceState &dev, int cfg_slot, cudaStream_t strea
     p.num_units = int(units);
     p.scale_log2 = pr.scale * 1.4426950408889634f;
     p.o_scale = pr.o_scale;
+    p.diag = pr.diag;
+    p.partial = pr.partial;
 
     const int grid = int(units < dev.num_sms ? units : dev.num_sms);
     fa_fwd_kernel<C><<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(mq, mk, mv, p);
     if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
-    if (p.num_splits > 1) {
+    if (p.num_splits > 1 && !p.partial) {
         const long long rows = (long long)pr.B * pr.Nq * pr.Hq;
         const long long want = (rows + 7) / 8;   // 8 rows (warps) per 256-thread block
         const int mgrid = int(want < 8LL * dev.num_sms ? want : 8LL * dev.num_sms);
@@ -411,7 +416,7 @@ int forward(const void *q, const void *k, const void *v, void *out, float *lse, 
                                              ((splitkv_o_bytes(B, Hq, Nq, d, num_splits) + 255) & ~size_t(255)));
     }
     const Problem pr{q, k, v, out, lse, B, Hq, Hkv, Nq, Nk, d, scale, causal, window,
-                     ws_bytes > 0 ? num_splits : 1, o_part, lse_part, o_scale};
+                     ws_bytes > 0 ? num_splits : 1, o_part, lse_part, o_scale, Nk - Nq, 0};
     if (elem == 2) return launch<Cfg128F8>(pr, *dev, kFp8Slot, st);
     return elem == 1 ? dispatch<true>(pr, *dev, st) : dispatch<false>(pr, *dev, st);
 }
@@ -554,161 +559,105 @@ int fa_device_status(void *stream, int *detail) {
 
 }  // extern "C"
 
-// ------------------------------------------------------------------ backward
+// ------------------------------------------------------------------ key-sharded partials
 
 namespace {
 
-using BwdCfg64 = fa::bwd::BwdCfg<64>;
-using BwdCfg128 = fa::bwd::BwdCfg<128>;
-
-// Workspace of the backward: the fp32 dQ accumulator [B, Nq, Hq, d], then (256-byte
-// aligned) D = rowsum(dO * O) [B, Hq, Nq].
-size_t bwd_acc_bytes(int B, int Hq, int Nq, int d) {
-    return (size_t(B) * size_t(Nq) * size_t(Hq) * size_t(d) * 4 + 255) & ~size_t(255);
-}
-size_t bwd_bytes(int B, int Hq, int Nq, int d) {
-    return bwd_acc_bytes(B, Hq, Nq, d) + size_t(B) * size_t(Hq) * size_t(Nq) * 4;
-}
-
-template <class C>
-int launch_bwd(const void *q, const void *k, const void *v, const void *out, const void *dout, const float *lse,
-               void *dq, void *dk, void *dv, int B, int Hq, int Hkv, int Nq, int Nk, float scale, int causal,
-               float *dq_acc, float *delta, DeviceState &dev, int slot, cudaStream_t st) {
-    auto kern = fa::bwd::fa_bwd_kernel<C>;
-    if (!dev.smem_attr_set[slot]) {
-        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) != cudaSuccess) {
-            cudaGetLastError();
-            return FA_ERR_CUDA;
-        }
-        dev.smem_attr_set[slot] = true;
-    }
-    CUtensorMap mq, mk, mv, mdo;
-    int rc;
-    if ((rc = encode_bnhd(&mq, q, C::D, Hq, Nq, B, C::CW, fa::bwd::kRows)) != FA_OK) return rc;
-    if ((rc = encode_bnhd(&mdo, dout, C::D, Hq, Nq, B, C::CW, fa::bwd::kRows)) != FA_OK) return rc;
-    if ((rc = encode_bnhd(&mk, k, C::D, Hkv, Nk, B, C::CW, fa::bwd::kRows)) != FA_OK) return rc;
-    if ((rc = encode_bnhd(&mv, v, C::D, Hkv, Nk, B, C::CW, fa::bwd::kRows)) != FA_OK) return rc;
-
-    // D and the zeroed accumulator
+template <int D>
+void merge_launch(const float *o_parts, const float *lse_parts, int R, void *out, float *lse, int B, int Hq, int Nq,
+                  int num_sms, cudaStream_t st) {
     const long long rows = (long long)B * Nq * Hq;
     const long long want = (rows + 7) / 8;
-    const int pgrid = int(want < 8LL * dev.num_sms ? want : 8LL * dev.num_sms);
-    fa::bwd::fa_bwd_pre_kernel<C::D><<<pgrid > 0 ? pgrid : 1, 256, 0, st>>>(
-        static_cast<const uint16_t *>(out), static_cast<const uint16_t *>(dout), delta, dq_acc, B, Hq, Nq);
-    if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
-
-    fa::bwd::BwdParams p{};
-    p.lse = lse;
-    p.delta = delta;
-    p.dq_acc = dq_acc;
-    p.dk = static_cast<uint16_t *>(dk);
-    p.dv = static_cast<uint16_t *>(dv);
-    p.status = dev.status_ptr;
-    p.B = B;
-    p.Hq = Hq;
-    p.Hkv = Hkv;
-    p.Nq = Nq;
-    p.Nk = Nk;
-    p.n_rep = Hq / Hkv;
-    p.causal = causal;
-    p.nkt = (Nk + fa::bwd::kRows - 1) / fa::bwd::kRows;
-    p.nqt = (Nq + fa::bwd::kRows - 1) / fa::bwd::kRows;
-    const long long units = (long long)B * Hkv * p.nkt;
-    if (units > 0x7fffffffLL) return FA_ERR_INVALID_ARG;
-    p.num_units = int(units);
-    p.scale = scale;
-    p.scale_log2 = scale * 1.4426950408889634f;
-    const int grid = int(units < dev.num_sms ? units : dev.num_sms);
-    kern<<<grid, C::THREADS, C::SMEM_BYTES, st>>>(mq, mk, mv, mdo, p);
-    if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
-
-    const size_t n4 = size_t(rows) * C::D / 4;
-    const int qgrid = int(std::min<size_t>((n4 + 255) / 256, size_t(dev.num_sms) * 8));
-    fa::bwd::fa_bwd_post_kernel<<<qgrid > 0 ? qgrid : 1, 256, 0, st>>>(reinterpret_cast<const float4 *>(dq_acc),
-                                                                      static_cast<uint2 *>(dq), n4, scale);
-    return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+    const int grid = int(want < 8LL * num_sms ? want : 8LL * num_sms);
+    fa_splitkv_merge_kernel<D, false><<<grid > 0 ? grid : 1, 256, 0, st>>>(o_parts, lse_parts,
+                                                                          static_cast<uint16_t *>(out), lse, B, Hq, Nq, R);
 }
 
 }  // namespace
 
 extern "C" {
 
-size_t fa_bwd_workspace_bytes(int B, int Hq, int Nq, int d) {
-    if (B < 0 || Hq < 0 || Nq < 0 || d <= 0) return 0;
-    return bwd_bytes(B, Hq, Nq, d);
-}
-
-int fa_bwd(const void *q, const void *k, const void *v, const void *out, const void *dout, const float *lse,
-           void *dq, void *dk, void *dv, int B, int Hq, int Hkv, int Nq, int Nk, int d, float scale, int causal,
-           void *workspace, size_t workspace_bytes, void *stream) {
-    // ---- host-only validation
-    if (B < 0 || Hq <= 0 || Hkv <= 0 || Nq < 0 || Nk < 0) return FA_ERR_INVALID_ARG;
-    if (Hq % Hkv != 0) return FA_ERR_INVALID_ARG;
+int fa_fwd_partial(const void *q, const void *k, const void *v, float *o_part, float *lse_part, int B, int Hq,
+                   int Hkv, int Nq, int Nk, int d, float scale, int causal, int key_offset, int Nk_total,
+                   void *stream) {
+    if (B < 0 || Hq <= 0 || Hkv <= 0 || Nq < 0 || Nk < 0 || Hq % Hkv != 0) return FA_ERR_INVALID_ARG;
     if (causal != 0 && causal != 1) return FA_ERR_INVALID_ARG;
+    if (key_offset < 0 || Nk_total < 0 || (long long)key_offset + Nk > Nk_total) return FA_ERR_INVALID_ARG;
     if (!std::isfinite(scale) || !(scale > 0.f)) return FA_ERR_INVALID_ARG;
-    if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED_HEAD_DIM;
+    if (tile_config(d, nullptr, nullptr, nullptr, nullptr) != FA_OK) return FA_ERR_UNSUPPORTED_HEAD_DIM;
     const size_t q_bytes = size_t(B) * size_t(Nq) * size_t(Hq) * size_t(d) * 2;
     const size_t kv_bytes = size_t(B) * size_t(Nk) * size_t(Hkv) * size_t(d) * 2;
+    const size_t op_bytes = size_t(B) * size_t(Nq) * size_t(Hq) * size_t(d) * 4;
     const size_t lse_bytes = size_t(B) * size_t(Hq) * size_t(Nq) * 4;
-    if (q_bytes == 0 && kv_bytes == 0) return FA_OK;
-    if (q_bytes > 0 && (q == nullptr || out == nullptr || dout == nullptr || lse == nullptr || dq == nullptr))
-        return FA_ERR_INVALID_ARG;
-    if (kv_bytes > 0 && (k == nullptr || v == nullptr || dk == nullptr || dv == nullptr)) return FA_ERR_INVALID_ARG;
-    auto mis = [](const void *p, uintptr_t a) { return p != nullptr && (reinterpret_cast<uintptr_t>(p) % a) != 0; };
-    if (mis(q, 16) || mis(k, 16) || mis(v, 16) || mis(out, 16) || mis(dout, 16) || mis(dq, 16) || mis(dk, 16) ||
-        mis(dv, 16) || mis(lse, 4))
+    if (q_bytes == 0) return FA_OK;
+    if (q == nullptr || o_part == nullptr || lse_part == nullptr) return FA_ERR_INVALID_ARG;
+    if (kv_bytes > 0 && (k == nullptr || v == nullptr)) return FA_ERR_INVALID_ARG;
+    auto mis = [](const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) != 0; };
+    if (mis(q, 16) || mis(o_part, 16) || mis(lse_part, 4) || (kv_bytes > 0 && (mis(k, 16) || mis(v, 16))))
         return FA_ERR_MISALIGNED;
-    // outputs must not overlap any input or each other
-    const void *ins[6] = {q, k, v, out, dout, lse};
-    const size_t in_bytes[6] = {q_bytes, kv_bytes, kv_bytes, q_bytes, q_bytes, lse_bytes};
-    void *outs[3] = {dq, dk, dv};
-    const size_t out_bytes[3] = {q_bytes, kv_bytes, kv_bytes};
-    for (int o = 0; o < 3; ++o) {
-        for (int i = 0; i < 6; ++i)
-            if (overlaps(outs[o], out_bytes[o], ins[i], in_bytes[i])) return FA_ERR_OVERLAP;
-        for (int o2 = o + 1; o2 < 3; ++o2)
-            if (overlaps(outs[o], out_bytes[o], outs[o2], out_bytes[o2])) return FA_ERR_OVERLAP;
-    }
-    const bool work = q_bytes > 0 && kv_bytes > 0;
-    const size_t ws_bytes = work ? bwd_bytes(B, Hq, Nq, d) : 0;
-    if (work) {
-        if (workspace == nullptr || workspace_bytes < ws_bytes) return FA_ERR_INVALID_ARG;
-        if (mis(workspace, 256)) return FA_ERR_MISALIGNED;
-        for (int i = 0; i < 6; ++i)
-            if (overlaps(workspace, ws_bytes, ins[i], in_bytes[i])) return FA_ERR_OVERLAP;
-        for (int o = 0; o < 3; ++o)
-            if (overlaps(workspace, ws_bytes, outs[o], out_bytes[o])) return FA_ERR_OVERLAP;
-    }
-
-    // ---- device checks
+    if (overlaps(o_part, op_bytes, q, q_bytes) || overlaps(o_part, op_bytes, k, kv_bytes) ||
+        overlaps(o_part, op_bytes, v, kv_bytes) || overlaps(lse_part, lse_bytes, q, q_bytes) ||
+        overlaps(lse_part, lse_bytes, k, kv_bytes) || overlaps(lse_part, lse_bytes, v, kv_bytes) ||
+        overlaps(lse_part, lse_bytes, o_part, op_bytes))
+        return FA_ERR_OVERLAP;
     DeviceState *dev = nullptr;
     int dev_id = -1;
     int rc = current_device(&dev, &dev_id);
     if (rc != FA_OK) return rc;
-    for (int i = 0; i < 6; ++i)
-        if (in_bytes[i] > 0 && (rc = check_device_range(ins[i], in_bytes[i], dev_id)) != FA_OK) return rc;
-    for (int o = 0; o < 3; ++o)
-        if (out_bytes[o] > 0 && (rc = check_device_range(outs[o], out_bytes[o], dev_id)) != FA_OK) return rc;
-    if (work && (rc = check_device_range(workspace, ws_bytes, dev_id)) != FA_OK) return rc;
-
-    cudaStream_t st = static_cast<cudaStream_t>(stream);
-    if (!work) {   // no query rows or no keys: every gradient that exists is zero
-        for (int o = 0; o < 3; ++o) {
-            if (out_bytes[o] == 0) continue;
-            const size_t n16 = out_bytes[o] / 16;
-            const int grid = int(std::min<size_t>((n16 + 255) / 256, size_t(dev->num_sms) * 8));
-            fa_no_keys_kernel<<<grid > 0 ? grid : 1, 256, 0, st>>>(static_cast<uint4 *>(outs[o]), n16, nullptr, 0);
-            if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
-        }
-        return FA_OK;
+    if ((rc = check_device_range(q, q_bytes, dev_id)) != FA_OK) return rc;
+    if ((rc = check_device_range(o_part, op_bytes, dev_id)) != FA_OK) return rc;
+    if ((rc = check_device_range(lse_part, lse_bytes, dev_id)) != FA_OK) return rc;
+    if (kv_bytes > 0) {
+        if ((rc = check_device_range(k, kv_bytes, dev_id)) != FA_OK) return rc;
+        if ((rc = check_device_range(v, kv_bytes, dev_id)) != FA_OK) return rc;
     }
-    float *dq_acc = static_cast<float *>(workspace);
-    float *delta = reinterpret_cast<float *>(static_cast<char *>(workspace) + bwd_acc_bytes(B, Hq, Nq, d));
-    if (d == 64)
-        return launch_bwd<BwdCfg64>(q, k, v, out, dout, lse, dq, dk, dv, B, Hq, Hkv, Nq, Nk, scale, causal, dq_acc,
-                                    delta, *dev, kBwdSlot0, st);
-    return launch_bwd<BwdCfg128>(q, k, v, out, dout, lse, dq, dk, dv, B, Hq, Hkv, Nq, Nk, scale, causal, dq_acc, delta,
-                                 *dev, kBwdSlot0 + 1, st);
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (Nk == 0) {   // an empty shard: O = 0, LSE = -inf (weight 0 in the merge)
+        const size_t n16 = op_bytes / 16;
+        const int grid = int(std::min<size_t>((n16 + 255) / 256, size_t(dev->num_sms) * 8));
+        fa_no_keys_kernel<<<grid > 0 ? grid : 1, 256, 0, st>>>(reinterpret_cast<uint4 *>(o_part), n16, lse_part,
+                                                             size_t(B) * Hq * Nq);
+        return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+    }
+    const Problem pr{q, k, v, nullptr, nullptr, B, Hq, Hkv, Nq, Nk, d, scale, causal, 0,
+                     1, o_part, lse_part, 1.f, Nk_total - Nq - key_offset, 1};
+    return dispatch<false>(pr, *dev, st);
+}
+
+int fa_merge_partials(const float *o_parts, const float *lse_parts, int R, void *out, float *lse, int B, int Hq,
+                      int Nq, int d, void *stream) {
+    if (R < 1 || B < 0 || Hq <= 0 || Nq < 0) return FA_ERR_INVALID_ARG;
+    if (tile_config(d, nullptr, nullptr, nullptr, nullptr) != FA_OK) return FA_ERR_UNSUPPORTED_HEAD_DIM;
+    const size_t rows = size_t(B) * size_t(Nq) * size_t(Hq);
+    if (rows == 0) return FA_OK;
+    if (o_parts == nullptr || lse_parts == nullptr || out == nullptr) return FA_ERR_INVALID_ARG;
+    const size_t op_bytes = size_t(R) * rows * size_t(d) * 4, lp_bytes = size_t(R) * rows * 4;
+    const size_t out_bytes = rows * size_t(d) * 2, lse_bytes = rows * 4;
+    auto mis = [](const void *p, uintptr_t a) { return p != nullptr && (reinterpret_cast<uintptr_t>(p) % a) != 0; };
+    if (mis(o_parts, 4) || mis(lse_parts, 4) || mis(out, 2) || mis(lse, 4)) return FA_ERR_MISALIGNED;
+    if (overlaps(out, out_bytes, o_parts, op_bytes) || overlaps(out, out_bytes, lse_parts, lp_bytes) ||
+        overlaps(lse, lse_bytes, o_parts, op_bytes) || overlaps(lse, lse_bytes, lse_parts, lp_bytes) ||
+        overlaps(lse, lse_bytes, out, out_bytes))
+        return FA_ERR_OVERLAP;
+    DeviceState *dev = nullptr;
+    int dev_id = -1;
+    int rc = current_device(&dev, &dev_id);
+    if (rc != FA_OK) return rc;
+    if ((rc = check_device_range(o_parts, op_bytes, dev_id)) != FA_OK) return rc;
+    if ((rc = check_device_range(lse_parts, lp_bytes, dev_id)) != FA_OK) return rc;
+    if ((rc = check_device_range(out, out_bytes, dev_id)) != FA_OK) return rc;
+    if (lse && (rc = check_device_range(lse, lse_bytes, dev_id)) != FA_OK) return rc;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    switch (d) {
+        case 32: merge_launch<32>(o_parts, lse_parts, R, out, lse, B, Hq, Nq, dev->num_sms, st); break;
+        case 64: merge_launch<64>(o_parts, lse_parts, R, out, lse, B, Hq, Nq, dev->num_sms, st); break;
+        case 80: merge_launch<80>(o_parts, lse_parts, R, out, lse, B, Hq, Nq, dev->num_sms, st); break;
+        case 96: merge_launch<96>(o_parts, lse_parts, R, out, lse, B, Hq, Nq, dev->num_sms, st); break;
+        case 128: merge_launch<128>(o_parts, lse_parts, R, out, lse, B, Hq, Nq, dev->num_sms, st); break;
+        case 192: merge_launch<192>(o_parts, lse_parts, R, out, lse, B, Hq, Nq, dev->num_sms, st); break;
+        default: merge_launch<256>(o_parts, lse_parts, R, out, lse, B, Hq, Nq, dev->num_sms, st); break;
+    }
+    return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
 }  // extern "C"

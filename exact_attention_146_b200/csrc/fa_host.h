@@ -1,0 +1,44 @@
+// fa_host.h -- host-side helpers shared by the translation units of libfa.so (defined in
+// fa_fwd.cu): per-device state and probing, pointer checks, TMA tensor-map encoding and a
+// zero-fill launch.  Internal to the library; not part of the C ABI.
+#pragma once
+
+#include <cstddef>
+#include <mutex>
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+namespace fa_host {
+
+constexpr int kNumCfgSlots = 19;   // forward: 7 head dims x 2 element types; backward: 2 head dims; FP8
+constexpr int kBwdSlot0 = 16;      // backward d = 64, 128 use slots 16, 17
+constexpr int kFp8Slot = 18;
+
+constexpr int kMaxDevices = 64;
+constexpr int kMaxSplits = 256;
+
+struct DeviceState {
+    bool probed = false;
+    bool supported = false;
+    int num_sms = 0;
+    int *status_ptr = nullptr;
+    bool smem_attr_set[kNumCfgSlots] = {};
+    int regs_ok[kNumCfgSlots] = {};   // 0 unknown, 1 verified, -1 mismatch
+};
+
+extern std::mutex g_mutex;   // guards the per-device state and lazily found addresses
+
+// The current device's state, probed once (sm_100 or not, SM count, status word address).
+int current_device(DeviceState **out, int *dev_out);
+// `bytes` starting at `p` must be device (or managed) memory of device `dev`, inside one allocation.
+int check_device_range(const void *p, size_t bytes, int dev);
+bool overlaps(const void *a, size_t na, const void *b, size_t nb);
+// 4-D view (d, H, N, B) of a [B, N, H, d] tensor, box (cw, heads, rows, 1); elem: 0 bf16,
+// 1 fp16, 2 E4M3 bytes.
+int encode_bnhd(CUtensorMap *m, const void *base, int d, int H, int N, int B, int cw, int rows, int heads = 1,
+                int elem = 0);
+// Zero `bytes` (a multiple of 16) at dst and set n_lse floats at lse (if not NULL) to -inf.
+int zero_fill(void *dst, size_t bytes, float *lse, size_t n_lse, int num_sms, cudaStream_t st);
+
+}  // namespace fa_host

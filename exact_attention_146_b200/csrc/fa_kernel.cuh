@@ -65,6 +65,10 @@ struct FwdParams {
     float *lse_part;      // num_splits > 1: partial LSE [split][B][Hq][Nq]
     float scale_log2;     // scale * log2(e) (FP8: times the Q and K dequantisation factors)
     float o_scale;        // FP8: the V dequantisation factor, applied to O with 1 / l
+    int diag;             // causal / window: row i sees keys j <= i + diag (Nk - Nq; for a key
+                          // shard at offset o of Nk_total keys, Nk_total - Nq - o)
+    int partial;          // 1: write the fp32 normalised O and the LSE of these keys to
+                          // o_part / lse_part (a key shard's partial) instead of out / lse
 };
 
 // Compile-time tiling for one head dimension.
@@ -185,7 +189,7 @@ __device__ __forceinline__ UnitInfo decode_unit(int u, const FwdParams &p) {
     w.q0 = qb * (C::NQT * kBlockQ);
     const int flat_rows = p.Nq * p.pack;
     const int nkv = (p.Nk + C::BC - 1) / C::BC;
-    const int diag = p.Nk - p.Nq;    // row i sees keys up to i + diag (causal / window)
+    const int diag = p.diag;         // row i sees keys up to i + diag (causal / window)
     w.j_lo = 0x7fffffff;
     w.j_hi = 0;
 #pragma unroll
@@ -608,7 +612,7 @@ __device__ void softmax_role(const FwdParams &p, uint32_t sbase, uint32_t tmem, 
         const int f_row = f_lo + row_in_tile;
         const int row = f_row / p.pack;            // this thread's query i and head hq
         const int hq = w.hq + (f_row - row * p.pack);
-        const int diag = p.Nk - p.Nq;              // causal: key j visible to row i iff j <= i + diag
+        const int diag = p.diag;                   // causal: key j visible to row i iff j <= i + diag
         const int row_lim = p.causal ? row + diag : 0x7fffffff;
         // sliding window: keys j > i + diag - W; the tile's first row has the lowest bound
         const int row_lo = p.window > 0 ? row + diag - p.window + 1 : -0x7fffffff;
@@ -700,7 +704,7 @@ __device__ void softmax_role(const FwdParams &p, uint32_t sbase, uint32_t tmem, 
             if constexpr (C::FP8) inv_l *= p.o_scale;
             const bool store = row < p.Nq;
             const size_t row_off = (size_t(w.b) * p.Nq + size_t(row)) * p.Hq + hq;   // [b][row][hq]
-            const bool split_mode = p.num_splits > 1;
+            const bool split_mode = p.num_splits > 1 || p.partial;
             uint16_t *orow = static_cast<uint16_t *>(p.out) + row_off * C::D;
             float *prow = split_mode ? p.o_part + (size_t(w.split) * p.B * p.Nq * p.Hq + row_off) * C::D : nullptr;
 #pragma unroll
@@ -825,6 +829,8 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
 // Split-KV merge: one warp per output row (b, i, hq).  With m = max_s LSE_s, the weights
 // w_s = e^(LSE_s - m) combine the per-split normalised outputs O = sum_s w_s O_s / sum_s w_s,
 // and LSE = m + ln sum_s w_s; a row no split saw (all LSE_s = -inf) gets O = 0, LSE = -inf.
+// The lanes read 32 splits' LSEs at once and pass the weights around by shuffle, so the
+// loads of the partial rows do not wait on one another.
 template <int D, bool F16>
 __global__ void __launch_bounds__(256) fa_splitkv_merge_kernel(const float *o_part, const float *lse_part,
                                                                uint16_t *out, float *lse, int B, int Hq,
@@ -841,23 +847,36 @@ __global__ void __launch_bounds__(256) fa_splitkv_merge_kernel(const float *o_pa
         const int b = int(bi / Nq);
         const long lse_off = (long(b) * Hq + hq) * Nq + i;
         float m = -INFINITY;
-        for (int sp = 0; sp < num_splits; ++sp) m = fmaxf(m, lse_part[sp * split_stride_l + lse_off]);
+        for (int base = 0; base < num_splits; base += 32) {
+            const int sp = base + lane;
+            if (sp < num_splits) m = fmaxf(m, lse_part[sp * split_stride_l + lse_off]);
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
         float acc[PER_LANE];
 #pragma unroll
         for (int e = 0; e < PER_LANE; ++e) acc[e] = 0.f;
         float wsum = 0.f;
         if (m != -INFINITY) {
-            for (int sp = 0; sp < num_splits; ++sp) {
-                const float ls = lse_part[sp * split_stride_l + lse_off];
-                const float wgt = ls == -INFINITY ? 0.f : __expf(ls - m);
-                wsum += wgt;
-                const float *src = o_part + sp * split_stride_o + r * D;
+            for (int base = 0; base < num_splits; base += 32) {
+                const int sp = base + lane;
+                const float ls = sp < num_splits ? lse_part[sp * split_stride_l + lse_off] : -INFINITY;
+                const float wl = ls == -INFINITY ? 0.f : __expf(ls - m);
+                wsum += wl;
+                const int n = min(32, num_splits - base);
+#pragma unroll 4
+                for (int t = 0; t < n; ++t) {
+                    const float wgt = __shfl_sync(0xffffffffu, wl, t);
+                    const float *src = o_part + (base + t) * split_stride_o + r * D;
 #pragma unroll
-                for (int e = 0; e < PER_LANE; ++e) {
-                    const int col = lane + 32 * e;
-                    if (col < D) acc[e] = fmaf(wgt, src[col], acc[e]);
+                    for (int e = 0; e < PER_LANE; ++e) {
+                        const int col = lane + 32 * e;
+                        if (col < D) acc[e] = fmaf(wgt, src[col], acc[e]);
+                    }
                 }
             }
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) wsum += __shfl_xor_sync(0xffffffffu, wsum, o);
         }
         const float inv = wsum > 0.f ? 1.f / wsum : 0.f;
 #pragma unroll

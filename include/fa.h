@@ -214,6 +214,30 @@ int fa_bwd(const void *q, const void *k, const void *v, const void *out, const v
            void *dq, void *dk, void *dv, int B, int Hq, int Hkv, int Nq, int Nk, int d, float scale, int causal,
            void *workspace, size_t workspace_bytes, void *stream);
 
+/*
+ * Key-sharded attention, for one sequence too long for one GPU: each GPU holds a shard of
+ * K and V (keys key_offset .. key_offset + Nk - 1 of a sequence of Nk_total keys) and all of
+ * Q, computes the partial (O_r, LSE_r) of its shard, the partials are exchanged (one
+ * all-gather), and every GPU merges them with the log-sum-exp identity of the split-KV
+ * forward (LSE = ln sum_r exp(LSE_r), O = sum_r exp(LSE_r - LSE) O_r).  The pages promise
+ * sequence-dimension parallelism (the kaiwu.csdn.net FlashAttention page, FA-2 section);
+ * the exchange is the caller's (e.g. an NCCL all-gather of o_part and lse_part).
+ *
+ * fa_fwd_partial: q [B, Nq, Hq, d] bf16; k, v [B, Nk, Hkv, d] bf16 (the shard); o_part
+ *   [B, Nq, Hq, d] fp32 (16-byte aligned) and lse_part [B, Hq, Nq] fp32, written: O of this
+ *   shard's keys normalised by its own sum, and the natural-log LSE of those keys (rows that
+ *   see none of them: O = 0, LSE = -inf).  causal: key g (global index) is visible to query
+ *   i iff g <= i + Nk_total - Nq.  0 <= key_offset, key_offset + Nk <= Nk_total.  Other
+ *   arguments and errors as fa_fwd.
+ * fa_merge_partials: o_parts [R, B, Nq, Hq, d] fp32 and lse_parts [R, B, Hq, Nq] fp32 (R >= 1
+ *   partials, stacked) -> out [B, Nq, Hq, d] bf16 and lse [B, Hq, Nq] fp32 (NULL: skipped).
+ */
+int fa_fwd_partial(const void *q, const void *k, const void *v, float *o_part, float *lse_part,
+                   int B, int Hq, int Hkv, int Nq, int Nk, int d, float scale, int causal,
+                   int key_offset, int Nk_total, void *stream);
+int fa_merge_partials(const float *o_parts, const float *lse_parts, int R, void *out, float *lse,
+                      int B, int Hq, int Nq, int d, void *stream);
+
 /* Human-readable text of a status code (static storage; never NULL). */
 const char *fa_status_string(int status);
 
