@@ -394,7 +394,7 @@ def run_bwd_sweep(args):
     names = (args.sweep_only or BWD_DEFAULT).split(",")
     for name in names:
         w = synth.WORKLOADS[name]
-        if w.d not in (64, 128) or w.dtype != "bf16" or w.window or w.splitkv:
+        if w.d not in (32, 64, 80, 96, 128) or w.dtype != "bf16" or w.window or w.splitkv:
             continue
         x = synth.make_inputs(w)
         q, k, v = (torch.from_numpy(x[n].view(np.int16)).view(torch.bfloat16).cuda() for n in ("q", "k", "v"))

@@ -30,7 +30,7 @@ FA_ERR_SCRATCH_LIMIT = 9
 SPLITKV_STATIC_SCRATCH_BYTES = 16 * 1024 * 1024
 
 EXPORTED = ("fa_fwd", "fa_fwd_window", "fa_fwd_splitkv", "fa_splitkv_workspace_bytes", "fa_splitkv_default_splits",
-            "fa_fwd_splitkv_static", "fa_fwd_f16", "fa_fwd_fp8", "fa_fwd_partial", "fa_merge_partials", "fa_bwd", "fa_bwd_workspace_bytes", "fa_status_string", "fa_device_status", "fa_tile_config", "fa_version")
+            "fa_fwd_splitkv_static", "fa_fwd_f16", "fa_fwd_fp8", "fa_fwd_partial", "fa_merge_partials", "fa_bwd", "fa_bwd_f16", "fa_bwd_workspace_bytes", "fa_status_string", "fa_device_status", "fa_tile_config", "fa_version")
 
 
 class FaError(RuntimeError):
@@ -72,6 +72,8 @@ def lib() -> ctypes.CDLL:
         L.fa_splitkv_default_splits.restype = ci
         L.fa_bwd.argtypes = [vp] * 9 + [ci] * 6 + [cf, ci, vp, ctypes.c_size_t, vp]
         L.fa_bwd.restype = ci
+        L.fa_bwd_f16.argtypes = [vp] * 9 + [ci] * 6 + [cf, ci, vp, ctypes.c_size_t, vp]
+        L.fa_bwd_f16.restype = ci
         L.fa_bwd_workspace_bytes.argtypes = [ci, ci, ci, ci]
         L.fa_bwd_workspace_bytes.restype = ctypes.c_size_t
         L.fa_status_string.argtypes = [ci]
@@ -258,13 +260,16 @@ def bwd_workspace_bytes(B: int, Hq: int, Nq: int, d: int) -> int:
 
 def fa_bwd(q, k, v, out, dout, lse, *, causal: bool = False, scale: float | None = None, dq=None, dk=None,
            dv=None, workspace=None, stream=None):
-    """Exact attention backward (fa_bwd) on [B, N, H, d] bf16 CUDA tensors: returns
-    (dq, dk, dv) for the loss sum(out * dout), given the forward's out and lse [B, Hq, Nq]
-    fp32.  `workspace` (uint8, >= bwd_workspace_bytes) is allocated here if None."""
+    """Exact attention backward (fa_bwd, fa_bwd_f16 for fp16) on [B, N, H, d] CUDA tensors:
+    returns (dq, dk, dv) for the loss sum(out * dout), given the forward's out and lse
+    [B, Hq, Nq] fp32.  `workspace` (uint8, >= bwd_workspace_bytes) is allocated here if None."""
     import torch
+    dt = q.dtype
+    if dt not in (torch.bfloat16, torch.float16):
+        raise ValueError(f"q must be bf16 or fp16, got {dt}")
     for name, t in (("q", q), ("k", k), ("v", v), ("out", out), ("dout", dout)):
-        if t.dtype != torch.bfloat16 or not t.is_cuda or not t.is_contiguous() or t.dim() != 4:
-            raise ValueError(f"{name} must be a contiguous 4-D bf16 CUDA tensor, got {t.dtype} {tuple(t.shape)}")
+        if t.dtype != dt or not t.is_cuda or not t.is_contiguous() or t.dim() != 4:
+            raise ValueError(f"{name} must be a contiguous 4-D {dt} CUDA tensor, got {t.dtype} {tuple(t.shape)}")
     B, Nq, Hq, d = q.shape
     Nk, Hkv = k.shape[1], k.shape[2]
     if lse.dtype != torch.float32 or tuple(lse.shape) != (B, Hq, Nq) or not lse.is_contiguous():
@@ -276,7 +281,8 @@ def fa_bwd(q, k, v, out, dout, lse, *, causal: bool = False, scale: float | None
     dv = torch.empty_like(v) if dv is None else dv
     if workspace is None:
         workspace = torch.empty(max(1, bwd_workspace_bytes(B, Hq, Nq, d)), dtype=torch.uint8, device=q.device)
-    rc = lib().fa_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), dout.data_ptr(), lse.data_ptr(),
+    entry = lib().fa_bwd_f16 if dt == torch.float16 else lib().fa_bwd
+    rc = entry(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), dout.data_ptr(), lse.data_ptr(),
                       dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), B, Hq, Hkv, Nq, Nk, d, float(scale),
                       1 if causal else 0, workspace.data_ptr(), workspace.numel() * workspace.element_size(),
                       _stream_handle(stream))

@@ -18,8 +18,10 @@ namespace {
 
 using namespace fa_host;
 
-using BwdCfg64 = fa::bwd::BwdCfg<64>;
-using BwdCfg128 = fa::bwd::BwdCfg<128>;
+// The backward covers every forward head dim whose S^T, dP^T, dV and dK fit the 512 TMEM
+// columns (256 + 2 d <= 512): d in {32, 64, 80, 96, 128}.  Per device, whether the dynamic
+// shared-memory size of each bf16 / fp16 instantiation has been set.
+bool g_bwd_smem_set[kMaxDevices][10] = {};
 
 // Workspace of the backward: the fp32 dQ accumulator [B, Nq, Hq, d], then (256-byte
 // aligned) D = rowsum(dO * O) [B, Hq, Nq].
@@ -33,27 +35,31 @@ size_t bwd_bytes(int B, int Hq, int Nq, int d) {
 template <class C>
 int launch_bwd(const void *q, const void *k, const void *v, const void *out, const void *dout, const float *lse,
                void *dq, void *dk, void *dv, int B, int Hq, int Hkv, int Nq, int Nk, float scale, int causal,
-               float *dq_acc, float *delta, DeviceState &dev, int slot, cudaStream_t st) {
+               float *dq_acc, float *delta, DeviceState &dev, int dev_id, int slot, cudaStream_t st) {
     auto kern = fa::bwd::fa_bwd_kernel<C>;
-    if (!dev.smem_attr_set[slot]) {
-        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) != cudaSuccess) {
-            cudaGetLastError();
-            return FA_ERR_CUDA;
+    {
+        std::lock_guard<std::mutex> lock(g_mutex);
+        if (!g_bwd_smem_set[dev_id][slot]) {
+            if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) != cudaSuccess) {
+                cudaGetLastError();
+                return FA_ERR_CUDA;
+            }
+            g_bwd_smem_set[dev_id][slot] = true;
         }
-        dev.smem_attr_set[slot] = true;
     }
+    constexpr int elem = C::F16 ? 1 : 0;
     CUtensorMap mq, mk, mv, mdo;
     int rc;
-    if ((rc = encode_bnhd(&mq, q, C::D, Hq, Nq, B, C::CW, fa::bwd::kRows)) != FA_OK) return rc;
-    if ((rc = encode_bnhd(&mdo, dout, C::D, Hq, Nq, B, C::CW, fa::bwd::kRows)) != FA_OK) return rc;
-    if ((rc = encode_bnhd(&mk, k, C::D, Hkv, Nk, B, C::CW, fa::bwd::kRows)) != FA_OK) return rc;
-    if ((rc = encode_bnhd(&mv, v, C::D, Hkv, Nk, B, C::CW, fa::bwd::kRows)) != FA_OK) return rc;
+    if ((rc = encode_bnhd(&mq, q, C::D, Hq, Nq, B, C::CW, fa::bwd::kRows, 1, elem)) != FA_OK) return rc;
+    if ((rc = encode_bnhd(&mdo, dout, C::D, Hq, Nq, B, C::CW, fa::bwd::kRows, 1, elem)) != FA_OK) return rc;
+    if ((rc = encode_bnhd(&mk, k, C::D, Hkv, Nk, B, C::CW, fa::bwd::kRows, 1, elem)) != FA_OK) return rc;
+    if ((rc = encode_bnhd(&mv, v, C::D, Hkv, Nk, B, C::CW, fa::bwd::kRows, 1, elem)) != FA_OK) return rc;
 
     // D and the zeroed accumulator
     const long long rows = (long long)B * Nq * Hq;
     const long long want = (rows + 7) / 8;
     const int pgrid = int(want < 8LL * dev.num_sms ? want : 8LL * dev.num_sms);
-    fa::bwd::fa_bwd_pre_kernel<C::D><<<pgrid > 0 ? pgrid : 1, 256, 0, st>>>(
+    fa::bwd::fa_bwd_pre_kernel<C::D, C::F16><<<pgrid > 0 ? pgrid : 1, 256, 0, st>>>(
         static_cast<const uint16_t *>(out), static_cast<const uint16_t *>(dout), delta, dq_acc, B, Hq, Nq);
     if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
 
@@ -84,29 +90,40 @@ int launch_bwd(const void *q, const void *k, const void *v, const void *out, con
 
     const size_t n4 = size_t(rows) * C::D / 4;
     const int qgrid = int(std::min<size_t>((n4 + 255) / 256, size_t(dev.num_sms) * 8));
-    fa::bwd::fa_bwd_post_kernel<<<qgrid > 0 ? qgrid : 1, 256, 0, st>>>(reinterpret_cast<const float4 *>(dq_acc),
+    fa::bwd::fa_bwd_post_kernel<C::F16><<<qgrid > 0 ? qgrid : 1, 256, 0, st>>>(reinterpret_cast<const float4 *>(dq_acc),
                                                                       static_cast<uint2 *>(dq), n4, scale);
     return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
-}  // namespace
-
-extern "C" {
-
-size_t fa_bwd_workspace_bytes(int B, int Hq, int Nq, int d) {
-    if (B < 0 || Hq < 0 || Nq < 0 || d <= 0) return 0;
-    return bwd_bytes(B, Hq, Nq, d);
+template <bool H>
+int dispatch_bwd(int d, const void *q, const void *k, const void *v, const void *out, const void *dout,
+                 const float *lse, void *dq, void *dk, void *dv, int B, int Hq, int Hkv, int Nq, int Nk, float scale,
+                 int causal, float *dq_acc, float *delta, DeviceState &dev, int dev_id, cudaStream_t st) {
+    constexpr int base = H ? 5 : 0;
+#define FA_BWD_CASE(DIM, IDX)                                                                                      \
+    case DIM:                                                                                                      \
+        return launch_bwd<fa::bwd::BwdCfg<DIM, H>>(q, k, v, out, dout, lse, dq, dk, dv, B, Hq, Hkv, Nq, Nk, scale, \
+                                                   causal, dq_acc, delta, dev, dev_id, base + IDX, st);
+    switch (d) {
+        FA_BWD_CASE(32, 0)
+        FA_BWD_CASE(64, 1)
+        FA_BWD_CASE(80, 2)
+        FA_BWD_CASE(96, 3)
+        FA_BWD_CASE(128, 4)
+        default: return FA_ERR_UNSUPPORTED_HEAD_DIM;
+    }
+#undef FA_BWD_CASE
 }
 
-int fa_bwd(const void *q, const void *k, const void *v, const void *out, const void *dout, const float *lse,
-           void *dq, void *dk, void *dv, int B, int Hq, int Hkv, int Nq, int Nk, int d, float scale, int causal,
-           void *workspace, size_t workspace_bytes, void *stream) {
+int backward(const void *q, const void *k, const void *v, const void *out, const void *dout, const float *lse,
+             void *dq, void *dk, void *dv, int B, int Hq, int Hkv, int Nq, int Nk, int d, float scale, int causal,
+             void *workspace, size_t workspace_bytes, void *stream, bool f16) {
     // ---- host-only validation
     if (B < 0 || Hq <= 0 || Hkv <= 0 || Nq < 0 || Nk < 0) return FA_ERR_INVALID_ARG;
     if (Hq % Hkv != 0) return FA_ERR_INVALID_ARG;
     if (causal != 0 && causal != 1) return FA_ERR_INVALID_ARG;
     if (!std::isfinite(scale) || !(scale > 0.f)) return FA_ERR_INVALID_ARG;
-    if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED_HEAD_DIM;
+    if (d != 32 && d != 64 && d != 80 && d != 96 && d != 128) return FA_ERR_UNSUPPORTED_HEAD_DIM;
     const size_t q_bytes = size_t(B) * size_t(Nq) * size_t(Hq) * size_t(d) * 2;
     const size_t kv_bytes = size_t(B) * size_t(Nk) * size_t(Hkv) * size_t(d) * 2;
     const size_t lse_bytes = size_t(B) * size_t(Hq) * size_t(Nq) * 4;
@@ -161,11 +178,33 @@ int fa_bwd(const void *q, const void *k, const void *v, const void *out, const v
     }
     float *dq_acc = static_cast<float *>(workspace);
     float *delta = reinterpret_cast<float *>(static_cast<char *>(workspace) + bwd_acc_bytes(B, Hq, Nq, d));
-    if (d == 64)
-        return launch_bwd<BwdCfg64>(q, k, v, out, dout, lse, dq, dk, dv, B, Hq, Hkv, Nq, Nk, scale, causal, dq_acc,
-                                    delta, *dev, kBwdSlot0, st);
-    return launch_bwd<BwdCfg128>(q, k, v, out, dout, lse, dq, dk, dv, B, Hq, Hkv, Nq, Nk, scale, causal, dq_acc, delta,
-                                 *dev, kBwdSlot0 + 1, st);
+    return f16 ? dispatch_bwd<true>(d, q, k, v, out, dout, lse, dq, dk, dv, B, Hq, Hkv, Nq, Nk, scale, causal, dq_acc,
+                                    delta, *dev, dev_id, st)
+               : dispatch_bwd<false>(d, q, k, v, out, dout, lse, dq, dk, dv, B, Hq, Hkv, Nq, Nk, scale, causal,
+                                     dq_acc, delta, *dev, dev_id, st);
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t fa_bwd_workspace_bytes(int B, int Hq, int Nq, int d) {
+    if (B < 0 || Hq < 0 || Nq < 0 || d <= 0) return 0;
+    return bwd_bytes(B, Hq, Nq, d);
+}
+
+int fa_bwd(const void *q, const void *k, const void *v, const void *out, const void *dout, const float *lse,
+           void *dq, void *dk, void *dv, int B, int Hq, int Hkv, int Nq, int Nk, int d, float scale, int causal,
+           void *workspace, size_t workspace_bytes, void *stream) {
+    return backward(q, k, v, out, dout, lse, dq, dk, dv, B, Hq, Hkv, Nq, Nk, d, scale, causal, workspace,
+                    workspace_bytes, stream, false);
+}
+
+int fa_bwd_f16(const void *q, const void *k, const void *v, const void *out, const void *dout, const float *lse,
+               void *dq, void *dk, void *dv, int B, int Hq, int Hkv, int Nq, int Nk, int d, float scale, int causal,
+               void *workspace, size_t workspace_bytes, void *stream) {
+    return backward(q, k, v, out, dout, lse, dq, dk, dv, B, Hq, Hkv, Nq, Nk, d, scale, causal, workspace,
+                    workspace_bytes, stream, true);
 }
 
 }  // extern "C"

@@ -35,6 +35,7 @@
 
 #include <cuda.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 
 #include "sm100.cuh"
 
@@ -61,21 +62,27 @@ struct BwdParams {
     float scale, scale_log2;
 };
 
-template <int D_>
+template <int D_, bool F16_ = false>
 struct BwdCfg {
     static constexpr int D = D_;
-    static constexpr int CW = 64;                     // bf16 elements per 128-byte swizzled row
-    static constexpr int RB = 128;
-    static constexpr int NCH = D / CW;                // 64-column chunks of a [128 x D] tile
-    static constexpr int CHUNK = kRows * RB;          // 16 KB: one chunk of a 128-row tile
-    static constexpr int TILE = NCH * CHUNK;          // [128 x D] bf16
+    static constexpr bool F16 = F16_;                 // fp16 Q, K, V, O, dO and gradients, else bf16
+    static constexpr int CW = (D == 32) ? 32 : 64;    // elements per swizzled row of a Q/K/V/dO tile
+    static constexpr int RB = CW * 2;                 // bytes per swizzled row (64 or 128)
+    static constexpr uint32_t LAYOUT = (RB == 128) ? 2u : 4u;   // UMMA 128-byte / 64-byte swizzle
+    static constexpr int SBO = 8 * RB;                // 8-row swizzle atom
+    static constexpr int NCH = (D + CW - 1) / CW;     // column chunks of a [128 x D] tile (the last
+                                                      // one zero-filled past d for d = 80, 96)
+    static constexpr int CHUNK = kRows * RB;          // one chunk of a 128-row tile
+    static constexpr int TILE = NCH * CHUNK;          // [128 x D] tile
+    static constexpr int DS_RB = 128, DS_CHUNK = kRows * DS_RB;  // dS^T: 128 queries, 128-byte swizzle
+    static constexpr int DCH = (D + 31) / 32;         // 32-column TMEM chunks of a D-wide row
     static constexpr int NQS = 2;                     // Q / dO slots
     static constexpr int SMEM_K = 0;
     static constexpr int SMEM_V = TILE;
     static constexpr int SMEM_Q = 2 * TILE;
     static constexpr int SMEM_DO = SMEM_Q + NQS * TILE;
     static constexpr int SMEM_DS = SMEM_DO + NQS * TILE;     // dS^T: two 64-query chunks
-    static constexpr int SMEM_VEC = SMEM_DS + 2 * CHUNK;     // (L log2e, D) x 128 floats
+    static constexpr int SMEM_VEC = SMEM_DS + 2 * DS_CHUNK;  // (L log2e, D) x 128 floats
     static constexpr int SMEM_BAR = SMEM_VEC + 2 * kRows * 4;
     // barriers
     static constexpr int B_KV_FULL = 0, B_KV_EMPTY = 1, B_Q_FULL = 2, B_Q_EMPTY = B_Q_FULL + NQS,
@@ -89,17 +96,18 @@ struct BwdCfg {
     static constexpr int SMEM_NEEDED = SMEM_MISC + 16 + 1024;
     static constexpr int SMEM_BYTES = SMEM_NEEDED > 120 * 1024 ? SMEM_NEEDED : 120 * 1024;
     // TMEM columns
-    static constexpr int COL_A = 0, COL_B = 128, COL_DV = 256, COL_DK = 256 + D;
+    static constexpr int COL_A = 0, COL_B = 128, COL_DV = 256, COL_DK = 256 + DCH * 32;
     static constexpr int TMEM_COLS = 512;
     // warps: 0 TMA, 1 MMA, 2-3 idle, 4-7 SG, 8-11 DW
     static constexpr int THREADS = 384;
     static constexpr int SG_WARP0 = 4, DW_WARP0 = 8;
-    static constexpr uint32_t IDESC_SS = sm100::idesc_f16kind_f32(kRows, kRows, 0, 0, false);
-    static constexpr uint32_t IDESC_TS = sm100::idesc_f16kind_f32(kRows, D, 0, 1, false);
-    static constexpr uint32_t IDESC_DQ = sm100::idesc_f16kind_f32(kRows, D, 1, 1, false);
+    static constexpr uint32_t IDESC_SS = sm100::idesc_f16kind_f32(kRows, kRows, 0, 0, F16);
+    static constexpr uint32_t IDESC_TS = sm100::idesc_f16kind_f32(kRows, D, 0, 1, F16);
+    static constexpr uint32_t IDESC_DQ = sm100::idesc_f16kind_f32(kRows, D, 1, 1, F16);
 
-    static_assert(D == 64 || D == 128, "backward head dims");
-    static_assert(COL_DK + D <= TMEM_COLS, "TMEM budget");
+    static_assert(D % 16 == 0 && D >= 32 && D <= 128, "backward head dims: MMA N granularity, TMEM budget");
+    static_assert(COL_DK + DCH * 32 <= TMEM_COLS, "TMEM budget");
+    static_assert(SMEM_DS % 1024 == 0, "dS^T needs 1024-byte alignment (128-byte swizzle atoms)");
     static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 };
 
@@ -236,11 +244,11 @@ template <class C>
 __device__ void mma_issuer(const BwdParams &p, uint32_t sbase, uint32_t tmem, const Ctl &ctl) {
     auto bar = [&](int i) { return sbase + C::SMEM_BAR + 8u * uint32_t(i); };
     // K-major descriptors (reduction over d): 16 elements = 32 bytes per k-slice inside a
-    // 64-column chunk, chunks C::CHUNK bytes apart.
-    auto kmaj = [&](uint32_t addr) { return sm100::opaque(sm100::smem_desc(addr, 16, 1024, 2)); };
-    // M/N-major descriptors (reduction over the 128 rows): 16 rows = 2048 bytes per k-slice,
-    // the 64-column chunks C::CHUNK bytes apart (leading byte offset).
-    auto mnmaj = [&](uint32_t addr) { return sm100::opaque(sm100::smem_desc(addr, C::CHUNK, 1024, 2)); };
+    // C::CW-column chunk, chunks C::CHUNK bytes apart.
+    auto kmaj = [&](uint32_t addr) { return sm100::opaque(sm100::smem_desc(addr, 16, C::SBO, C::LAYOUT)); };
+    // M/N-major descriptors (reduction over the 128 rows): 16 rows = 16 * C::RB bytes per
+    // k-slice, the column chunks C::CHUNK bytes apart (leading byte offset).
+    auto mnmaj = [&](uint32_t addr) { return sm100::opaque(sm100::smem_desc(addr, C::CHUNK, C::SBO, C::LAYOUT)); };
     uint32_t n_step = 0, n_unit = 0;
     bool ok = true;
     for (int u = blockIdx.x; ok && u < p.num_units; u += gridDim.x) {
@@ -249,7 +257,7 @@ __device__ void mma_issuer(const BwdParams &p, uint32_t sbase, uint32_t tmem, co
         if (!warp_wait(bar(C::B_KV_FULL), n_unit & 1u, ctl, kSiteKvFull)) { ok = false; break; }
         const uint64_t k_km = kmaj(sbase + C::SMEM_K), v_km = kmaj(sbase + C::SMEM_V);
         const uint64_t k_mn = mnmaj(sbase + C::SMEM_K);
-        const uint64_t ds_mn = mnmaj(sbase + C::SMEM_DS);
+        const uint64_t ds_mn = sm100::opaque(sm100::smem_desc(sbase + C::SMEM_DS, C::DS_CHUNK, 1024, 2));
         for (int s = 0; s < w.nsteps; ++s, ++n_step) {
             const int slot = int(n_step % C::NQS);
             if (!warp_wait(bar(C::B_Q_FULL + slot), (n_step / C::NQS) & 1u, ctl, kSiteQFull)) { ok = false; break; }
@@ -288,8 +296,8 @@ __device__ void mma_issuer(const BwdParams &p, uint32_t sbase, uint32_t tmem, co
             sm100::tc_fence_after_sync();
 #pragma unroll
             for (int kk = 0; kk < kRows / 16; ++kk) {   // dQ = dS K
-                const uint32_t off = uint32_t(kk * 16 * C::RB) >> 4;
-                sm100::mma_bf16_ss_elected(tmem + C::COL_A, ds_mn + off, k_mn + off, C::IDESC_DQ, kk > 0 ? 1u : 0u);
+                const uint32_t a_off = uint32_t(kk * 16 * C::DS_RB) >> 4, b_off = uint32_t(kk * 16 * C::RB) >> 4;
+                sm100::mma_bf16_ss_elected(tmem + C::COL_A, ds_mn + a_off, k_mn + b_off, C::IDESC_DQ, kk > 0 ? 1u : 0u);
             }
             sm100::tc_commit_elected(bar(C::B_DQ_FULL));
         }
@@ -346,7 +354,7 @@ __device__ void sg_role(const BwdParams &p, uint32_t sbase, uint8_t *smem, uint3
                 const int q_lim = p.Nq - i0;                         // local query bound
                 const int key_lo_q = p.causal ? key - diag - i0 : -0x7fffffff;   // first local q seeing key
                 const bool key_ok = key < p.Nk;
-                uint8_t *ds_row = smem + C::SMEM_DS + r * C::RB;
+                uint8_t *ds_row = smem + C::SMEM_DS + r * C::DS_RB;
 #pragma unroll 1
                 for (int c = 0; c < kRows / 32; ++c) {
                     uint32_t sv[32], dp[32];
@@ -365,14 +373,14 @@ __device__ void sg_role(const BwdParams &p, uint32_t sbase, uint8_t *smem, uint3
                             pr[h] = pv;
                             dsr[h] = pv * (__uint_as_float(dp[e + h]) - dvv[ql]);
                         }
-                        pk[e / 2] = sm100::pack_bf16x2(pr[0], pr[1]);
-                        dk[e / 2] = sm100::pack_bf16x2(dsr[0], dsr[1]);
+                        pk[e / 2] = sm100::pack_x2<C::F16>(pr[0], pr[1]);
+                        dk[e / 2] = sm100::pack_x2<C::F16>(dsr[0], dsr[1]);
                     }
                     tmem_st16(tmem + lane_off + uint32_t(C::COL_A + 16 * c), pk);
                     tmem_st16(tmem + lane_off + uint32_t(C::COL_B + 16 * c), dk);
                     // dS^T row r, queries 32c .. 32c+31: chunk c/2, 16-byte units (c%2)*4 .. +3,
                     // 128-byte swizzle (unit index XOR row % 8)
-                    uint8_t *chunk_row = ds_row + (c / 2) * C::CHUNK;
+                    uint8_t *chunk_row = ds_row + (c / 2) * C::DS_CHUNK;
 #pragma unroll
                     for (int v4 = 0; v4 < 4; ++v4) {
                         const int unit = ((c % 2) * 4 + v4) ^ (r & 7);
@@ -420,9 +428,9 @@ __device__ void dw_role(const BwdParams &p, uint32_t sbase, uint32_t tmem, const
             float *dst = p.dq_acc + ((size_t(w.b) * p.Nq + size_t(q)) * p.Hq + hq) * C::D;
             // the whole dQ row into registers first, so region A is free for the next
             // step's S^T while the reductions run
-            uint32_t v[C::D];
+            uint32_t v[C::DCH * 32];
 #pragma unroll
-            for (int c = 0; c < C::D / 32; ++c)
+            for (int c = 0; c < C::DCH; ++c)
                 sm100::tmem_ld32_sync(tmem + lane_off + uint32_t(C::COL_A + 32 * c),
                                       *reinterpret_cast<uint32_t(*)[32]>(v + 32 * c));
             sm100::tc_fence_before_sync();
@@ -438,7 +446,7 @@ __device__ void dw_role(const BwdParams &p, uint32_t sbase, uint32_t tmem, const
         if (!warp_wait(bar(C::B_ACC_FULL), n_unit & 1u, ctl, kSiteAccFull)) return;
         sm100::tc_fence_after_sync();
 #pragma unroll 1
-        for (int c = 0; c < C::D / 32; ++c) {
+        for (int c = 0; c < C::DCH; ++c) {
             uint32_t dv[32], dk[32];
             sm100::tmem_ld32_sync(tmem + lane_off + uint32_t(C::COL_DV + 32 * c), dv);
             sm100::tmem_ld32_sync(tmem + lane_off + uint32_t(C::COL_DK + 32 * c), dk);
@@ -446,11 +454,13 @@ __device__ void dw_role(const BwdParams &p, uint32_t sbase, uint32_t tmem, const
                 uint32_t pv[16], pk[16];
 #pragma unroll
                 for (int i = 0; i < 16; ++i) {
-                    pv[i] = sm100::pack_bf16x2(__uint_as_float(dv[2 * i]), __uint_as_float(dv[2 * i + 1]));
-                    pk[i] = sm100::pack_bf16x2(__uint_as_float(dk[2 * i]) * p.scale, __uint_as_float(dk[2 * i + 1]) * p.scale);
+                    pv[i] = sm100::pack_x2<C::F16>(__uint_as_float(dv[2 * i]), __uint_as_float(dv[2 * i + 1]));
+                    pk[i] = sm100::pack_x2<C::F16>(__uint_as_float(dk[2 * i]) * p.scale,
+                                                   __uint_as_float(dk[2 * i + 1]) * p.scale);
                 }
 #pragma unroll
                 for (int v4 = 0; v4 < 4; ++v4) {
+                    if (32 * c + 8 * v4 >= C::D) break;   // d = 80, 96: the last chunk is partial
                     *reinterpret_cast<uint4 *>(p.dv + kv_row * C::D + 32 * c + 8 * v4) =
                         make_uint4(pv[4 * v4], pv[4 * v4 + 1], pv[4 * v4 + 2], pv[4 * v4 + 3]);
                     *reinterpret_cast<uint4 *>(p.dk + kv_row * C::D + 32 * c + 8 * v4) =
@@ -527,7 +537,13 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
 }
 
 // D_i = dO_i . O_i in fp32 (one warp per row) and a zeroed dQ accumulator.
-template <int D>
+template <bool F16>
+__device__ __forceinline__ float elem_to_f32(uint16_t bits) {
+    if constexpr (F16) return __half2float(__ushort_as_half(bits));
+    else return __uint_as_float(uint32_t(bits) << 16);
+}
+
+template <int D, bool F16>
 __global__ void __launch_bounds__(256) fa_bwd_pre_kernel(const uint16_t *out, const uint16_t *dout, float *delta,
                                                          float *dq_acc, int B, int Hq, int Nq) {
     const long rows = long(B) * Nq * Hq;
@@ -536,8 +552,8 @@ __global__ void __launch_bounds__(256) fa_bwd_pre_kernel(const uint16_t *out, co
          r += long(gridDim.x) * blockDim.x / 32) {
         float acc = 0.f;
         for (int c = lane; c < D; c += 32) {
-            const float o = __uint_as_float(uint32_t(out[r * D + c]) << 16);
-            const float g = __uint_as_float(uint32_t(dout[r * D + c]) << 16);
+            const float o = elem_to_f32<F16>(out[r * D + c]);
+            const float g = elem_to_f32<F16>(dout[r * D + c]);
             acc = fmaf(o, g, acc);
             dq_acc[r * D + c] = 0.f;
         }
@@ -553,12 +569,13 @@ __global__ void __launch_bounds__(256) fa_bwd_pre_kernel(const uint16_t *out, co
     }
 }
 
-// dQ = bf16(scale * acc)
+// dQ = bf16 (fp16) of scale * acc
+template <bool F16>
 __global__ void fa_bwd_post_kernel(const float4 *acc, uint2 *dq, size_t n4, float scale) {
     const size_t stride = size_t(gridDim.x) * blockDim.x;
     for (size_t i = size_t(blockIdx.x) * blockDim.x + threadIdx.x; i < n4; i += stride) {
         const float4 a = acc[i];
-        dq[i] = make_uint2(sm100::pack_bf16x2(a.x * scale, a.y * scale), sm100::pack_bf16x2(a.z * scale, a.w * scale));
+        dq[i] = make_uint2(sm100::pack_x2<F16>(a.x * scale, a.y * scale), sm100::pack_x2<F16>(a.z * scale, a.w * scale));
     }
 }
 

@@ -197,8 +197,8 @@ int fa_fwd_splitkv_static(const void *q, const void *k, const void *v, void *out
  *   k, v         [B, Nk, Hkv, d] bf16, read only
  *   lse          [B, Hq, Nq] fp32 (natural log), read only
  *   dq           [B, Nq, Hq, d] bf16, written;  dk, dv [B, Nk, Hkv, d] bf16, written
- *   d in {64, 128} (FA_ERR_UNSUPPORTED_HEAD_DIM otherwise); causal in {0, 1}; the other
- *   sizes and the scale as fa_fwd
+ *   d in {32, 64, 80, 96, 128} (FA_ERR_UNSUPPORTED_HEAD_DIM otherwise: S^T, dP^T, dV and dK
+ *   share the 512 TMEM columns); causal in {0, 1}; the other sizes and the scale as fa_fwd
  *   workspace    caller-owned device scratch of at least fa_bwd_workspace_bytes bytes,
  *                256-byte aligned (fp32 dQ accumulator and D); no initial contents are
  *                needed (the call zeroes what it accumulates into); contents undefined
@@ -213,6 +213,10 @@ size_t fa_bwd_workspace_bytes(int B, int Hq, int Nq, int d);
 int fa_bwd(const void *q, const void *k, const void *v, const void *out, const void *dout, const float *lse,
            void *dq, void *dk, void *dv, int B, int Hq, int Hkv, int Nq, int Nk, int d, float scale, int causal,
            void *workspace, size_t workspace_bytes, void *stream);
+/* fa_bwd_f16: the same with fp16 q, k, v, out, dout, dq, dk, dv (P and dS rounded to fp16). */
+int fa_bwd_f16(const void *q, const void *k, const void *v, const void *out, const void *dout, const float *lse,
+               void *dq, void *dk, void *dv, int B, int Hq, int Hkv, int Nq, int Nk, int d, float scale, int causal,
+               void *workspace, size_t workspace_bytes, void *stream);
 
 /*
  * Key-sharded attention, for one sequence too long for one GPU: each GPU holds a shard of

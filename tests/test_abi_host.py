@@ -149,7 +149,7 @@ def _bwd(L, d=128, ws=FAKE + (12 << 30), ws_bytes=1 << 30, dq=FAKE + (5 << 30), 
 
 def test_bwd_validation(L):
     assert fa.bwd_workspace_bytes(2, 4, 100, 128) == ((2 * 100 * 4 * 128 * 4 + 255) // 256) * 256 + 2 * 4 * 100 * 4
-    assert _bwd(L, d=96) == fa.FA_ERR_UNSUPPORTED_HEAD_DIM
+    assert _bwd(L, d=192) == fa.FA_ERR_UNSUPPORTED_HEAD_DIM and _bwd(L, d=48) == fa.FA_ERR_UNSUPPORTED_HEAD_DIM
     assert _bwd(L, causal=2) == fa.FA_ERR_INVALID_ARG
     assert _bwd(L, lse=None) == fa.FA_ERR_INVALID_ARG
     assert _bwd(L, ws=None) == fa.FA_ERR_INVALID_ARG

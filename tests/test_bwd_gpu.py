@@ -41,12 +41,12 @@ def inputs(B, Hq, Hkv, Nq, Nk, d, seed, **kw):
     return synth.make_inputs(w), synth.make_grad_output(w)
 
 
-def run_bwd(x, do_bits, scale, causal):
-    """Forward (for O and LSE) then fa_bwd, both through the C ABI."""
+def run_bwd(x, do_bits, scale, causal, dtype="bf16"):
+    """Forward (for O and LSE) then fa_bwd (fa_bwd_f16), both through the C ABI."""
     import torch
     import exact_attention_146_b200 as fa
-    q, k, v = (_parity.to_device(x[n], torch) for n in ("q", "k", "v"))
-    do = _parity.to_device(do_bits, torch)
+    q, k, v = (_parity.to_device(x[n], torch, dtype) for n in ("q", "k", "v"))
+    do = _parity.to_device(do_bits, torch, dtype)
     out, lse = fa.fa_fwd(q, k, v, causal=causal, scale=scale)
     dq = torch.full_like(q, float("nan"))
     dk = torch.full_like(k, float("nan"))
@@ -77,7 +77,7 @@ def compare_grads(got, ref, what):
         assert mx <= TOL_BWD_MAX_REL * max(ref_max, 1e-6), f"{what} {name}: max|d| {mx:.3e} (ref max {ref_max:.3e})"
 
 
-@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("d", [32, 64, 80, 96, 128])
 @pytest.mark.parametrize("Nq,Nk", [(1, 1), (17, 17), (128, 128), (129, 300), (300, 129), (256, 256)])
 @pytest.mark.parametrize("causal", [False, True])
 def test_bwd_small(orc, d, Nq, Nk, causal):
@@ -107,6 +107,17 @@ def test_bwd_medium(orc, causal):
     got = run_bwd(x, do, scale, causal)
     ref = orc.backward(x["q"], x["k"], x["v"], do, scale, causal)
     compare_grads(got, ref, f"medium causal={causal}")
+
+
+@pytest.mark.parametrize("d", [32, 80, 128])
+@pytest.mark.parametrize("causal", [False, True])
+def test_bwd_f16(orc, d, causal):
+    """fp16 inputs and gradients (fa_bwd_f16) against the oracle reading the same half bits."""
+    x, do = inputs(2, 4, 2, 200, 333, d, seed=d + 17, dtype="f16")
+    scale = 1.0 / math.sqrt(d)
+    got = run_bwd(x, do, scale, causal, dtype="f16")
+    ref = orc.backward(x["q"], x["k"], x["v"], do, scale, causal, dtype="f16")
+    compare_grads(got, ref, f"f16 d={d} causal={causal}")
 
 
 def test_bwd_empty_sides():
