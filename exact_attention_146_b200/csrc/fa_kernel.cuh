@@ -90,6 +90,15 @@ struct TileCfg {
     static constexpr int CW = RB / ES;                    // elements per swizzled smem row
     static constexpr int KSTEP = 32 / ES;                 // K elements per MMA (32 bytes)
     static constexpr int PCOLS = BC * ES / 4;             // TMEM columns of one row of P
+#ifndef FA_NO_PSPLIT
+    // P is handed to the P V MMAs in two 64-key halves: the first half of P V runs while
+    // the softmax computes the second half of P.  Worth it where the exponentials dominate
+    // (d <= 80: 6-10 % faster); at d >= 96 the extra register pressure costs more than the
+    // overlap gains, so the hand-off stays whole there.
+    static constexpr bool PSPLIT = (BC == 128) && !FP8 && D <= 80;
+#else
+    static constexpr bool PSPLIT = false;
+#endif
     static constexpr int NCH = (D + CW - 1) / CW;         // column chunks of a tile
     static constexpr int Q_CHUNK = kBlockQ * RB;
     static constexpr int KV_CHUNK = BC * RB;
@@ -108,7 +117,7 @@ struct TileCfg {
     static constexpr int SMEM_Q = 0;
     static constexpr int SMEM_KV = NQT * NQB * Q_TILE;
     static constexpr int SMEM_BAR = SMEM_KV + NS * KV_TILE;
-    static constexpr int NUM_BARS = 2 * NS + 2 * NQT * NQB + 3 * NQT * SB + 3 * NQT + 1;
+    static constexpr int NUM_BARS = 2 * NS + 2 * NQT * NQB + 4 * NQT * SB + 3 * NQT + 1;
     static constexpr int SMEM_MISC = SMEM_BAR + NUM_BARS * 8;
     // Each CTA holds all 512 TMEM columns, so ask for enough shared memory that a
     // second CTA can never be resident on the same SM (it would only wait in alloc).
@@ -150,7 +159,8 @@ struct TileCfg {
     static constexpr int B_FULL = 0, B_EMPTY = NS, B_QFULL = 2 * NS, B_QEMPTY = 2 * NS + NQT * NQB,
                          B_SFULL = 2 * NS + 2 * NQT * NQB,   // S_t in buffer b computed
                          B_PFULL = B_SFULL + NQT * SB,       // P_t written over buffer b
-                         B_PVDONE = B_PFULL + NQT * SB,      // the P V MMA reading buffer b done
+                         B_PHALF = B_PFULL + NQT * SB,       // its first 64 keys written (PSPLIT)
+                         B_PVDONE = B_PHALF + NQT * SB,      // the P V MMA reading buffer b done
                          B_ODONE = B_PVDONE + NQT * SB,      // a P V MMA of tile t done (rescale)
                          B_OFINAL = B_ODONE + NQT,           // the last P V of tile t in a unit done
                          B_OEMPTY = B_OFINAL + NQT,          // epilogue finished reading O_t
@@ -357,7 +367,7 @@ __device__ __forceinline__ void issue_qk(uint32_t sbase, uint32_t tmem, int t, i
     }
 }
 
-template <class C>
+template <class C, int KK_BEGIN = 0, int KK_END = C::BC / C::KSTEP>
 __device__ __forceinline__ void issue_pv(uint32_t sbase, uint32_t tmem, int t, int slot, int sbuf, bool accumulate) {
     // V tile is [BC rows x d] row-major: MN-major B operand; 16 key rows per MMA,
     // 64-element column chunks C::KV_CHUNK bytes apart (leading byte offset).  P is the
@@ -367,7 +377,7 @@ __device__ __forceinline__ void issue_pv(uint32_t sbase, uint32_t tmem, int t, i
     const uint32_t d_tmem = tmem + uint32_t(C::O_COL0 + t * C::OST);
     // one MMA takes KSTEP keys: 32 bytes of each P row = 8 TMEM columns, KSTEP rows of V
 #pragma unroll
-    for (int kk = 0; kk < C::BC / C::KSTEP; ++kk) {
+    for (int kk = KK_BEGIN; kk < KK_END; ++kk) {
         if constexpr (C::FP8)
             sm100::mma_f8_ts_elected(d_tmem, a_tmem + uint32_t(kk * 8), b0 + uint64_t((kk * C::KSTEP * C::RB) >> 4),
                                      C::IDESC_O, (accumulate || kk > 0) ? 1u : 0u);
@@ -426,14 +436,28 @@ __device__ void mma_role(const FwdParams &p, uint32_t sbase, uint32_t tmem, cons
         // O_t += P_t,j V_j from the V tile in `slot`.
         auto issue_o = [&](int t, int j, int slot) -> bool {
             const int sb = int(p_got[t] % C::SB);
-            if (!warp_wait_bar<kRoleControl>(bar(C::B_PFULL + t * C::SB + sb), (p_got[t] / C::SB) & 1u, ctl,
-                                             kSitePFull))
+            if (!C::PSPLIT && !warp_wait_bar<kRoleControl>(bar(C::B_PFULL + t * C::SB + sb), (p_got[t] / C::SB) & 1u,
+                                                            ctl, kSitePFull))
                 return false;
             if (j == w.js[t] && u_local > 0 &&
                 !warp_wait_bar<kRoleControl>(bar(C::B_OEMPTY + t), (u_local - 1) & 1u, ctl, kSiteOEmpty))
                 return false;
-            sm100::tc_fence_after_sync();
-            issue_pv<C>(sbase, tmem, t, slot, sb, j > w.js[t]);
+            if constexpr (C::PSPLIT) {
+                // the first 64 keys of P are in TMEM
+                if (!warp_wait_bar<kRoleControl>(bar(C::B_PHALF + t * C::SB + sb), (p_got[t] / C::SB) & 1u, ctl,
+                                                 kSitePFull))
+                    return false;
+                sm100::tc_fence_after_sync();
+                issue_pv<C, 0, C::BC / C::KSTEP / 2>(sbase, tmem, t, slot, sb, j > w.js[t]);
+                if (!warp_wait_bar<kRoleControl>(bar(C::B_PFULL + t * C::SB + sb), (p_got[t] / C::SB) & 1u, ctl,
+                                                 kSitePFull))
+                    return false;
+                sm100::tc_fence_after_sync();
+                issue_pv<C, C::BC / C::KSTEP / 2>(sbase, tmem, t, slot, sb, true);
+            } else {
+                sm100::tc_fence_after_sync();
+                issue_pv<C>(sbase, tmem, t, slot, sb, j > w.js[t]);
+            }
             sm100::tc_commit_elected(bar(C::B_ODONE + t));
             if (!C::PSEP) sm100::tc_commit_elected(bar(C::B_PVDONE + t * C::SB + sb));
             if (j == w.je[t] - 1) sm100::tc_commit_elected(bar(C::B_OFINAL + t));
@@ -552,9 +576,9 @@ __device__ __forceinline__ float exp_pack_store_e4m3(const uint32_t (&s)[BC], fl
     return (a0 + a1) + (b0 + b1);
 }
 
-template <int BC, int SOFT_EXP, bool MIXED, bool F16>
+template <int BC, int SOFT_EXP, bool MIXED, bool F16, bool SPLIT = false>
 __device__ __forceinline__ float exp_pack_store(const uint32_t (&s)[BC], float c_log2, float neg_m,
-                                                uint32_t p_taddr) {
+                                                uint32_t p_taddr, uint32_t half_bar = 0) {
     const uint64_t c2 = sm100::pack2(c_log2, c_log2);
     const uint64_t nm2 = sm100::pack2(neg_m, neg_m);
     uint64_t acc0 = sm100::pack2(0.f, 0.f), acc1 = acc0;
@@ -581,6 +605,13 @@ __device__ __forceinline__ float exp_pack_store(const uint32_t (&s)[BC], float c
             pk[i] = sm100::pack_x2<F16>(lo, hi);
         }
         sm100::tmem_st32(p_taddr + uint32_t(32 * c), pk);
+        if constexpr (SPLIT) {
+            if (c == 0) {   // first 64 keys of P (and any rescale of O before it) are in TMEM
+                sm100::tmem_st_wait();
+                sm100::tc_fence_before_sync();
+                sm100::mbar_arrive(half_bar);
+            }
+        }
     }
     float a0, a1, b0, b1;
     sm100::unpack2(acc0, a0, a1);
@@ -602,6 +633,23 @@ __device__ void softmax_role(const FwdParams &p, uint32_t sbase, uint32_t tmem, 
     const uint32_t o_taddr = tmem + lane_off + uint32_t(C::O_COL0 + t * C::OST);
     const float c_log2 = p.scale_log2;
     uint32_t scnt = 0, ocnt = 0, ofin = 0;
+    // Lazy rescale: O_t holds the sum up to block j-1 at the old reference max; wait for
+    // that MMA (completion number `odone`), then scale this warp's rows by alpha (1 where
+    // the max held).
+    auto rescale_o = [&](bool need, float alpha, uint32_t odone) -> bool {
+        if (!__any_sync(0xffffffffu, need)) return true;
+        if (!warp_wait_bar(bar(C::B_ODONE + t), odone & 1u, ctl, kSiteODone)) return false;
+        sm100::tc_fence_after_sync();
+#pragma unroll
+        for (int c = 0; c < C::O_CHUNKS; ++c) {
+            uint32_t o[32];
+            sm100::tmem_ld32_sync(o_taddr + uint32_t(32 * c), o);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+            sm100::tmem_st32(o_taddr + uint32_t(32 * c), o);
+        }
+        return true;
+    };
 
     for (int u = blockIdx.x; u < p.num_units; u += gridDim.x) {
         const UnitInfo w = decode_unit<C>(u, p);
@@ -664,29 +712,22 @@ __device__ void softmax_role(const FwdParams &p, uint32_t sbase, uint32_t tmem, 
                     m_ref = mx_s;
                     need_rescale = true;
                 }
+                // with a split hand-off, O is rescaled before any of P is handed over (the
+                // first P V MMAs accumulate into O while the rest of P is computed)
+                if constexpr (C::PSPLIT)
+                    if (!rescale_o(need_rescale, alpha, ocnt + uint32_t(j - js) - 1u)) goto unwind;
                 const float neg_m = (m_ref == -INFINITY) ? 0.f : -m_ref;
+                const uint32_t half_bar = bar(C::B_PHALF + t * C::SB + sb);
                 if constexpr (C::FP8)
                     row_sum = exp_pack_store_e4m3<BC>(s, c_log2, neg_m, p_taddr);
                 else
-                    row_sum = need_mask ? exp_pack_store<BC, C::SOFT_EXP, false, C::F16>(s, c_log2, neg_m, p_taddr)
-                                        : exp_pack_store<BC, C::SOFT_EXP, true, C::F16>(s, c_log2, neg_m, p_taddr);
+                    row_sum = need_mask
+                                  ? exp_pack_store<BC, C::SOFT_EXP, false, C::F16, C::PSPLIT>(s, c_log2, neg_m, p_taddr, half_bar)
+                                  : exp_pack_store<BC, C::SOFT_EXP, true, C::F16, C::PSPLIT>(s, c_log2, neg_m, p_taddr, half_bar);
             }
             l = l * alpha + row_sum;
-
-            if (__any_sync(0xffffffffu, need_rescale)) {
-                // O_t holds the sum up to block j-1 at the old reference; wait for that
-                // MMA, then scale this warp's rows by alpha (1 where the max held).
-                if (!warp_wait_bar(bar(C::B_ODONE + t), (ocnt + uint32_t(j - js) - 1u) & 1u, ctl, kSiteODone)) goto unwind;
-                sm100::tc_fence_after_sync();
-#pragma unroll
-                for (int c = 0; c < C::O_CHUNKS; ++c) {
-                    uint32_t o[32];
-                    sm100::tmem_ld32_sync(o_taddr + uint32_t(32 * c), o);
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-                    sm100::tmem_st32(o_taddr + uint32_t(32 * c), o);
-                }
-            }
+            if constexpr (!C::PSPLIT)
+                if (!rescale_o(need_rescale, alpha, ocnt + uint32_t(j - js) - 1u)) goto unwind;
             sm100::tmem_st_wait();
             sm100::tc_fence_before_sync();
             sm100::mbar_arrive(bar(C::B_PFULL + t * C::SB + sb));
@@ -787,6 +828,7 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         for (int i = 0; i < C::NQT * C::SB; ++i) {
             sm100::mbar_init(bar(C::B_SFULL + i), 1);
             sm100::mbar_init(bar(C::B_PFULL + i), 128);
+            sm100::mbar_init(bar(C::B_PHALF + i), 128);
             sm100::mbar_init(bar(C::B_PVDONE + i), 1);
         }
         for (int t = 0; t < C::NQT; ++t) {
