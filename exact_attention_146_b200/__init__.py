@@ -30,7 +30,7 @@ FA_ERR_SCRATCH_LIMIT = 9
 SPLITKV_STATIC_SCRATCH_BYTES = 16 * 1024 * 1024
 
 EXPORTED = ("fa_fwd", "fa_fwd_window", "fa_fwd_splitkv", "fa_splitkv_workspace_bytes", "fa_splitkv_default_splits",
-            "fa_fwd_splitkv_static", "fa_fwd_f16", "fa_fwd_fp8", "fa_fwd_partial", "fa_merge_partials", "fa_bwd", "fa_bwd_f16", "fa_bwd_workspace_bytes", "fa_status_string", "fa_device_status", "fa_tile_config", "fa_version")
+            "fa_fwd_splitkv_static", "fa_fwd_f16", "fa_fwd_fp8", "fa_fwd_partial", "fa_merge_partials", "fa_bwd", "fa_bwd_f16", "fa_bwd_window", "fa_bwd_workspace_bytes", "fa_status_string", "fa_device_status", "fa_tile_config", "fa_version")
 
 
 class FaError(RuntimeError):
@@ -74,6 +74,8 @@ def lib() -> ctypes.CDLL:
         L.fa_bwd.restype = ci
         L.fa_bwd_f16.argtypes = [vp] * 9 + [ci] * 6 + [cf, ci, vp, ctypes.c_size_t, vp]
         L.fa_bwd_f16.restype = ci
+        L.fa_bwd_window.argtypes = [vp] * 9 + [ci] * 6 + [cf, ci, vp, ctypes.c_size_t, vp]
+        L.fa_bwd_window.restype = ci
         L.fa_bwd_workspace_bytes.argtypes = [ci, ci, ci, ci]
         L.fa_bwd_workspace_bytes.restype = ctypes.c_size_t
         L.fa_status_string.argtypes = [ci]
@@ -259,7 +261,7 @@ def bwd_workspace_bytes(B: int, Hq: int, Nq: int, d: int) -> int:
 
 
 def fa_bwd(q, k, v, out, dout, lse, *, causal: bool = False, scale: float | None = None, dq=None, dk=None,
-           dv=None, workspace=None, stream=None):
+           dv=None, workspace=None, stream=None, window: int | None = None):
     """Exact attention backward (fa_bwd, fa_bwd_f16 for fp16) on [B, N, H, d] CUDA tensors:
     returns (dq, dk, dv) for the loss sum(out * dout), given the forward's out and lse
     [B, Hq, Nq] fp32.  `workspace` (uint8, >= bwd_workspace_bytes) is allocated here if None."""
@@ -281,10 +283,16 @@ def fa_bwd(q, k, v, out, dout, lse, *, causal: bool = False, scale: float | None
     dv = torch.empty_like(v) if dv is None else dv
     if workspace is None:
         workspace = torch.empty(max(1, bwd_workspace_bytes(B, Hq, Nq, d)), dtype=torch.uint8, device=q.device)
-    entry = lib().fa_bwd_f16 if dt == torch.float16 else lib().fa_bwd
+    mask = 1 if causal else 0
+    if window is not None:      # fa_bwd_window: the sliding window (bf16)
+        if dt != torch.bfloat16:
+            raise ValueError("the sliding-window backward takes bf16")
+        entry, mask = lib().fa_bwd_window, int(window)
+    else:
+        entry = lib().fa_bwd_f16 if dt == torch.float16 else lib().fa_bwd
     rc = entry(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), dout.data_ptr(), lse.data_ptr(),
                       dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), B, Hq, Hkv, Nq, Nk, d, float(scale),
-                      1 if causal else 0, workspace.data_ptr(), workspace.numel() * workspace.element_size(),
+                      mask, workspace.data_ptr(), workspace.numel() * workspace.element_size(),
                       _stream_handle(stream))
     if rc != FA_OK:
         raise FaError(rc, "fa_bwd")

@@ -35,7 +35,7 @@ size_t bwd_bytes(int B, int Hq, int Nq, int d) {
 template <class C>
 int launch_bwd(const void *q, const void *k, const void *v, const void *out, const void *dout, const float *lse,
                void *dq, void *dk, void *dv, int B, int Hq, int Hkv, int Nq, int Nk, float scale, int causal,
-               float *dq_acc, float *delta, DeviceState &dev, int dev_id, int slot, cudaStream_t st) {
+               int window, float *dq_acc, float *delta, DeviceState &dev, int dev_id, int slot, cudaStream_t st) {
     auto kern = fa::bwd::fa_bwd_kernel<C>;
     {
         std::lock_guard<std::mutex> lock(g_mutex);
@@ -77,6 +77,7 @@ int launch_bwd(const void *q, const void *k, const void *v, const void *out, con
     p.Nk = Nk;
     p.n_rep = Hq / Hkv;
     p.causal = causal;
+    p.window = window;
     p.nkt = (Nk + fa::bwd::kRows - 1) / fa::bwd::kRows;
     p.nqt = (Nq + fa::bwd::kRows - 1) / fa::bwd::kRows;
     const long long units = (long long)B * Hkv * p.nkt;
@@ -98,12 +99,12 @@ int launch_bwd(const void *q, const void *k, const void *v, const void *out, con
 template <bool H>
 int dispatch_bwd(int d, const void *q, const void *k, const void *v, const void *out, const void *dout,
                  const float *lse, void *dq, void *dk, void *dv, int B, int Hq, int Hkv, int Nq, int Nk, float scale,
-                 int causal, float *dq_acc, float *delta, DeviceState &dev, int dev_id, cudaStream_t st) {
+                 int causal, int window, float *dq_acc, float *delta, DeviceState &dev, int dev_id, cudaStream_t st) {
     constexpr int base = H ? 5 : 0;
 #define FA_BWD_CASE(DIM, IDX)                                                                                      \
     case DIM:                                                                                                      \
         return launch_bwd<fa::bwd::BwdCfg<DIM, H>>(q, k, v, out, dout, lse, dq, dk, dv, B, Hq, Hkv, Nq, Nk, scale, \
-                                                   causal, dq_acc, delta, dev, dev_id, base + IDX, st);
+                                                   causal, window, dq_acc, delta, dev, dev_id, base + IDX, st);
     switch (d) {
         FA_BWD_CASE(32, 0)
         FA_BWD_CASE(64, 1)
@@ -117,11 +118,12 @@ int dispatch_bwd(int d, const void *q, const void *k, const void *v, const void 
 
 int backward(const void *q, const void *k, const void *v, const void *out, const void *dout, const float *lse,
              void *dq, void *dk, void *dv, int B, int Hq, int Hkv, int Nq, int Nk, int d, float scale, int causal,
-             void *workspace, size_t workspace_bytes, void *stream, bool f16) {
+             int window, void *workspace, size_t workspace_bytes, void *stream, bool f16) {
     // ---- host-only validation
     if (B < 0 || Hq <= 0 || Hkv <= 0 || Nq < 0 || Nk < 0) return FA_ERR_INVALID_ARG;
     if (Hq % Hkv != 0) return FA_ERR_INVALID_ARG;
     if (causal != 0 && causal != 1) return FA_ERR_INVALID_ARG;
+    if (window < 0 || (window > 0 && !causal)) return FA_ERR_INVALID_ARG;
     if (!std::isfinite(scale) || !(scale > 0.f)) return FA_ERR_INVALID_ARG;
     if (d != 32 && d != 64 && d != 80 && d != 96 && d != 128) return FA_ERR_UNSUPPORTED_HEAD_DIM;
     const size_t q_bytes = size_t(B) * size_t(Nq) * size_t(Hq) * size_t(d) * 2;
@@ -178,9 +180,9 @@ int backward(const void *q, const void *k, const void *v, const void *out, const
     }
     float *dq_acc = static_cast<float *>(workspace);
     float *delta = reinterpret_cast<float *>(static_cast<char *>(workspace) + bwd_acc_bytes(B, Hq, Nq, d));
-    return f16 ? dispatch_bwd<true>(d, q, k, v, out, dout, lse, dq, dk, dv, B, Hq, Hkv, Nq, Nk, scale, causal, dq_acc,
-                                    delta, *dev, dev_id, st)
-               : dispatch_bwd<false>(d, q, k, v, out, dout, lse, dq, dk, dv, B, Hq, Hkv, Nq, Nk, scale, causal,
+    return f16 ? dispatch_bwd<true>(d, q, k, v, out, dout, lse, dq, dk, dv, B, Hq, Hkv, Nq, Nk, scale, causal, window,
+                                    dq_acc, delta, *dev, dev_id, st)
+               : dispatch_bwd<false>(d, q, k, v, out, dout, lse, dq, dk, dv, B, Hq, Hkv, Nq, Nk, scale, causal, window,
                                      dq_acc, delta, *dev, dev_id, st);
 }
 
@@ -196,15 +198,23 @@ size_t fa_bwd_workspace_bytes(int B, int Hq, int Nq, int d) {
 int fa_bwd(const void *q, const void *k, const void *v, const void *out, const void *dout, const float *lse,
            void *dq, void *dk, void *dv, int B, int Hq, int Hkv, int Nq, int Nk, int d, float scale, int causal,
            void *workspace, size_t workspace_bytes, void *stream) {
-    return backward(q, k, v, out, dout, lse, dq, dk, dv, B, Hq, Hkv, Nq, Nk, d, scale, causal, workspace,
+    return backward(q, k, v, out, dout, lse, dq, dk, dv, B, Hq, Hkv, Nq, Nk, d, scale, causal, 0, workspace,
                     workspace_bytes, stream, false);
 }
 
 int fa_bwd_f16(const void *q, const void *k, const void *v, const void *out, const void *dout, const float *lse,
                void *dq, void *dk, void *dv, int B, int Hq, int Hkv, int Nq, int Nk, int d, float scale, int causal,
                void *workspace, size_t workspace_bytes, void *stream) {
-    return backward(q, k, v, out, dout, lse, dq, dk, dv, B, Hq, Hkv, Nq, Nk, d, scale, causal, workspace,
+    return backward(q, k, v, out, dout, lse, dq, dk, dv, B, Hq, Hkv, Nq, Nk, d, scale, causal, 0, workspace,
                     workspace_bytes, stream, true);
+}
+
+int fa_bwd_window(const void *q, const void *k, const void *v, const void *out, const void *dout, const float *lse,
+                  void *dq, void *dk, void *dv, int B, int Hq, int Hkv, int Nq, int Nk, int d, float scale, int window,
+                  void *workspace, size_t workspace_bytes, void *stream) {
+    if (window < 1) return FA_ERR_INVALID_ARG;
+    return backward(q, k, v, out, dout, lse, dq, dk, dv, B, Hq, Hkv, Nq, Nk, d, scale, 1, window, workspace,
+                    workspace_bytes, stream, false);
 }
 
 }  // extern "C"

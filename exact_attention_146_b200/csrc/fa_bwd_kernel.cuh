@@ -57,6 +57,7 @@ struct BwdParams {
     uint16_t *dk, *dv;    // [B, Nk, Hkv, d] bf16 bits
     int *status;
     int B, Hq, Hkv, Nq, Nk, n_rep, causal;
+    int window;           // 0, or W >= 1: sliding window of the W keys ending at the causal diagonal
     int nkt, nqt;         // key tiles, query tiles (of 128 rows)
     int num_units;        // B * Hkv * nkt
     float scale, scale_log2;
@@ -112,7 +113,7 @@ struct BwdCfg {
 };
 
 struct Unit {
-    int b, kvh, kt, i_lo, nsteps;
+    int b, kvh, kt, i_lo, i_hi, nsteps;   // query tiles [i_lo, i_hi) see the key tile
 };
 
 __device__ __forceinline__ Unit decode_unit(int u, const BwdParams &p) {
@@ -129,18 +130,26 @@ __device__ __forceinline__ Unit decode_unit(int u, const BwdParams &p) {
     w.b = r / p.Hkv;
     w.kvh = r - w.b * p.Hkv;
     w.i_lo = 0;
+    w.i_hi = p.nqt;
+    const int diag = p.Nk - p.Nq;
     if (p.causal) {   // first query tile whose last row sees key k0 = kt * 128
-        const int x = w.kt * kRows - (p.Nk - p.Nq);
+        const int x = w.kt * kRows - diag;
         w.i_lo = x > 0 ? x / kRows : 0;
         if (w.i_lo > p.nqt) w.i_lo = p.nqt;
     }
-    w.nsteps = p.n_rep * (p.nqt - w.i_lo);
+    if (p.window > 0) {   // query q sees key k only if q < k - diag + W: the tile's last key bounds it
+        const long long q_end = (long long)w.kt * kRows + (kRows - 1) - diag + p.window;   // exclusive
+        const long long t_end = q_end <= 0 ? 0 : (q_end + kRows - 1) / kRows;
+        if (t_end < w.i_hi) w.i_hi = int(t_end);
+        if (w.i_hi < w.i_lo) w.i_hi = w.i_lo;
+    }
+    w.nsteps = p.n_rep * (w.i_hi - w.i_lo);
     return w;
 }
 
 // step s of a unit -> (query head, query tile)
 __device__ __forceinline__ void step_of(const Unit &w, int s, const BwdParams &p, int &hq, int &it) {
-    const int per_head = p.nqt - w.i_lo;
+    const int per_head = w.i_hi - w.i_lo;
     const int r = s / per_head;
     hq = w.kvh * p.n_rep + r;
     it = w.i_lo + (s - r * per_head);
@@ -353,6 +362,8 @@ __device__ void sg_role(const BwdParams &p, uint32_t sbase, uint8_t *smem, uint3
                 // key visible to query q iff key < Nk, q < Nq and (causal) key <= q + diag
                 const int q_lim = p.Nq - i0;                         // local query bound
                 const int key_lo_q = p.causal ? key - diag - i0 : -0x7fffffff;   // first local q seeing key
+                // sliding window: local queries q < key - diag + W - i0 still see the key
+                const int key_hi_q = p.window > 0 ? key - diag + p.window - i0 : 0x7fffffff;
                 const bool key_ok = key < p.Nk;
                 uint8_t *ds_row = smem + C::SMEM_DS + r * C::DS_RB;
 #pragma unroll 1
@@ -367,7 +378,7 @@ __device__ void sg_role(const BwdParams &p, uint32_t sbase, uint8_t *smem, uint3
 #pragma unroll
                         for (int h = 0; h < 2; ++h) {
                             const int ql = 32 * c + e + h;
-                            const bool vis = key_ok && ql < q_lim && ql >= key_lo_q;
+                            const bool vis = key_ok && ql < q_lim && ql >= key_lo_q && ql < key_hi_q;
                             const float x = fmaf(__uint_as_float(sv[e + h]), p.scale_log2, -l2v[ql]);
                             const float pv = vis ? sm100::ex2_approx(x) : 0.f;
                             pr[h] = pv;

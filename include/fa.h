@@ -213,10 +213,15 @@ size_t fa_bwd_workspace_bytes(int B, int Hq, int Nq, int d);
 int fa_bwd(const void *q, const void *k, const void *v, const void *out, const void *dout, const float *lse,
            void *dq, void *dk, void *dv, int B, int Hq, int Hkv, int Nq, int Nk, int d, float scale, int causal,
            void *workspace, size_t workspace_bytes, void *stream);
-/* fa_bwd_f16: the same with fp16 q, k, v, out, dout, dq, dk, dv (P and dS rounded to fp16). */
+/* fa_bwd_f16: the same with fp16 q, k, v, out, dout, dq, dk, dv (P and dS rounded to fp16).
+ * fa_bwd_window: fa_bwd for the sliding-window mask of fa_fwd_window (window >= 1; out and
+ *   lse from fa_fwd_window with the same W); query tiles outside a key tile's band are skipped. */
 int fa_bwd_f16(const void *q, const void *k, const void *v, const void *out, const void *dout, const float *lse,
                void *dq, void *dk, void *dv, int B, int Hq, int Hkv, int Nq, int Nk, int d, float scale, int causal,
                void *workspace, size_t workspace_bytes, void *stream);
+int fa_bwd_window(const void *q, const void *k, const void *v, const void *out, const void *dout, const float *lse,
+                  void *dq, void *dk, void *dv, int B, int Hq, int Hkv, int Nq, int Nk, int d, float scale, int window,
+                  void *workspace, size_t workspace_bytes, void *stream);
 
 /*
  * Key-sharded attention, for one sequence too long for one GPU: each GPU holds a shard of

@@ -159,6 +159,9 @@ def test_bwd_validation(L):
     assert _bwd(L, dq=FAKE) == fa.FA_ERR_OVERLAP                       # dq over q
     assert _bwd(L, ws=FAKE + (7 << 30)) == fa.FA_ERR_OVERLAP           # workspace over dk
     assert _bwd(L) in (fa.FA_ERR_UNSUPPORTED_DEVICE, fa.FA_ERR_NOT_DEVICE_MEMORY)
+    assert L.fa_bwd_window(FAKE, FAKE + (1 << 30), FAKE + (2 << 30), FAKE + (3 << 30), FAKE + (6 << 30),
+                           FAKE + (4 << 30), FAKE + (5 << 30), FAKE + (7 << 30), FAKE + (8 << 30), 1, 2, 1, 64, 64,
+                           128, 0.125, 0, FAKE + (12 << 30), 1 << 30, None) == fa.FA_ERR_INVALID_ARG   # W = 0
 
 
 def test_fp8_validation(L):

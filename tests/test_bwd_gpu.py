@@ -120,6 +120,30 @@ def test_bwd_f16(orc, d, causal):
     compare_grads(got, ref, f"f16 d={d} causal={causal}")
 
 
+@pytest.mark.parametrize("W", [1, 100, 300, 5000])
+@pytest.mark.parametrize("shape", [(1, 4, 2, 600, 600, 128), (1, 2, 1, 300, 700, 64), (1, 2, 2, 500, 260, 96)])
+def test_bwd_window(orc, W, shape):
+    """Sliding-window backward (fa_bwd_window) after fa_fwd_window, against the oracle's
+    gradients with the same window (query tiles outside a key tile's band are skipped)."""
+    import torch
+    import exact_attention_146_b200 as fa
+    B, Hq, Hkv, Nq, Nk, d = shape
+    x, do_bits = inputs(B, Hq, Hkv, Nq, Nk, d, seed=W + Nq)
+    scale = 1.0 / math.sqrt(d)
+    q, k, v = (_parity.to_device(x[n], torch) for n in ("q", "k", "v"))
+    do = _parity.to_device(do_bits, torch)
+    out, lse = fa.fa_fwd(q, k, v, causal=True, scale=scale, window=W)
+    dq, dk, dv = fa.fa_bwd(q, k, v, out, do, lse, causal=True, scale=scale, window=W,
+                           dq=torch.full_like(q, float("nan")), dk=torch.full_like(k, float("nan")),
+                           dv=torch.full_like(v, float("nan")))
+    st, word = fa.device_status()
+    assert st == fa.FA_OK, f"device status {st} ({word:#x})"
+    torch.cuda.synchronize()
+    got = tuple(_parity.bf16_to_f64(t) for t in (dq, dk, dv))
+    ref = orc.backward(x["q"], x["k"], x["v"], do_bits, scale, True, window=W)
+    compare_grads(got, ref, f"window W={W} {shape}")
+
+
 def test_bwd_empty_sides():
     """Nq = 0: dK = dV = 0; Nk = 0: dQ = 0."""
     import torch
