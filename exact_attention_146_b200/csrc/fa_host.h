@@ -11,9 +11,10 @@
 
 namespace fa_host {
 
-constexpr int kNumCfgSlots = 19;   // forward: 7 head dims x 2 element types; backward: 2 head dims; FP8
-constexpr int kBwdSlot0 = 16;      // backward d = 64, 128 use slots 16, 17
-constexpr int kFp8Slot = 18;
+// Forward instantiations with per-device launch state: slots 0-6 bf16 and 8-14 fp16 (one per
+// head dim), 15 the FP8 one.  (The backward keeps its own state in fa_bwd.cu.)
+constexpr int kNumCfgSlots = 16;
+constexpr int kFp8Slot = 15;
 
 constexpr int kMaxDevices = 64;
 constexpr int kMaxSplits = 256;

@@ -90,15 +90,11 @@ struct TileCfg {
     static constexpr int CW = RB / ES;                    // elements per swizzled smem row
     static constexpr int KSTEP = 32 / ES;                 // K elements per MMA (32 bytes)
     static constexpr int PCOLS = BC * ES / 4;             // TMEM columns of one row of P
-#ifndef FA_NO_PSPLIT
     // P is handed to the P V MMAs in two 64-key halves: the first half of P V runs while
     // the softmax computes the second half of P.  Worth it where the exponentials dominate
     // (d <= 80: 6-10 % faster); at d >= 96 the extra register pressure costs more than the
     // overlap gains, so the hand-off stays whole there.
     static constexpr bool PSPLIT = (BC == 128) && !FP8 && D <= 80;
-#else
-    static constexpr bool PSPLIT = false;
-#endif
     static constexpr int NCH = (D + CW - 1) / CW;         // column chunks of a tile
     static constexpr int Q_CHUNK = kBlockQ * RB;
     static constexpr int KV_CHUNK = BC * RB;
