@@ -60,12 +60,21 @@ def tensor_peak(pk, w):
 FORWARD_SOURCES = ("fa_fwd.cu", "fa_host.h", "fa_kernel.cuh", "sm100.cuh")
 
 
+def _code_only(text: str) -> str:
+    """C/C++ source with comments removed and whitespace collapsed (none of these files
+    has a comment marker inside a string literal)."""
+    text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", " ", text)
+    return " ".join(text.split())
+
+
 def kernel_source_hash() -> str:
-    """Hash of the sources the forward kernel and its launch are built from (the backward's
-    own files are left out, so they can change without invalidating forward profiles)."""
+    """Hash of the code (comments aside) the forward kernel and its launch are built from;
+    the backward's own files are left out, so they can change without invalidating forward
+    profiles."""
     h = hashlib.sha256()
     for name in FORWARD_SOURCES:
-        h.update((ROOT / "exact_attention_146_b200" / "csrc" / name).read_bytes())
+        h.update(_code_only((ROOT / "exact_attention_146_b200" / "csrc" / name).read_text()).encode())
     return h.hexdigest()[:16]
 
 

@@ -9,19 +9,24 @@
 // the output is divided by l once at the end.
 //
 // How it maps onto a B200 SM (one CTA per SM, persistent over work units):
-//   * work unit = (batch b, query head hq, block of NQT x 128 query rows);
+//   * work unit = (batch b, query head hq, block of NQT x 128 query rows; with GQA
+//     packing the n_rep heads of one KV head share a unit, their rows stacked; with
+//     split-KV or a key-shard partial, also a slice of the key tiles);
 //   * TMA warp (one thread): Q tiles once per unit, then K_j, V_j into an NS-slot
 //     shared-memory ring guarded by full/empty mbarriers;
 //   * MMA warp (one thread): S_t = Q_t K_j^T with tcgen05.mma into TMEM (fp32), and
-//     O_t += P_t V_j with P read straight from TMEM (it overwrites S_t as bf16);
+//     O_t += P_t V_j with P read straight from TMEM (it overwrites S_t as bf16 / fp16 /
+//     E4M3, or has columns of its own for d <= 64);
 //     the two query tiles are interleaved so that one tile's softmax runs while the
 //     tensor core works on the other tile;
 //   * softmax warpgroup t (128 threads, thread r owns row r of tile t, which is TMEM
 //     lane r): loads its row of S_t, masks, takes the row max, p = 2^(s*scale*log2e - m)
-//     with one FFMA + ex2 per element, writes P back as bf16, keeps m and l in
+//     with one FFMA + ex2 per element, writes P back (in two halves for d <= 80, so the
+//     first half of P V overlaps the second half of the exponentials), keeps m and l in
 //     registers, rescales its O row in TMEM only when the max grew by more than
 //     2^8 (the final O / l is unchanged by the reference max used), and at the end
-//     writes O / l as bf16 and LSE = (m + log2 l) ln 2.
+//     writes O / l and LSE = (m + log2 l) ln 2 (split-KV / key shards: fp32 O / l and the
+//     slice's LSE to a workspace, combined by fa_splitkv_merge_kernel).
 // Every pipeline wait is bounded: after a time limit the kernel records
 // FA_ERR_DEVICE_TIMEOUT in a device status word, unwinds every role, waits for its own
 // in-flight copies and MMAs, frees TMEM and returns.

@@ -175,6 +175,37 @@ def test_fp8_validation(L):
     assert call() in (fa.FA_ERR_UNSUPPORTED_DEVICE, fa.FA_ERR_NOT_DEVICE_MEMORY)
 
 
+def test_partial_and_merge_validation(L):
+    """Key-shard partial: 0 <= key_offset, key_offset + Nk <= Nk_total; merge: R >= 1."""
+    def partial(key_offset=0, nk_total=64, Nk=64, d=128, o_part=FAKE + (3 << 30)):
+        return L.fa_fwd_partial(FAKE, FAKE + (1 << 30), FAKE + (2 << 30), o_part, FAKE + (4 << 30),
+                                1, 2, 1, 16, Nk, d, 0.125, 1, key_offset, nk_total, None)
+    assert partial(key_offset=-1) == fa.FA_ERR_INVALID_ARG
+    assert partial(key_offset=1, nk_total=64) == fa.FA_ERR_INVALID_ARG        # shard runs past the end
+    assert partial(d=48) == fa.FA_ERR_UNSUPPORTED_HEAD_DIM
+    assert partial(o_part=FAKE + (3 << 30) + 4) == fa.FA_ERR_MISALIGNED       # fp32 partial needs 16 bytes
+    assert partial(o_part=FAKE) == fa.FA_ERR_OVERLAP                           # partial over q
+    assert partial() in (fa.FA_ERR_UNSUPPORTED_DEVICE, fa.FA_ERR_NOT_DEVICE_MEMORY)
+
+    def merge(R=2, out=FAKE + (6 << 30), d=128):
+        return L.fa_merge_partials(FAKE, FAKE + (2 << 30), R, out, FAKE + (7 << 30), 1, 2, 16, d, None)
+    assert merge(R=0) == fa.FA_ERR_INVALID_ARG
+    assert merge(d=100) == fa.FA_ERR_UNSUPPORTED_HEAD_DIM
+    assert merge(out=FAKE + 64) == fa.FA_ERR_OVERLAP                          # out over the partials
+    assert merge() in (fa.FA_ERR_UNSUPPORTED_DEVICE, fa.FA_ERR_NOT_DEVICE_MEMORY)
+
+
+def test_f16_entry_validates_like_bf16(L):
+    args = (FAKE, FAKE + (1 << 30), FAKE + (2 << 30), FAKE + (3 << 30), FAKE + (4 << 30), 1, 2, 1, 64, 64)
+    assert L.fa_fwd_f16(*args, 48, 0.125, 0, None) == fa.FA_ERR_UNSUPPORTED_HEAD_DIM
+    assert L.fa_fwd_f16(*args, 128, -1.0, 0, None) == fa.FA_ERR_INVALID_ARG
+    assert L.fa_fwd_f16(*args, 128, 0.125, 3, None) == fa.FA_ERR_INVALID_ARG
+    assert L.fa_fwd_f16(*args, 128, 0.125, 1, None) in (fa.FA_ERR_UNSUPPORTED_DEVICE, fa.FA_ERR_NOT_DEVICE_MEMORY)
+    assert L.fa_bwd_f16(FAKE, FAKE + (1 << 30), FAKE + (2 << 30), FAKE + (3 << 30), FAKE + (6 << 30), FAKE + (4 << 30),
+                        FAKE + (5 << 30), FAKE + (7 << 30), FAKE + (8 << 30), 1, 2, 1, 64, 64, 192, 0.125, 0,
+                        FAKE + (12 << 30), 1 << 30, None) == fa.FA_ERR_UNSUPPORTED_HEAD_DIM
+
+
 def test_empty_problems_are_noops(L):
     # no output rows: nothing to validate against the device, nothing launched
     assert call(L, B=0, q=None, k=None, v=None, out=None, lse=None) == fa.FA_OK
