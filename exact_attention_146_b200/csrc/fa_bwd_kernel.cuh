@@ -90,7 +90,8 @@ struct BwdCfg {
                          B_S_FULL = B_Q_EMPTY + NQS, B_P_FULL = B_S_FULL + 1, B_MMA34 = B_P_FULL + 1,
                          B_DQ_FULL = B_MMA34 + 1, B_DQ_EMPTY = B_DQ_FULL + 1, B_ACC_FULL = B_DQ_EMPTY + 1,
                          B_ACC_EMPTY = B_ACC_FULL + 1, B_VEC = B_ACC_EMPTY + 1, B_DRAIN = B_VEC + 1,
-                         NUM_BARS = B_DRAIN + 1;
+                         B_P_HALF = B_DRAIN + 1,   // P^T, dS^T of the first 64 queries in TMEM
+                         NUM_BARS = B_P_HALF + 1;
     static constexpr int SMEM_MISC = SMEM_BAR + NUM_BARS * 8;
     // Each CTA holds all 512 TMEM columns: ask for enough shared memory that a second CTA
     // can never be resident on the same SM (it would only wait in the allocation).
@@ -282,21 +283,28 @@ __device__ void mma_issuer(const BwdParams &p, uint32_t sbase, uint32_t tmem, co
                 sm100::mma_bf16_ss_elected(tmem + C::COL_B, v_km + off, do_km + off, C::IDESC_SS, kk > 0 ? 1u : 0u);
             }
             sm100::tc_commit_elected(bar(C::B_S_FULL));
-            if (!warp_wait(bar(C::B_P_FULL), n_step & 1u, ctl, kSitePFull)) { ok = false; break; }
+            // dV += P^T dO, dK += dS^T Q over the step's queries: the first 64 as soon as the
+            // SG warpgroup has written them, the rest once it has finished
+            if (!warp_wait(bar(C::B_P_HALF), n_step & 1u, ctl, kSitePFull)) { ok = false; break; }
             if (s == 0 && n_unit > 0 && !warp_wait(bar(C::B_ACC_EMPTY), (n_unit - 1u) & 1u, ctl, kSiteAccEmpty)) {
                 ok = false;
                 break;
             }
-            sm100::tc_fence_after_sync();
+            for (int half = 0; half < 2; ++half) {
+                if (half == 1 && !warp_wait(bar(C::B_P_FULL), n_step & 1u, ctl, kSitePFull)) { ok = false; break; }
+                sm100::tc_fence_after_sync();
 #pragma unroll
-            for (int kk = 0; kk < kRows / 16; ++kk) {   // dV += P^T dO, dK += dS^T Q
-                const uint32_t boff = uint32_t(kk * 16 * C::RB) >> 4;
-                const uint32_t acc = (s > 0 || kk > 0) ? 1u : 0u;
-                sm100::mma_bf16_ts_elected(tmem + C::COL_DV, tmem + C::COL_A + uint32_t(kk * 8), do_mn + boff,
-                                           C::IDESC_TS, acc);
-                sm100::mma_bf16_ts_elected(tmem + C::COL_DK, tmem + C::COL_B + uint32_t(kk * 8), q_mn + boff,
-                                           C::IDESC_TS, acc);
+                for (int k4 = 0; k4 < kRows / 32; ++k4) {
+                    const int kk = half * (kRows / 32) + k4;
+                    const uint32_t boff = uint32_t(kk * 16 * C::RB) >> 4;
+                    const uint32_t acc = (s > 0 || kk > 0) ? 1u : 0u;
+                    sm100::mma_bf16_ts_elected(tmem + C::COL_DV, tmem + C::COL_A + uint32_t(kk * 8), do_mn + boff,
+                                               C::IDESC_TS, acc);
+                    sm100::mma_bf16_ts_elected(tmem + C::COL_DK, tmem + C::COL_B + uint32_t(kk * 8), q_mn + boff,
+                                               C::IDESC_TS, acc);
+                }
             }
+            if (!ok) break;
             sm100::tc_commit_elected(bar(C::B_MMA34));
             sm100::tc_commit_elected(bar(C::B_Q_EMPTY + slot));
             if (s == w.nsteps - 1) sm100::tc_commit_elected(bar(C::B_ACC_FULL));
@@ -397,6 +405,11 @@ __device__ void sg_role(const BwdParams &p, uint32_t sbase, uint8_t *smem, uint3
                         const int unit = ((c % 2) * 4 + v4) ^ (r & 7);
                         *reinterpret_cast<uint4 *>(chunk_row + unit * 16) =
                             make_uint4(dk[4 * v4], dk[4 * v4 + 1], dk[4 * v4 + 2], dk[4 * v4 + 3]);
+                    }
+                    if (c == 1) {   // the first 64 queries' P^T and dS^T are in TMEM
+                        sm100::tmem_st_wait();
+                        sm100::tc_fence_before_sync();
+                        sm100::mbar_arrive(bar(C::B_P_HALF));
                     }
                 }
             }
@@ -511,6 +524,7 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         }
         sm100::mbar_init(bar(C::B_S_FULL), 1);
         sm100::mbar_init(bar(C::B_P_FULL), kRows);
+        sm100::mbar_init(bar(C::B_P_HALF), kRows);
         sm100::mbar_init(bar(C::B_MMA34), 1);
         sm100::mbar_init(bar(C::B_DQ_FULL), 1);
         sm100::mbar_init(bar(C::B_DQ_EMPTY), kRows);
