@@ -99,6 +99,11 @@ struct BwdCfg {
     static constexpr int SMEM_BYTES = SMEM_NEEDED > 120 * 1024 ? SMEM_NEEDED : 120 * 1024;
     // TMEM columns
     static constexpr int COL_A = 0, COL_B = 128, COL_DV = 256, COL_DK = 256 + DCH * 32;
+    // dQ of a step: d <= 64 fits the upper half of region A (S^T columns the SG warpgroup has
+    // read; P^T uses the lower half), so its MMA need not wait for the dV MMAs to read P^T;
+    // larger d take all of region A once they have
+    static constexpr bool DQ_UPPER = D <= 64;
+    static constexpr int COL_DQ = DQ_UPPER ? COL_A + 64 : COL_A;
     static constexpr int TMEM_COLS = 512;
     // warps: 0 TMA, 1 MMA, 2-3 idle, 4-7 SG, 8-11 DW
     static constexpr int THREADS = 384;
@@ -305,16 +310,18 @@ __device__ void mma_issuer(const BwdParams &p, uint32_t sbase, uint32_t tmem, co
                 }
             }
             if (!ok) break;
-            sm100::tc_commit_elected(bar(C::B_MMA34));
+            if constexpr (!C::DQ_UPPER) sm100::tc_commit_elected(bar(C::B_MMA34));
             sm100::tc_commit_elected(bar(C::B_Q_EMPTY + slot));
             if (s == w.nsteps - 1) sm100::tc_commit_elected(bar(C::B_ACC_FULL));
-            // dQ goes over region A: wait until the dV MMAs have read P^T from it
-            if (!warp_wait(bar(C::B_MMA34), n_step & 1u, ctl, kSiteMma34)) { ok = false; break; }
-            sm100::tc_fence_after_sync();
+            // dQ over all of region A: wait until the dV MMAs have read P^T from it
+            if constexpr (!C::DQ_UPPER) {
+                if (!warp_wait(bar(C::B_MMA34), n_step & 1u, ctl, kSiteMma34)) { ok = false; break; }
+                sm100::tc_fence_after_sync();
+            }
 #pragma unroll
             for (int kk = 0; kk < kRows / 16; ++kk) {   // dQ = dS K
                 const uint32_t a_off = uint32_t(kk * 16 * C::DS_RB) >> 4, b_off = uint32_t(kk * 16 * C::RB) >> 4;
-                sm100::mma_bf16_ss_elected(tmem + C::COL_A, ds_mn + a_off, k_mn + b_off, C::IDESC_DQ, kk > 0 ? 1u : 0u);
+                sm100::mma_bf16_ss_elected(tmem + C::COL_DQ, ds_mn + a_off, k_mn + b_off, C::IDESC_DQ, kk > 0 ? 1u : 0u);
             }
             sm100::tc_commit_elected(bar(C::B_DQ_FULL));
         }
@@ -455,7 +462,7 @@ __device__ void dw_role(const BwdParams &p, uint32_t sbase, uint32_t tmem, const
             uint32_t v[C::DCH * 32];
 #pragma unroll
             for (int c = 0; c < C::DCH; ++c)
-                sm100::tmem_ld32_sync(tmem + lane_off + uint32_t(C::COL_A + 32 * c),
+                sm100::tmem_ld32_sync(tmem + lane_off + uint32_t(C::COL_DQ + 32 * c),
                                       *reinterpret_cast<uint32_t(*)[32]>(v + 32 * c));
             sm100::tc_fence_before_sync();
             sm100::mbar_arrive(bar(C::B_DQ_EMPTY));
