@@ -18,6 +18,33 @@ namespace {
 
 using namespace fa_host;
 
+using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                   const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                   const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+// The fp32 dQ accumulator [B, Nq, Hq, d] as a 4-D (d, Hq, Nq, B) tensor with [64 x 32] boxes
+// (128-byte rows, 128-byte swizzle): the destination of the TMA reductions.
+int encode_dq_acc(CUtensorMap *m, float *base, int d, int Hq, int Nq, int B) {
+    static EncodeTiledFn fn = [] {
+        void *f = nullptr;
+        cudaDriverEntryPointQueryResult q{};
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) != cudaSuccess ||
+            q != cudaDriverEntryPointSuccess)
+            return static_cast<EncodeTiledFn>(nullptr);
+        return reinterpret_cast<EncodeTiledFn>(f);
+    }();
+    if (fn == nullptr) return FA_ERR_CUDA;
+    const cuuint64_t dims[4] = {cuuint64_t(d), cuuint64_t(Hq), cuuint64_t(Nq), cuuint64_t(B)};
+    const cuuint64_t strides[3] = {cuuint64_t(d) * 4, cuuint64_t(Hq) * d * 4, cuuint64_t(Nq) * Hq * d * 4};
+    const cuuint32_t box[4] = {32, 1, 64, 1};
+    const cuuint32_t estr[4] = {1, 1, 1, 1};
+    const CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, base, dims, strides, box, estr,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? FA_OK : FA_ERR_CUDA;
+}
+
 // The backward covers every forward head dim whose S^T, dP^T, dV and dK fit the 512 TMEM
 // columns (256 + 2 d <= 512): d in {32, 64, 80, 96, 128}.  Per device, whether the dynamic
 // shared-memory size of each bf16 / fp16 instantiation has been set.
@@ -48,12 +75,13 @@ int launch_bwd(const void *q, const void *k, const void *v, const void *out, con
         }
     }
     constexpr int elem = C::F16 ? 1 : 0;
-    CUtensorMap mq, mk, mv, mdo;
+    CUtensorMap mq, mk, mv, mdo, mdq;
     int rc;
     if ((rc = encode_bnhd(&mq, q, C::D, Hq, Nq, B, C::CW, fa::bwd::kRows, 1, elem)) != FA_OK) return rc;
     if ((rc = encode_bnhd(&mdo, dout, C::D, Hq, Nq, B, C::CW, fa::bwd::kRows, 1, elem)) != FA_OK) return rc;
     if ((rc = encode_bnhd(&mk, k, C::D, Hkv, Nk, B, C::CW, fa::bwd::kRows, 1, elem)) != FA_OK) return rc;
     if ((rc = encode_bnhd(&mv, v, C::D, Hkv, Nk, B, C::CW, fa::bwd::kRows, 1, elem)) != FA_OK) return rc;
+    if ((rc = encode_dq_acc(&mdq, dq_acc, C::D, Hq, Nq, B)) != FA_OK) return rc;
 
     // D and the zeroed accumulator
     const long long rows = (long long)B * Nq * Hq;
@@ -86,7 +114,7 @@ int launch_bwd(const void *q, const void *k, const void *v, const void *out, con
     p.scale = scale;
     p.scale_log2 = scale * 1.4426950408889634f;
     const int grid = int(units < dev.num_sms ? units : dev.num_sms);
-    kern<<<grid, C::THREADS, C::SMEM_BYTES, st>>>(mq, mk, mv, mdo, p);
+    kern<<<grid, C::THREADS, C::SMEM_BYTES, st>>>(mq, mk, mv, mdo, mdq, p);
     if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
 
     const size_t n4 = size_t(rows) * C::D / 4;

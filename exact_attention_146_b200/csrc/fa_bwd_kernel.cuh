@@ -22,8 +22,10 @@
 //   MMA  dK_j += dS^T Q_i     (A = dS^T from TMEM)
 //   MMA  dQ_i  = dS K_j       (A = dS^T in shared memory, M-major; into region A once
 //                              P^T has been consumed)
-//   warpgroup DW (thread = query row): dQ_i rows -> fp32 reductions into a dQ accumulator
-//        in global memory (every key tile of the head contributes)
+//   warpgroup DW (thread = query row): dQ_i rows -> shared memory (the step's Q and dO
+//        slots, free once its MMAs are done) -> TMA bulk tensor reductions (add) into an
+//        fp32 dQ accumulator in global memory (every key tile of the head contributes);
+//        the slots go back to the TMA producer when the reductions have read them
 //
 // and at the end of the unit DW writes dV_j and scale * dK_j as bf16.  Each shared-memory
 // tile serves two MMAs in both roles (K-major where it is reduced over d, M/N-major where
@@ -47,7 +49,7 @@ constexpr int kRows = 128;   // key rows per unit = query rows per step = TMEM l
 enum BwdSite : int {
     kSiteKvFull = 21, kSiteKvEmpty = 22, kSiteQFull = 23, kSiteQEmpty = 24, kSiteSFull = 25, kSitePFull = 26,
     kSiteMma34 = 27, kSiteDqFull = 28, kSiteDqEmpty = 29, kSiteAccFull = 30, kSiteAccEmpty = 31, kSiteVec = 32,
-    kSiteDrain = 33
+    kSiteDrain = 33, kSiteStaged = 34
 };
 
 struct BwdParams {
@@ -91,7 +93,13 @@ struct BwdCfg {
                          B_DQ_FULL = B_MMA34 + 1, B_DQ_EMPTY = B_DQ_FULL + 1, B_ACC_FULL = B_DQ_EMPTY + 1,
                          B_ACC_EMPTY = B_ACC_FULL + 1, B_VEC = B_ACC_EMPTY + 1, B_DRAIN = B_VEC + 1,
                          B_P_HALF = B_DRAIN + 1,   // P^T, dS^T of the first 64 queries in TMEM
-                         NUM_BARS = B_P_HALF + 1;
+                         B_STAGED = B_P_HALF + 1,  // all 128 dQ rows of a step staged
+                         NUM_BARS = B_STAGED + 1;
+    // dQ leaves through [64 rows x 32 fp32] boxes (8 KB, 128-byte swizzle) staged in the
+    // step's Q slot, then its dO slot (B_Q_EMPTY is arrived once their reductions have
+    // read them)
+    static constexpr int DQ_BOX = 64 * 128;
+    static constexpr int DQ_NBOX = DCH * 2;
     static constexpr int SMEM_MISC = SMEM_BAR + NUM_BARS * 8;
     // Each CTA holds all 512 TMEM columns: ask for enough shared memory that a second CTA
     // can never be resident on the same SM (it would only wait in the allocation).
@@ -115,6 +123,7 @@ struct BwdCfg {
     static_assert(D % 16 == 0 && D >= 32 && D <= 128, "backward head dims: MMA N granularity, TMEM budget");
     static_assert(COL_DK + DCH * 32 <= TMEM_COLS, "TMEM budget");
     static_assert(SMEM_DS % 1024 == 0, "dS^T needs 1024-byte alignment (128-byte swizzle atoms)");
+    static_assert(DQ_NBOX * DQ_BOX <= 2 * TILE && TILE % DQ_BOX == 0, "dQ staging fits the Q and dO slots");
     static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 };
 
@@ -199,6 +208,17 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16
         "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
         : "memory");
 }
+
+// Element-wise add of a [64 rows x 32 fp32] shared-memory box (128-byte swizzle) into the
+// tensor at (x, y, z, w) of `map`, tracked by this thread's bulk-async group.
+__device__ __forceinline__ void tma_reduce_add_4d(const CUtensorMap *map, uint32_t src, int x, int y, int z, int w) {
+    asm volatile("cp.reduce.async.bulk.tensor.4d.global.shared::cta.add.bulk_group [%0, {%2, %3, %4, %5}], [%1];"
+                 ::"l"(reinterpret_cast<uint64_t>(map)), "r"(src), "r"(x), "r"(y), "r"(z), "r"(w)
+                 : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_read_all() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
 // Make this thread's generic-proxy shared-memory writes visible to the tensor core.
 __device__ __forceinline__ void fence_proxy_async_smem() {
@@ -311,7 +331,6 @@ __device__ void mma_issuer(const BwdParams &p, uint32_t sbase, uint32_t tmem, co
             }
             if (!ok) break;
             if constexpr (!C::DQ_UPPER) sm100::tc_commit_elected(bar(C::B_MMA34));
-            sm100::tc_commit_elected(bar(C::B_Q_EMPTY + slot));
             if (s == w.nsteps - 1) sm100::tc_commit_elected(bar(C::B_ACC_FULL));
             // dQ over all of region A: wait until the dV MMAs have read P^T from it
             if constexpr (!C::DQ_UPPER) {
@@ -433,10 +452,17 @@ unwind:
 // ------------------------------------------------------------------ DW: dQ, dK, dV out (warps 8-11)
 
 template <class C>
-__device__ void dw_role(const BwdParams &p, uint32_t sbase, uint32_t tmem, const Ctl &ctl, int warp, int lane) {
+__device__ void dw_role(const BwdParams &p, const CUtensorMap *tm_dq, uint32_t sbase, uint8_t *smem, uint32_t tmem,
+                        const Ctl &ctl, int warp, int lane) {
     auto bar = [&](int i) { return sbase + C::SMEM_BAR + 8u * uint32_t(i); };
     const int r = (warp % 4) * 32 + lane;
     const uint32_t lane_off = uint32_t((warp % 4) * 32) << 16;
+    const bool issuer = warp == C::DW_WARP0;   // this warp's lane 0 issues the reductions
+    // staging box bi of a slot: the Q slot's bytes first, then the dO slot's
+    auto box_off = [&](int slot, int bi) -> int {
+        const int off = bi * C::DQ_BOX;
+        return off < C::TILE ? C::SMEM_Q + slot * C::TILE + off : C::SMEM_DO + slot * C::TILE + (off - C::TILE);
+    };
     uint32_t n_step = 0, n_unit = 0;
     for (int u = blockIdx.x; u < p.num_units; u += gridDim.x) {
         const Unit w = decode_unit(u, p);
@@ -454,9 +480,9 @@ __device__ void dw_role(const BwdParams &p, uint32_t sbase, uint32_t tmem, const
             int hq, it;
             step_of(w, s, p, hq, it);
             const int q = it * kRows + r;
-            if (!warp_wait(bar(C::B_DQ_FULL), n_step & 1u, ctl, kSiteDqFull)) return;
+            if (!warp_wait(bar(C::B_DQ_FULL), n_step & 1u, ctl, kSiteDqFull)) goto done;
             sm100::tc_fence_after_sync();
-            float *dst = p.dq_acc + ((size_t(w.b) * p.Nq + size_t(q)) * p.Hq + hq) * C::D;
+            (void)q;
             // the whole dQ row into registers first, so region A is free for the next
             // step's S^T while the reductions run
             uint32_t v[C::DCH * 32];
@@ -466,15 +492,38 @@ __device__ void dw_role(const BwdParams &p, uint32_t sbase, uint32_t tmem, const
                                       *reinterpret_cast<uint32_t(*)[32]>(v + 32 * c));
             sm100::tc_fence_before_sync();
             sm100::mbar_arrive(bar(C::B_DQ_EMPTY));
-            if (q < p.Nq) {
+            // stage the row (its MMAs are complete, so the step's Q and dO slots are free):
+            // row r of box (c, r / 64), 128-byte swizzle (16-byte unit index XOR row % 8)
+            const int slot = int(n_step % C::NQS);
 #pragma unroll
-                for (int m = 0; m < C::D / 4; ++m)
-                    atomicAdd(reinterpret_cast<float4 *>(dst + 4 * m),
-                              make_float4(__uint_as_float(v[4 * m]), __uint_as_float(v[4 * m + 1]),
-                                          __uint_as_float(v[4 * m + 2]), __uint_as_float(v[4 * m + 3])));
+            for (int c = 0; c < C::DCH; ++c) {
+                uint8_t *row = smem + box_off(slot, 2 * c + r / 64) + (r % 64) * 128;
+#pragma unroll
+                for (int u = 0; u < 8; ++u)
+                    *reinterpret_cast<uint4 *>(row + ((u ^ (r & 7)) * 16)) =
+                        make_uint4(v[32 * c + 4 * u], v[32 * c + 4 * u + 1], v[32 * c + 4 * u + 2], v[32 * c + 4 * u + 3]);
+            }
+            fence_proxy_async_smem();
+            sm100::mbar_arrive(bar(C::B_STAGED));
+            if (issuer) {
+                if (!warp_wait(bar(C::B_STAGED), n_step & 1u, ctl, kSiteStaged)) goto done;
+                if (lane == 0) {
+                    // rows past Nq and columns past d fall outside the tensor and are skipped;
+                    // a box that starts past Nq is not issued
+#pragma unroll
+                    for (int bi = 0; bi < C::DQ_NBOX; ++bi) {
+                        const int row0 = it * kRows + (bi % 2) * 64;
+                        if (row0 < p.Nq)
+                            tma_reduce_add_4d(tm_dq, sbase + box_off(slot, bi), (bi / 2) * 32, hq, row0, w.b);
+                    }
+                    bulk_commit();
+                    bulk_wait_read_all();
+                    sm100::mbar_arrive(bar(C::B_Q_EMPTY + slot));   // the slot back to the producer
+                }
+                __syncwarp();
             }
         }
-        if (!warp_wait(bar(C::B_ACC_FULL), n_unit & 1u, ctl, kSiteAccFull)) return;
+        if (!warp_wait(bar(C::B_ACC_FULL), n_unit & 1u, ctl, kSiteAccFull)) goto done;
         sm100::tc_fence_after_sync();
 #pragma unroll 1
         for (int c = 0; c < C::DCH; ++c) {
@@ -503,6 +552,8 @@ __device__ void dw_role(const BwdParams &p, uint32_t sbase, uint32_t tmem, const
         sm100::mbar_arrive(bar(C::B_ACC_EMPTY));
         ++n_unit;
     }
+done:
+    if (issuer && lane == 0) bulk_wait_all();   // every reduction has landed before the CTA exits
 }
 
 // ------------------------------------------------------------------ kernels
@@ -511,7 +562,7 @@ template <class C>
 __global__ void __launch_bounds__(C::THREADS, 1)
 fa_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
               const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
-              const __grid_constant__ BwdParams p) {
+              const __grid_constant__ CUtensorMap tm_dq, const __grid_constant__ BwdParams p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const uint32_t sbase = sm100::smem_u32(smem);
@@ -532,6 +583,7 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         sm100::mbar_init(bar(C::B_S_FULL), 1);
         sm100::mbar_init(bar(C::B_P_FULL), kRows);
         sm100::mbar_init(bar(C::B_P_HALF), kRows);
+        sm100::mbar_init(bar(C::B_STAGED), kRows);
         sm100::mbar_init(bar(C::B_MMA34), 1);
         sm100::mbar_init(bar(C::B_DQ_FULL), 1);
         sm100::mbar_init(bar(C::B_DQ_EMPTY), kRows);
@@ -558,7 +610,7 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     } else if (warp >= C::SG_WARP0 && warp < C::SG_WARP0 + 4) {
         sg_role<C>(p, sbase, smem, tmem, ctl, warp, lane);
     } else if (warp >= C::DW_WARP0 && warp < C::DW_WARP0 + 4) {
-        dw_role<C>(p, sbase, tmem, ctl, warp, lane);
+        dw_role<C>(p, &tm_dq, sbase, smem, tmem, ctl, warp, lane);
     }
     __syncwarp();
 
