@@ -199,6 +199,25 @@ __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, const C
     return all;
 }
 
+// Two 32-column TMEM loads of this thread's lane (a from ta, b from tb) behind one wait.
+#define FA_BWD_R8(a, i) "=r"(a[i]), "=r"(a[i + 1]), "=r"(a[i + 2]), "=r"(a[i + 3]), "=r"(a[i + 4]), "=r"(a[i + 5]), \
+                        "=r"(a[i + 6]), "=r"(a[i + 7])
+__device__ __forceinline__ void tmem_ld32x2_sync(uint32_t ta, uint32_t (&a)[32], uint32_t tb, uint32_t (&b)[32]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%64];\n\t"
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+        "{%32,%33,%34,%35,%36,%37,%38,%39,%40,%41,%42,%43,%44,%45,%46,%47,"
+        "%48,%49,%50,%51,%52,%53,%54,%55,%56,%57,%58,%59,%60,%61,%62,%63}, [%65];\n\t"
+        "tcgen05.wait::ld.sync.aligned;"
+        : FA_BWD_R8(a, 0), FA_BWD_R8(a, 8), FA_BWD_R8(a, 16), FA_BWD_R8(a, 24), FA_BWD_R8(b, 0), FA_BWD_R8(b, 8),
+          FA_BWD_R8(b, 16), FA_BWD_R8(b, 24)
+        : "r"(ta), "r"(tb)
+        : "memory");
+}
+#undef FA_BWD_R8
+
 // 16 consecutive TMEM columns of this thread's lane from registers (not yet waited on).
 __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
     asm volatile(
@@ -403,8 +422,14 @@ __device__ void sg_role(const BwdParams &p, uint32_t sbase, uint8_t *smem, uint3
 #pragma unroll 1
                 for (int c = 0; c < kRows / 32; ++c) {
                     uint32_t sv[32], dp[32];
-                    sm100::tmem_ld32_sync(tmem + lane_off + uint32_t(C::COL_A + 32 * c), sv);
-                    sm100::tmem_ld32_sync(tmem + lane_off + uint32_t(C::COL_B + 32 * c), dp);
+                    if constexpr (C::D < 128) {   // both loads behind one wait (d = 128: the
+                                                  // extra live registers cost more than it saves)
+                        tmem_ld32x2_sync(tmem + lane_off + uint32_t(C::COL_A + 32 * c), sv,
+                                         tmem + lane_off + uint32_t(C::COL_B + 32 * c), dp);
+                    } else {
+                        sm100::tmem_ld32_sync(tmem + lane_off + uint32_t(C::COL_A + 32 * c), sv);
+                        sm100::tmem_ld32_sync(tmem + lane_off + uint32_t(C::COL_B + 32 * c), dp);
+                    }
                     uint32_t pk[16], dk[16];
 #pragma unroll
                     for (int e = 0; e < 32; e += 2) {
