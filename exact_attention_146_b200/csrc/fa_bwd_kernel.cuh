@@ -34,6 +34,7 @@
 #pragma once
 
 #include <cstdint>
+#include <type_traits>
 
 #include <cuda.h>
 #include <cuda_bf16.h>
@@ -431,21 +432,46 @@ __device__ void sg_role(const BwdParams &p, uint32_t sbase, uint8_t *smem, uint3
                         sm100::tmem_ld32_sync(tmem + lane_off + uint32_t(C::COL_B + 32 * c), dp);
                     }
                     uint32_t pk[16], dk[16];
+                    // the chunk's 32 queries all see this thread's key (most chunks): no
+                    // per-element test when that holds for the whole warp
+                    const int q0 = 32 * c;
+                    const bool full = key_ok && q0 + 32 <= q_lim && q0 >= key_lo_q && q0 + 32 <= key_hi_q;
+                    const bool warp_full = __all_sync(0xffffffffu, full);
+                    // L log2e and D of the chunk's queries: broadcast 16-byte shared loads
+                    const float4 *l2v4 = reinterpret_cast<const float4 *>(l2v + q0);
+                    const float4 *dvv4 = reinterpret_cast<const float4 *>(dvv + q0);
+                    // two straight-line copies of the loop (no branch per element, so the
+                    // 32 exponentials of a chunk can overlap)
+                    auto chunk = [&](auto masked) {
 #pragma unroll
-                    for (int e = 0; e < 32; e += 2) {
-                        float pr[2], dsr[2];
+                        for (int e4 = 0; e4 < 8; ++e4) {
+                            const float4 l4 = l2v4[e4], d4 = dvv4[e4];
+                            float pr[4], dsr[4];
 #pragma unroll
-                        for (int h = 0; h < 2; ++h) {
-                            const int ql = 32 * c + e + h;
-                            const bool vis = key_ok && ql < q_lim && ql >= key_lo_q && ql < key_hi_q;
-                            const float x = fmaf(__uint_as_float(sv[e + h]), p.scale_log2, -l2v[ql]);
-                            const float pv = vis ? sm100::ex2_approx(x) : 0.f;
-                            pr[h] = pv;
-                            dsr[h] = pv * (__uint_as_float(dp[e + h]) - dvv[ql]);
+                            for (int h = 0; h < 4; ++h) {
+                                const int e = 4 * e4 + h;
+                                const float lq = h == 0 ? l4.x : h == 1 ? l4.y : h == 2 ? l4.z : l4.w;
+                                const float dq = h == 0 ? d4.x : h == 1 ? d4.y : h == 2 ? d4.z : d4.w;
+                                const float x = fmaf(__uint_as_float(sv[e]), p.scale_log2, -lq);
+                                float pv;
+                                if constexpr (decltype(masked)::value) {
+                                    const int ql = q0 + e;
+                                    const bool vis = key_ok && ql < q_lim && ql >= key_lo_q && ql < key_hi_q;
+                                    pv = vis ? sm100::ex2_approx(x) : 0.f;
+                                } else {
+                                    pv = sm100::ex2_approx(x);
+                                }
+                                pr[h] = pv;
+                                dsr[h] = pv * (__uint_as_float(dp[e]) - dq);
+                            }
+                            pk[2 * e4] = sm100::pack_x2<C::F16>(pr[0], pr[1]);
+                            pk[2 * e4 + 1] = sm100::pack_x2<C::F16>(pr[2], pr[3]);
+                            dk[2 * e4] = sm100::pack_x2<C::F16>(dsr[0], dsr[1]);
+                            dk[2 * e4 + 1] = sm100::pack_x2<C::F16>(dsr[2], dsr[3]);
                         }
-                        pk[e / 2] = sm100::pack_x2<C::F16>(pr[0], pr[1]);
-                        dk[e / 2] = sm100::pack_x2<C::F16>(dsr[0], dsr[1]);
-                    }
+                    };
+                    if (warp_full) chunk(std::false_type{});
+                    else chunk(std::true_type{});
                     tmem_st16(tmem + lane_off + uint32_t(C::COL_A + 16 * c), pk);
                     tmem_st16(tmem + lane_off + uint32_t(C::COL_B + 16 * c), dk);
                     // dS^T row r, queries 32c .. 32c+31: chunk c/2, 16-byte units (c%2)*4 .. +3,
