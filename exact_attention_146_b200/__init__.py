@@ -1,4 +1,8 @@
-"""B200-native exact attention forward: Python binding of libfa.so.
+"""B200-native exact attention: Python binding of libfa.so.
+
+Forward (fa_fwd: bf16 / fp16, causal or sliding window, split-KV; fa_fwd_fp8: E4M3),
+key-shard partials and their merge (fa_fwd_partial, fa_merge_partials; see kshard for the
+multi-GPU exchange) and the backward pass (fa_bwd).
 
 This module only marshals arguments (torch tensors -> device pointers, sizes and the
 current CUDA stream) into the C ABI declared in ``include/fa.h``; every step of the
@@ -11,11 +15,13 @@ import ctypes
 import math
 from pathlib import Path
 
-__all__ = ["fa_fwd", "device_status", "tile_config", "status_string", "FaError", "lib",
-           "SUPPORTED_HEAD_DIMS", "LIB_PATH"]
+__all__ = ["fa_fwd", "fa_fwd_fp8", "fa_fwd_partial", "fa_merge_partials", "fa_bwd", "fa_fwd_raw",
+           "splitkv_workspace_bytes", "splitkv_default_splits", "bwd_workspace_bytes", "device_status",
+           "tile_config", "status_string", "FaError", "lib", "SUPPORTED_HEAD_DIMS", "BWD_HEAD_DIMS", "LIB_PATH"]
 
 LIB_PATH = Path(__file__).resolve().parent / "libfa.so"
-SUPPORTED_HEAD_DIMS = (32, 64, 80, 96, 128, 192, 256)
+SUPPORTED_HEAD_DIMS = (32, 64, 80, 96, 128, 192, 256)   # forward
+BWD_HEAD_DIMS = (32, 64, 80, 96, 128)                    # backward
 
 FA_OK = 0
 FA_ERR_INVALID_ARG = 1
