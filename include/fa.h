@@ -26,7 +26,8 @@
  *
  * Conventions for every entry point:
  *  - All tensors are dense, row-major (C-contiguous), owned by the caller; the library
- *    allocates no device memory per call and keeps no pointer after it returns.
+ *    allocates no device memory per call (scratch is the caller's workspace, or the
+ *    static array of fa_fwd_splitkv_static) and keeps no pointer after it returns.
  *  - Pointers to tensors are DEVICE pointers on the calling thread's current CUDA device.
  *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
  *  - Work is enqueued asynchronously on `stream`; no host synchronisation happens,
@@ -252,9 +253,10 @@ const char *fa_status_string(int status);
 
 /*
  * fa_device_status -- synchronises `stream`, then returns and clears the current
- * device's kernel status word: FA_OK, or FA_ERR_DEVICE_TIMEOUT if a pipeline wait in
- * an fa_fwd kernel ran out of time.  FA_ERR_CUDA if the synchronisation itself failed.
- * If `detail` is not NULL it receives the raw status word (bits 8.. name the wait).
+ * device's kernel status word: FA_OK, or FA_ERR_DEVICE_TIMEOUT if a pipeline wait in a
+ * forward or backward kernel ran out of time.  FA_ERR_CUDA if the synchronisation itself
+ * failed.  If `detail` is not NULL it receives the raw status word (bits 8..15 name the
+ * wait: 1-12 forward, 21-34 backward; bits 16.. the CTA).
  */
 int fa_device_status(void *stream, int *detail);
 
