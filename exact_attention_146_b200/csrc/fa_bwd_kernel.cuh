@@ -1,7 +1,7 @@
 // fa_bwd_kernel.cuh -- exact attention backward for sm_100a (tcgen05 + TMEM + TMA).
 //
 // The backward pass recomputes S and P from Q, K, V instead of storing them: the
-// kaiwu.csdn.net page on the FlashAttention principle (section 2.3) and the
+// lpnh.cn YOLO11 / FlashAttention-2 article (section 2.3, "reverse recomputation") and the
 // hwcomputing.csdn.net article "FlashAttention in CANN ops-transformer" ("performance
 // tuning") describe it; with the forward's log-sum-exp L_i, P_ij = exp(scale S_ij - L_i)
 // exactly, so nothing but L (and D_i = dO_i . O_i) has to be kept from the forward.  The

@@ -185,7 +185,7 @@ int fa_fwd_splitkv_static(const void *q, const void *k, const void *v, void *out
 /*
  * fa_bwd -- exact attention backward: the gradients dQ, dK, dV of L = sum O (.) dO, with
  * S and P recomputed from Q, K, V and the forward's LSE instead of being stored (the
- * kaiwu.csdn.net FlashAttention principle page, section 2.3; the hwcomputing.csdn.net
+ * lpnh.cn YOLO11 / FlashAttention-2 article, section 2.3 "reverse recomputation"; the hwcomputing.csdn.net
  * FlashAttention article, "performance tuning"):
  *
  *     P = exp(scale Q K^T - LSE)  (masked),   dV = P^T dO,   dP = dO V^T,
@@ -230,7 +230,9 @@ int fa_bwd_window(const void *q, const void *k, const void *v, const void *out, 
  * Q, computes the partial (O_r, LSE_r) of its shard, the partials are exchanged (one
  * all-gather), and every GPU merges them with the log-sum-exp identity of the split-KV
  * forward (LSE = ln sum_r exp(LSE_r), O = sum_r exp(LSE_r - LSE) O_r).  The pages promise
- * sequence-dimension parallelism (the kaiwu.csdn.net FlashAttention page, FA-2 section);
+ * sequence-dimension parallelism (the yunthe.com attention-variants page, closing paragraph of
+ * its section "Flash Attention IO optimisation principle and code practice", on FlashAttention-2
+ * parallelising over the sequence dimension; the lpnh.cn article, section 2.4, on FA-2's grid);
  * the exchange is the caller's (e.g. an NCCL all-gather of o_part and lse_part).
  *
  * fa_fwd_partial: q [B, Nq, Hq, d] bf16; k, v [B, Nk, Hkv, d] bf16 (the shard); o_part

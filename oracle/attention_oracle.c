@@ -47,8 +47,8 @@
  *
  * The backward pass (oracle_attention_bwd) is the gradient of L = sum O (.) dO through
  * the same definition: the pages ask for it by recomputation from Q, K, V (hwcomputing
- * article, "performance tuning"; kaiwu.csdn.net page on the FlashAttention principle,
- * section 2.3 on recomputing S and P in the backward pass).  With P the probability
+ * article, "performance tuning"; the lpnh.cn YOLO11 / FlashAttention-2 article,
+ * section 2.3 "reverse recomputation", on recomputing S and P in the backward pass).  With P the probability
  * matrix of the forward, the chain rule through O = P V and the row softmax gives
  *     dV = P^T dO,  dP = dO V^T,  dS_ij = P_ij (dP_ij - sum_k P_ik dP_ik),
  *     dQ = scale dS K,  dK = scale dS^T Q,
