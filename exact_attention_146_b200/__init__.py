@@ -17,7 +17,8 @@ from pathlib import Path
 
 __all__ = ["fa_fwd", "fa_fwd_fp8", "fa_fwd_partial", "fa_merge_partials", "fa_bwd", "fa_fwd_raw",
            "splitkv_workspace_bytes", "splitkv_default_splits", "bwd_workspace_bytes", "device_status",
-           "tile_config", "status_string", "FaError", "lib", "SUPPORTED_HEAD_DIMS", "BWD_HEAD_DIMS", "LIB_PATH"]
+           "tile_config", "status_string", "FaError", "lib", "SUPPORTED_HEAD_DIMS", "BWD_HEAD_DIMS", "LIB_PATH",
+           "withheld_load_forward"]
 
 LIB_PATH = Path(__file__).resolve().parent / "libfa.so"
 SUPPORTED_HEAD_DIMS = (32, 64, 80, 96, 128, 192, 256)   # forward
@@ -36,7 +37,8 @@ FA_ERR_SCRATCH_LIMIT = 9
 SPLITKV_STATIC_SCRATCH_BYTES = 16 * 1024 * 1024
 
 EXPORTED = ("fa_fwd", "fa_fwd_window", "fa_fwd_splitkv", "fa_splitkv_workspace_bytes", "fa_splitkv_default_splits",
-            "fa_fwd_splitkv_static", "fa_fwd_f16", "fa_fwd_fp8", "fa_fwd_partial", "fa_merge_partials", "fa_bwd", "fa_bwd_f16", "fa_bwd_window", "fa_bwd_workspace_bytes", "fa_status_string", "fa_device_status", "fa_tile_config", "fa_version")
+            "fa_fwd_splitkv_static", "fa_fwd_f16", "fa_fwd_fp8", "fa_fwd_partial", "fa_merge_partials", "fa_bwd", "fa_bwd_f16", "fa_bwd_window", "fa_bwd_workspace_bytes", "fa_status_string", "fa_device_status", "fa_tile_config", "fa_version",
+            "fa_test_withheld_load")
 
 
 class FaError(RuntimeError):
@@ -86,6 +88,8 @@ def lib() -> ctypes.CDLL:
         L.fa_bwd_workspace_bytes.restype = ctypes.c_size_t
         L.fa_status_string.argtypes = [ci]
         L.fa_status_string.restype = ctypes.c_char_p
+        L.fa_test_withheld_load.argtypes = [vp, vp, vp, vp, vp, ci, ci, ci, ci, ci, cf, ci, ci, ctypes.c_uint, vp]
+        L.fa_test_withheld_load.restype = ci
         L.fa_device_status.argtypes = [vp, ctypes.POINTER(ci)]
         L.fa_device_status.restype = ci
         L.fa_tile_config.argtypes = [ci] + [ctypes.POINTER(ci)] * 4
@@ -303,6 +307,28 @@ def fa_bwd(q, k, v, out, dout, lse, *, causal: bool = False, scale: float | None
     if rc != FA_OK:
         raise FaError(rc, "fa_bwd")
     return dq, dk, dv
+
+
+def withheld_load_forward(q, k, v, withheld_load: int, wait_limit_us: int, *, causal: bool = False,
+                          scale: float | None = None, out=None, lse=None, stream=None):
+    """Failure-path test (fa_test_withheld_load): the d = 64 bf16 forward in a build whose
+    waits give up after wait_limit_us and whose producer leaves out K/V load number
+    `withheld_load`; the timeout is then reported by device_status().  Outputs undefined."""
+    import torch
+    B, Nq, Hq, d = q.shape
+    Nk, Hkv = k.shape[1], k.shape[2]
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, Hq, Nq), dtype=torch.float32, device=q.device)
+    rc = lib().fa_test_withheld_load(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
+                                     B, Hq, Hkv, Nq, Nk, float(scale), 1 if causal else 0, int(withheld_load),
+                                     int(wait_limit_us), _stream_handle(stream))
+    if rc != FA_OK:
+        raise FaError(rc, "fa_test_withheld_load")
+    return out, lse
 
 
 def device_status(stream=None) -> tuple[int, int]:

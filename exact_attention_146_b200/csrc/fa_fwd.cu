@@ -164,6 +164,9 @@ template <bool H> using Cfg192 = TileCfg<192, 64, 2, 4, 1, 1, false, 0, H>;
 template <bool H> using Cfg256 = TileCfg<256, 64, 1, 4, 1, 2, false, 0, H>;
 // FP8 (E4M3) inputs, d = 128: 16 KB tiles, so eight K/V slots
 using Cfg128F8 = TileCfg<128, 128, 2, 8, 1, 1, false, 0, false, true>;
+// The d = 64 bf16 tiling built for the failure-path test (fa_test_withheld_load): wait limit
+// taken from the parameters, one K/V load left out by the producer.
+using Cfg64Fault = TileCfg<64, 128, 2, 8, 2, 1, true, 2, false, false, true>;
 struct Problem {
     const void *q, *k, *v;
     void *out;
@@ -178,6 +181,8 @@ struct Problem {
     float o_scale;      // FP8: V dequantisation factor (1 otherwise)
     int diag;           // causal diagonal offset (Nk - Nq unless a key shard)
     int partial;        // write the shard partial (fp32 O, LSE) to o_part / lse_part
+    unsigned long long wait_limit_ns = kWaitLimitNs;   // failure-path test build only
+    int withheld_load = -1;                              // failure-path test build only
 };
 
 // Workspace layout of the split-KV forward: partial O, then (256-byte aligned) partial LSE.
@@ -256,6 +261,8 @@ int launch(const Problem &pr, DeviceState &dev, int cfg_slot, cudaStream_t strea
     p.o_scale = pr.o_scale;
     p.diag = pr.diag;
     p.partial = pr.partial;
+    p.wait_limit_ns = pr.wait_limit_ns;
+    p.withheld_load = pr.withheld_load;
 
     const int grid = int(units < dev.num_sms ? units : dev.num_sms);
     fa_fwd_kernel<C><<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(mq, mk, mv, p);
@@ -346,9 +353,17 @@ namespace {
 // (1, W >= 1).
 // `library_scratch`: the workspace is the library's own static scratch (already known to be
 // device memory of the current device), so its device-range check is skipped.
+// `fault`: run the failure-path test build instead (d = 64, bf16): {wait limit in ns, index of
+// the withheld K/V load}.
+struct FaultHook {
+    unsigned long long wait_limit_ns;
+    int withheld_load;
+};
+
 int forward(const void *q, const void *k, const void *v, void *out, float *lse, int B, int Hq, int Hkv,
             int Nq, int Nk, int d, float scale, int causal, int window, int num_splits, void *workspace,
-            size_t workspace_bytes, void *stream, bool library_scratch = false, int elem = 0, float o_scale = 1.f) {
+            size_t workspace_bytes, void *stream, bool library_scratch = false, int elem = 0, float o_scale = 1.f,
+            const FaultHook *fault = nullptr) {
     // ---- host-only validation (no CUDA call before this block passes)
     if (B < 0 || Hq <= 0 || Hkv <= 0 || Nq < 0 || Nk < 0) return FA_ERR_INVALID_ARG;
     if (Hq % Hkv != 0) return FA_ERR_INVALID_ARG;
@@ -417,6 +432,13 @@ int forward(const void *q, const void *k, const void *v, void *out, float *lse, 
     }
     const Problem pr{q, k, v, out, lse, B, Hq, Hkv, Nq, Nk, d, scale, causal, window,
                      ws_bytes > 0 ? num_splits : 1, o_part, lse_part, o_scale, Nk - Nq, 0};
+    if (fault != nullptr) {
+        if (d != 64 || elem != 0 || ws_bytes > 0) return FA_ERR_UNSUPPORTED_HEAD_DIM;
+        Problem pf = pr;
+        pf.wait_limit_ns = fault->wait_limit_ns;
+        pf.withheld_load = fault->withheld_load;
+        return launch<Cfg64Fault>(pf, *dev, kFaultSlot, st);
+    }
     if (elem == 2) return launch<Cfg128F8>(pr, *dev, kFp8Slot, st);
     return elem == 1 ? dispatch<true>(pr, *dev, st) : dispatch<false>(pr, *dev, st);
 }
@@ -536,6 +558,15 @@ int fa_fwd_window(const void *q, const void *k, const void *v, void *out, float 
                   int Hkv, int Nq, int Nk, int d, float scale, int window, void *stream) {
     if (window < 1) return FA_ERR_INVALID_ARG;
     return forward(q, k, v, out, lse, B, Hq, Hkv, Nq, Nk, d, scale, 1, window, 1, nullptr, 0, stream);
+}
+
+int fa_test_withheld_load(const void *q, const void *k, const void *v, void *out, float *lse, int B, int Hq,
+                          int Hkv, int Nq, int Nk, float scale, int causal, int withheld_load,
+                          unsigned int wait_limit_us, void *stream) {
+    if (withheld_load < 0 || wait_limit_us < 1u || wait_limit_us > 1000000u) return FA_ERR_INVALID_ARG;
+    const FaultHook hook{1000ull * wait_limit_us, withheld_load};
+    return forward(q, k, v, out, lse, B, Hq, Hkv, Nq, Nk, 64, scale, causal, 0, 1, nullptr, 0, stream, false, 0, 1.f,
+                   &hook);
 }
 
 int fa_device_status(void *stream, int *detail) {

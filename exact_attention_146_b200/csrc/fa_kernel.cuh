@@ -74,11 +74,16 @@ struct FwdParams {
                           // shard at offset o of Nk_total keys, Nk_total - Nq - o)
     int partial;          // 1: write the fp32 normalised O and the LSE of these keys to
                           // o_part / lse_part (a key shard's partial) instead of out / lse
+    // Failure-path test instantiation only (TileCfg FAULT): the per-wait limit, and the index
+    // (in issue order K_0, V_0, K_1, ...) of one K/V load the producer leaves out, so the wait
+    // for it runs out and the kernel takes its timeout path.  Ignored by every other build.
+    unsigned long long wait_limit_ns;
+    int withheld_load;
 };
 
 // Compile-time tiling for one head dimension.
 template <int D_, int BC_, int NQT_, int NS_, int NQB_ = 1, int SB_ = 1, bool PSEP_ = false, int SOFT_EXP_ = 0,
-          bool F16_ = false, bool FP8_ = false>
+          bool F16_ = false, bool FP8_ = false, bool FAULT_ = false>
 struct TileCfg {
     static constexpr int D = D_;        // head dim
     static constexpr int BC = BC_;      // key/value rows per tile
@@ -90,6 +95,8 @@ struct TileCfg {
     static constexpr int SOFT_EXP = SOFT_EXP_;   // exponentials on the FMA pipe: pairs per 8
     static constexpr bool F16 = F16_;   // element type of Q, K, V, P and O: fp16, else bf16
     static constexpr bool FP8 = FP8_;   // Q, K, V and P in OCP E4M3 (kind::f8f6f4); O stays bf16
+    static constexpr bool FAULT = FAULT_;   // failure-path test build: wait limit from the
+                                            // parameters, one K/V load withheld
     static constexpr int ES = FP8 ? 1 : 2;                // bytes per Q/K/V/P element
     static constexpr int RB = (D * ES >= 128) ? 128 : 64; // bytes per swizzled smem row
     static constexpr int CW = RB / ES;                    // elements per swizzled smem row
@@ -239,6 +246,7 @@ __device__ __forceinline__ UnitInfo decode_unit(int u, const FwdParams &p) {
 struct Ctl {
     volatile int *abort_flag;
     int *status;
+    uint64_t limit_ns;   // per-wait limit (kWaitLimitNs outside the failure-path test build)
 };
 
 // Poll `bar` until the phase of parity `parity` completes.  Gives up when another role
@@ -266,10 +274,9 @@ __device__ __forceinline__ bool wait_slow(uint32_t bar, uint32_t parity, Ctl ctl
 constexpr int kRoleSoftmax = 0, kRoleControl = 1;
 
 template <int ROLE = kRoleControl>
-__device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, const Ctl &ctl, int site,
-                                         uint64_t limit_ns = kWaitLimitNs) {
+__device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, const Ctl &ctl, int site) {
     if (sm100::mbar_try_wait(bar, parity)) return true;
-    return wait_slow<ROLE>(bar, parity, ctl, site, limit_ns);
+    return wait_slow<ROLE>(bar, parity, ctl, site, ctl.limit_ns);
 }
 
 // Warp-uniform wait: every lane polls, the warp proceeds only if all lanes saw it.
@@ -317,6 +324,12 @@ __device__ void producer_role(const CUtensorMap *tm_q, const CUtensorMap *tm_k, 
 #pragma unroll
             for (int which = 0; which < 2; ++which) {
                 const int s = int(kv_cnt % C::NS);
+                if constexpr (C::FAULT) {
+                    if (kv_cnt == uint32_t(p.withheld_load)) {   // left out: nothing will fill this slot
+                        ++kv_cnt;
+                        continue;
+                    }
+                }
                 if (!warp_wait_bar<kRoleControl>(bar(C::B_EMPTY + s), ((kv_cnt / C::NS) & 1u) ^ 1u, ctl, kSiteKvEmpty)) { ok = false; break; }
                 const uint32_t fb = bar(C::B_FULL + s);
                 sm100::mbar_arrive_expect_tx_elected(fb, C::KV_TILE);
@@ -329,19 +342,20 @@ __device__ void producer_role(const CUtensorMap *tm_q, const CUtensorMap *tm_k, 
             }
         }
     }
-    if (!ok) {
-        // Unwinding after a timeout: let this thread's copies still in flight land
-        // before the CTA exits (the last load issued into each slot, and each Q tile).
+    if (!ok || *ctl.abort_flag) {
+        // Unwinding after a timeout (here or in another role): let this thread's copies
+        // still in flight land before the CTA exits (the last load issued into each slot,
+        // and each Q tile).
         const uint32_t first = kv_cnt > uint32_t(C::NS) ? kv_cnt - C::NS : 0u;
         for (uint32_t n = first; n < kv_cnt; ++n)
             wait_slow<kRoleControl>(bar(C::B_FULL + int(n % C::NS)), (n / C::NS) & 1u, ctl, kSiteProducerDrain,
-                      kWaitLimitNs / 10, true);
+                      ctl.limit_ns / 10, true);
 #pragma unroll
         for (int t = 0; t < C::NQT; ++t) {
             const uint32_t first_q = qcnt[t] > uint32_t(C::NQB) ? qcnt[t] - C::NQB : 0u;
             for (uint32_t n = first_q; n < qcnt[t]; ++n)
                 wait_slow<kRoleControl>(bar(C::B_QFULL + t * C::NQB + int(n % C::NQB)), (n / C::NQB) & 1u, ctl,
-                          kSiteProducerDrain, kWaitLimitNs / 10, true);
+                          kSiteProducerDrain, ctl.limit_ns / 10, true);
         }
     }
 }
@@ -533,7 +547,7 @@ __device__ void mma_role(const FwdParams &p, uint32_t sbase, uint32_t tmem, cons
     }
     // Every MMA this thread issued is complete before the CTA may free TMEM.
     sm100::tc_commit_elected(bar(C::B_DRAIN));
-    wait_slow<kRoleControl>(bar(C::B_DRAIN), 0u, ctl, kSiteDrain, kWaitLimitNs, true);
+    wait_slow<kRoleControl>(bar(C::B_DRAIN), 0u, ctl, kSiteDrain, ctl.limit_ns, true);
 }
 
 // ------------------------------------------------------------------ softmax / epilogue
@@ -814,7 +828,7 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     const int lane = int(threadIdx.x) % 32;
     uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(smem + C::SMEM_MISC);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + C::SMEM_MISC + 4);
-    const Ctl ctl{abort_flag, p.status};
+    const Ctl ctl{abort_flag, p.status, C::FAULT ? uint64_t(p.wait_limit_ns) : kWaitLimitNs};
 
     if (threadIdx.x == 0) {
         auto bar = [&](int i) { return sbase + C::SMEM_BAR + 8u * uint32_t(i); };

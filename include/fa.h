@@ -251,6 +251,23 @@ int fa_merge_partials(const float *o_parts, const float *lse_parts, int R, void 
                       int B, int Hq, int Nq, int d, void *stream);
 
 /* Human-readable text of a status code (static storage; never NULL). */
+/*
+ * fa_test_withheld_load -- the failure path of the forward kernel, for tests (no counterpart
+ * on the pages: it exercises this library's own bounded waits).  Runs the d = 64 bf16 forward
+ * (arguments, layouts and checks as fa_fwd with d = 64) in a build whose pipeline waits give
+ * up after wait_limit_us microseconds (1 .. 1000000) and whose TMA producer leaves out one
+ * K/V tile load: number `withheld_load` (>= 0) of its CTA, counted in issue order K_0, V_0,
+ * K_1, V_1, ...  Nothing ever fills that slot, so the consumer's wait for it runs out: the
+ * kernel records FA_ERR_DEVICE_TIMEOUT in the status word, every role unwinds (the producer
+ * waits for its copies in flight, the MMA thread for its MMAs, TMEM is freed) and the kernel
+ * returns.  fa_device_status then reports it; out and lse are undefined.  A later call runs
+ * normally.  If the withheld load is past the last load a CTA issues, the call is an ordinary
+ * forward.  Returns FA_ERR_INVALID_ARG for a negative index or a limit out of range.
+ */
+int fa_test_withheld_load(const void *q, const void *k, const void *v, void *out, float *lse,
+                          int B, int Hq, int Hkv, int Nq, int Nk, float scale, int causal,
+                          int withheld_load, unsigned int wait_limit_us, void *stream);
+
 const char *fa_status_string(int status);
 
 /*

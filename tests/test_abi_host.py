@@ -195,6 +195,18 @@ def test_partial_and_merge_validation(L):
     assert merge() in (fa.FA_ERR_UNSUPPORTED_DEVICE, fa.FA_ERR_NOT_DEVICE_MEMORY)
 
 
+def test_withheld_load_validation(L):
+    """The failure-path test entry: index >= 0, limit in 1 .. 10^6 us, then fa_fwd's checks."""
+    def call(load=1, limit=20000, scale=0.125):
+        return L.fa_test_withheld_load(FAKE, FAKE + (1 << 30), FAKE + (2 << 30), FAKE + (3 << 30), FAKE + (4 << 30),
+                                       1, 1, 1, 256, 256, scale, 0, load, limit, None)
+    assert call(load=-1) == fa.FA_ERR_INVALID_ARG
+    assert call(limit=0) == fa.FA_ERR_INVALID_ARG
+    assert call(limit=2000000) == fa.FA_ERR_INVALID_ARG
+    assert call(scale=-1.0) == fa.FA_ERR_INVALID_ARG
+    assert call() in (fa.FA_ERR_UNSUPPORTED_DEVICE, fa.FA_ERR_NOT_DEVICE_MEMORY)
+
+
 def test_f16_entry_validates_like_bf16(L):
     args = (FAKE, FAKE + (1 << 30), FAKE + (2 << 30), FAKE + (3 << 30), FAKE + (4 << 30), 1, 2, 1, 64, 64)
     assert L.fa_fwd_f16(*args, 48, 0.125, 0, None) == fa.FA_ERR_UNSUPPORTED_HEAD_DIM
