@@ -74,3 +74,38 @@ def test_empty_shard_is_neutral(orc):
     assert torch.isneginf(l_all[1]).all() and (o_all[1] == 0).all()
     Oref, Lref = orc.forward(x["q"], x["k"], x["v"], 0.125, False)
     _parity.compare(_parity.bf16_to_f64(out), lse.cpu().numpy().astype(np.float64), Oref, Lref, "empty shard")
+
+
+@pytest.mark.parametrize("R", [2, 3])
+def test_row_block_exchange_layout(orc, R):
+    """The all-to-all by query rows, emulated on one GPU: each of R shards' partials is cut
+    by destination (kshard.send_blocks), every destination stacks what it would receive
+    (kshard.received_layout) and merges only its rows; the rows, put back in order, equal
+    the oracle's forward over all keys."""
+    import torch
+    import exact_attention_146_b200 as fa
+    B, Hq, Hkv, Nq, Nk, d = 2, 4, 2, 301, 900, 128
+    w = synth.Workload("ksrows", 5950 + R, B, Hq, Hkv, Nq, Nk, d, False, seed=R)
+    x = synth.make_inputs(w)
+    q, k, v = (_parity.to_device(x[n], torch) for n in ("q", "k", "v"))
+    scale = 1.0 / math.sqrt(d)
+    sends = []
+    for r in range(R):
+        off, n = kshard.shard_range(Nk, r, R)
+        o_p, l_p = fa.fa_fwd_partial(q, k[:, off:off + n].contiguous(), v[:, off:off + n].contiguous(),
+                                     key_offset=off, nk_total=Nk, causal=True, scale=scale)
+        sends.append(kshard.send_blocks(o_p, l_p, R))
+    outs, lses = [], []
+    for s in range(R):
+        row0, n = kshard.shard_range(B * Nq, s, R)
+        o_recv = torch.cat([o_send[row0:row0 + n] for o_send, _, _ in sends])
+        l_recv = torch.cat([l_send[row0:row0 + n] for _, l_send, _ in sends])
+        o_parts, l_parts = kshard.received_layout(o_recv, l_recv, R, n, Hq, d)
+        o_rows, l_rows = fa.fa_merge_partials(o_parts, l_parts)
+        outs.append(o_rows.reshape(n, Hq, d))
+        lses.append(l_rows.reshape(Hq, n).t())
+    out = torch.cat(outs).view(B, Nq, Hq, d)
+    lse = torch.cat(lses).view(B, Nq, Hq).permute(0, 2, 1).contiguous()
+    assert fa.device_status()[0] == fa.FA_OK
+    Oref, Lref = orc.forward(x["q"], x["k"], x["v"], scale, True)
+    _parity.compare(_parity.bf16_to_f64(out), lse.cpu().numpy().astype(np.float64), Oref, Lref, f"rows R={R}")
