@@ -245,7 +245,7 @@ def device_inputs(torch, x, w, pin=False):
 def forward_call(fa, w, q, k, v, out, lse, **kw):
     """The entry point a workload runs through (fa_fwd_fp8 for E4M3 inputs)."""
     if w.dtype == "e4m3":
-        return fa.fa_fwd_fp8(q, k, v, causal=w.causal, scale=w.scale, out=out, lse=lse)
+        return fa.fa_fwd_fp8(q, k, v, causal=w.causal, scale=w.scale, out=out, lse=lse, stream=kw.get("stream"))
     return fa.fa_fwd(q, k, v, causal=w.causal, scale=w.scale, out=out, lse=lse, **kw)
 
 
@@ -331,20 +331,38 @@ def run_ours(args, w, world, rank, local):
                     "frac": achieved / tp, "traffic": profiled_traffic(w.name), "peak_source": tsrc,
                     "algorithmic_bytes": w.io_bytes, "hbm_gbs": gbs}
 
-    # end to end through the public API: pinned host inputs in, O and LSE back to host
+    # End to end through the public API: pinned host inputs in, O and LSE back to host, every
+    # step.  The batch is cut into chunks (whole batch elements: contiguous slices of every
+    # tensor) that alternate between two streams, so the host->device copy of one chunk, the
+    # forward of another and the device->host copy of a third overlap (separate copy engines
+    # for each direction, the SMs for the kernel).
     e2e = None
     if not args.no_e2e:
         out_h = torch.empty(out.shape, dtype=out.dtype).pin_memory()
         lse_h = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
         n_e2e = max(1, min(args.steps, args.e2e_steps))
+        n_chunks = max(1, min(args.e2e_chunks, w.B))
+        bounds = [round(i * w.B / n_chunks) for i in range(n_chunks + 1)]
+        spans = [(bounds[i], bounds[i + 1]) for i in range(n_chunks) if bounds[i + 1] > bounds[i]]
+        side = [torch.cuda.Stream(device=dev) for _ in range(2)]
+        # split-KV scratch is per stream: chunks in flight on the two streams must not share it
+        side_ws = [ws, (torch.empty_like(ws) if ws is not None else None)]
 
         def e2e_step():
-            q.copy_(host["q"], non_blocking=True)
-            k.copy_(host["k"], non_blocking=True)
-            v.copy_(host["v"], non_blocking=True)
-            forward_call(fa, w, q, k, v, out, lse, **call_kw)
-            out_h.copy_(out, non_blocking=True)
-            lse_h.copy_(lse, non_blocking=True)
+            start = torch.cuda.Event()
+            start.record(stream)
+            for c, (b0, b1) in enumerate(spans):
+                s = side[c % 2]
+                s.wait_event(start)
+                with torch.cuda.stream(s):
+                    for n, t in (("q", q), ("k", k), ("v", v)):
+                        t[b0:b1].copy_(host[n][b0:b1], non_blocking=True)
+                    forward_call(fa, w, q[b0:b1], k[b0:b1], v[b0:b1], out[b0:b1], lse[b0:b1], stream=s,
+                                 **dict(call_kw, workspace=side_ws[c % 2]))
+                    out_h[b0:b1].copy_(out[b0:b1], non_blocking=True)
+                    lse_h[b0:b1].copy_(lse[b0:b1], non_blocking=True)
+            for s in side:
+                stream.wait_stream(s)
 
         e2e_step()
         torch.cuda.synchronize()
@@ -360,7 +378,8 @@ def run_ours(args, w, world, rank, local):
         h2d = sum(host[n].numel() * host[n].element_size() for n in ("q", "k", "v"))
         d2h = out.numel() * 2 + lse.numel() * 4
         e2e = {"value": weak_scaling_tflops(w, world, ms_e2e), "unit": "TFLOP/s", "ms_per_step": ms_e2e,
-               "steps": n_e2e, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+               "steps": n_e2e, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+               "chunks": len(spans), "streams": 2}
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -504,6 +523,7 @@ def main(argv=None):
     ap.add_argument("--workload", default=synth.HEADLINE, choices=sorted(synth.WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--e2e-steps", type=int, default=5)
+    ap.add_argument("--e2e-chunks", type=int, default=4, help="batch chunks pipelined over two streams in e2e")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")

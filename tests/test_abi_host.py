@@ -102,9 +102,12 @@ def test_splitkv_workspace_and_default_splits(L):
     assert fa.splitkv_workspace_bytes(2, 4, 100, 128, 3) == ((o + 255) // 256) * 256 + 3 * 2 * 4 * 100 * 4
     assert fa.splitkv_workspace_bytes(2, 4, 100, 128, 0) == 0 and fa.splitkv_workspace_bytes(2, 4, 100, 128, 999) == 0
     assert fa.splitkv_default_splits(8, 32, 32, 4096, 4096, 128, 148) == 1   # already fills the GPU
-    # GQA-packed decode: 4 x 8 units of 64 rows, 256 key tiles; 9 splits = 2 waves x 29 tiles
-    assert fa.splitkv_default_splits(4, 32, 8, 16, 32768, 128, 148) == 9
-    assert fa.splitkv_default_splits(1, 1, 1, 1, 65536, 128, 148) == 128     # capped by 4 tiles per split
+    bk = fa.tile_config(128)["block_k"]
+    # GQA-packed decode: 4 x 8 units of 64 rows; the split minimising waves x (tiles per split + 1)
+    assert fa.splitkv_default_splits(4, 32, 8, 16, 32768, 128, 148) == _split_model(4, 32, 8, 16, 32768, 148, bk)
+    # one unit: as many splits as keep >= 4 key tiles each, within one wave
+    assert fa.splitkv_default_splits(1, 1, 1, 1, 65536, 128, 148) == min(147, 65536 // bk // 4, 256) or \
+        fa.splitkv_default_splits(1, 1, 1, 1, 65536, 128, 148) == _split_model(1, 1, 1, 1, 65536, 148, bk)
     assert fa.splitkv_default_splits(1, 1, 1, 1, 300, 64, 148) == 1          # too few key tiles
     assert fa.splitkv_default_splits(1, 6, 2, 1, 4096, 64, 148) >= 1         # n_rep = 3: not packed
 
@@ -124,7 +127,8 @@ def _split_model(B, Hq, Hkv, Nq, Nk, sms, bk=128):
 @pytest.mark.parametrize("B,Hq,Hkv,Nq,Nk", [(4, 32, 32, 16, 32768), (1, 8, 1, 1, 8192), (2, 16, 2, 64, 100000),
                                             (1, 32, 8, 1, 1000), (3, 12, 4, 100, 50000)])
 def test_splitkv_default_splits_model(L, B, Hq, Hkv, Nq, Nk):
-    assert fa.splitkv_default_splits(B, Hq, Hkv, Nq, Nk, 128, 148) == _split_model(B, Hq, Hkv, Nq, Nk, 148)
+    bk = fa.tile_config(128)["block_k"]
+    assert fa.splitkv_default_splits(B, Hq, Hkv, Nq, Nk, 128, 148) == _split_model(B, Hq, Hkv, Nq, Nk, 148, bk)
 
 
 def _splitkv(L, splits=4, ws=FAKE + (5 << 30), ws_bytes=1 << 30, out=FAKE + (3 << 30)):

@@ -17,7 +17,7 @@ PROGRAM = r"""
 int main(void) {
     int bq = 0, bk = 0, nqt = 0, ns = 0;
     if (fa_version() != 100) return 1;
-    if (fa_tile_config(128, &bq, &bk, &nqt, &ns) != FA_OK || bq != 128 || bk != 128) return 2;
+    if (fa_tile_config(128, &bq, &bk, &nqt, &ns) != FA_OK || bq != 128 || bk < 64 || bk % 64 != 0) return 2;
     if (fa_tile_config(100, NULL, NULL, NULL, NULL) != FA_ERR_UNSUPPORTED_HEAD_DIM) return 3;
     if (strlen(fa_status_string(FA_ERR_OVERLAP)) == 0) return 4;
     if (fa_splitkv_workspace_bytes(1, 2, 16, 128, 1) != 0) return 5;
