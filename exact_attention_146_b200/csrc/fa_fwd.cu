@@ -234,6 +234,12 @@ int launch(const Problem &pr, DeviceState &dev, int cfg_slot, cudaStream_t strea
         return rc;
     if ((rc = encode_bnhd(&mk, pr.k, C::D, pr.Hkv, pr.Nk, pr.B, C::CW, C::BC, 1, elem)) != FA_OK) return rc;
     if ((rc = encode_bnhd(&mv, pr.v, C::D, pr.Hkv, pr.Nk, pr.B, C::CW, C::BC, 1, elem)) != FA_OK) return rc;
+    // O through shared memory and TMA stores: boxes of 64 columns x one warp's 32 flat rows
+    // (pack heads x 32 / pack queries); only for the bf16 / fp16 output of a plain forward
+    CUtensorMap mo = mq;
+    const bool o_tma = C::OSTAGE && pr.partial == 0 && pr.num_splits <= 1 && pack <= 32;
+    if (o_tma && (rc = encode_bnhd(&mo, pr.out, C::D, pr.Hq, pr.Nq, pr.B, 64, 32 / pack, pack, C::F16 ? 1 : 0)) != FA_OK)
+        return rc;
 
     FwdParams p{};
     p.out = pr.out;
@@ -263,9 +269,10 @@ int launch(const Problem &pr, DeviceState &dev, int cfg_slot, cudaStream_t strea
     p.partial = pr.partial;
     p.wait_limit_ns = pr.wait_limit_ns;
     p.withheld_load = pr.withheld_load;
+    p.o_tma = o_tma ? 1 : 0;
 
     const int grid = int(units < dev.num_sms ? units : dev.num_sms);
-    fa_fwd_kernel<C><<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(mq, mk, mv, p);
+    fa_fwd_kernel<C><<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(mq, mk, mv, mo, p);
     if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
     if (p.num_splits > 1 && !p.partial) {
         const long long rows = (long long)pr.B * pr.Nq * pr.Hq;

@@ -79,6 +79,7 @@ struct FwdParams {
     // for it runs out and the kernel takes its timeout path.  Ignored by every other build.
     unsigned long long wait_limit_ns;
     int withheld_load;
+    int o_tma;            // 1: the epilogue writes O through shared memory and TMA stores (tm_o)
 };
 
 // Compile-time tiling for one head dimension.
@@ -127,9 +128,15 @@ struct TileCfg {
     static constexpr int SMEM_BAR = SMEM_KV + NS * KV_TILE;
     static constexpr int NUM_BARS = 2 * NS + 2 * NQT * NQB + 4 * NQT * SB + 3 * NQT + 1;
     static constexpr int SMEM_MISC = SMEM_BAR + NUM_BARS * 8;
+    // Output staging (d = 64 .. 128): each softmax warp writes its 32 rows of O, 64 columns
+    // at a time, into 4 KB of its own (128-byte rows, 128-byte swizzle) and stores them with
+    // one TMA box, so the epilogue writes whole lines instead of one 16-byte piece per row.
+    static constexpr bool OSTAGE = (D >= 64 && D <= 128);
+    static constexpr int SMEM_OST = ((SMEM_MISC + 16 + 1023) / 1024) * 1024;
+    static constexpr int OST_BYTES = OSTAGE ? 32 * 128 : 0;   // per warp
     // Each CTA holds all 512 TMEM columns, so ask for enough shared memory that a
     // second CTA can never be resident on the same SM (it would only wait in alloc).
-    static constexpr int SMEM_NEEDED = SMEM_MISC + 16 + 1024;
+    static constexpr int SMEM_NEEDED = SMEM_OST + 4 * NQT * OST_BYTES + 1024;
     static constexpr int SMEM_BYTES = SMEM_NEEDED > 120 * 1024 ? SMEM_NEEDED : 120 * 1024;
     // warps: one warpgroup per query tile (softmax), then a control warpgroup holding the
     // TMA warp and the MMA warp (two warps of it idle: register reallocation works on
@@ -652,8 +659,8 @@ __device__ __forceinline__ float exp_pack_store(const uint32_t (&s)[BC], float c
 }
 
 template <class C>
-__device__ void softmax_role(const FwdParams &p, uint32_t sbase, uint32_t tmem, const Ctl &ctl,
-                             int warp, int lane) {
+__device__ void softmax_role(const FwdParams &p, const CUtensorMap *tm_o, uint32_t sbase, uint32_t tmem,
+                             const Ctl &ctl, int warp, int lane) {
     constexpr int BC = C::BC;
     auto bar = [&](int i) { return sbase + C::SMEM_BAR + 8u * uint32_t(i); };
     const int t = warp / 4;
@@ -782,6 +789,44 @@ __device__ void softmax_role(const FwdParams &p, uint32_t sbase, uint32_t tmem, 
             const bool split_mode = p.num_splits > 1 || p.partial;
             uint16_t *orow = static_cast<uint16_t *>(p.out) + row_off * C::D;
             float *prow = split_mode ? p.o_part + (size_t(w.split) * p.B * p.Nq * p.Hq + row_off) * C::D : nullptr;
+            if (C::OSTAGE && p.o_tma && !split_mode) {
+                // 64 columns per pass: this warp's 32 rows (lane = row) into its staging
+                // buffer as one 128-byte-swizzled TMA box (16-byte unit i of row r at unit
+                // i ^ (r % 8)), then one TMA store; rows past Nq and columns past d lie
+                // outside the tensor and are not written.
+                const uint32_t stage = sbase + uint32_t(C::SMEM_OST + warp * C::OST_BYTES);
+                const int row0 = (f_lo + quarter * 32) / p.pack;   // first query of the box
+#pragma unroll
+                for (int c2 = 0; c2 < (C::D + 63) / 64; ++c2) {
+                    uint32_t pk[32];
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        uint32_t o[32];
+                        if (nk > 0) {
+                            sm100::tmem_ld32_sync(o_taddr + uint32_t(64 * c2 + 32 * h), o);
+                        } else {
+#pragma unroll
+                            for (int i = 0; i < 32; ++i) o[i] = 0u;
+                        }
+#pragma unroll
+                        for (int i = 0; i < 16; ++i)
+                            pk[16 * h + i] = sm100::pack_x2<C::F16>(__uint_as_float(o[2 * i]) * inv_l,
+                                                                    __uint_as_float(o[2 * i + 1]) * inv_l);
+                    }
+#pragma unroll
+                    for (int u16 = 0; u16 < 8; ++u16)
+                        sm100::st_shared_v4(stage + uint32_t(lane * 128 + ((u16 ^ (lane & 7)) * 16)), pk[4 * u16],
+                                            pk[4 * u16 + 1], pk[4 * u16 + 2], pk[4 * u16 + 3]);
+                    sm100::fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0 && row0 < p.Nq) {   // (a box wholly past Nq has nothing to write)
+                        sm100::tma_store_4d(tm_o, stage, 64 * c2, w.hq, row0, w.b);
+                        sm100::bulk_commit_group();
+                        sm100::bulk_wait_group_read0();   // the staging buffer may be rewritten
+                    }
+                    __syncwarp();
+                }
+            } else {
 #pragma unroll
             for (int c = 0; c < C::O_CHUNKS; ++c) {
                 uint32_t o[32];
@@ -819,6 +864,7 @@ __device__ void softmax_role(const FwdParams &p, uint32_t sbase, uint32_t tmem, 
                     }
                 }
             }
+            }
             sm100::tc_fence_before_sync();
             sm100::mbar_arrive(bar(C::B_OEMPTY + t));
             const float lse_row = l > 0.f ? (m_ref + log2f(l)) * 0.6931471805599453f : -INFINITY;
@@ -832,6 +878,7 @@ __device__ void softmax_role(const FwdParams &p, uint32_t sbase, uint32_t tmem, 
     }
 unwind:
     sm100::tmem_st_wait();
+    if (C::OSTAGE && lane == 0) sm100::bulk_wait_group0();   // this warp's O stores are complete
 }
 
 // ------------------------------------------------------------------ kernel
@@ -839,7 +886,8 @@ unwind:
 template <class C>
 __global__ void __launch_bounds__(C::THREADS, 1)
 fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-              const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ FwdParams p) {
+              const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
+              const __grid_constant__ FwdParams p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const uint32_t sbase = sm100::smem_u32(smem);
@@ -885,7 +933,7 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
 
     if (warp < C::SOFTMAX_WARPS) {
         if constexpr (C::REALLOC_REGS) sm100::regs_increase<C::SOFTMAX_REGS>();
-        softmax_role<C>(p, sbase, tmem, ctl, warp, lane);
+        softmax_role<C>(p, &tm_o, sbase, tmem, ctl, warp, lane);
     } else {
         if constexpr (C::REALLOC_REGS) sm100::regs_decrease<C::CONTROL_REGS>();
         if (warp == C::TMA_WARP) {
