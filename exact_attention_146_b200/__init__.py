@@ -38,7 +38,7 @@ SPLITKV_STATIC_SCRATCH_BYTES = 16 * 1024 * 1024
 
 EXPORTED = ("fa_fwd", "fa_fwd_window", "fa_fwd_splitkv", "fa_splitkv_workspace_bytes", "fa_splitkv_default_splits",
             "fa_fwd_splitkv_static", "fa_fwd_f16", "fa_fwd_fp8", "fa_fwd_partial", "fa_merge_partials", "fa_bwd", "fa_bwd_f16", "fa_bwd_window", "fa_bwd_workspace_bytes", "fa_status_string", "fa_device_status", "fa_tile_config", "fa_version",
-            "fa_test_withheld_load")
+            "fa_test_withheld_load", "fa_fwd_window_f16", "fa_fwd_splitkv_f16")
 
 
 class FaError(RuntimeError):
@@ -69,6 +69,10 @@ def lib() -> ctypes.CDLL:
         L.fa_merge_partials.argtypes = [vp, vp, ci, vp, vp, ci, ci, ci, ci, vp]
         L.fa_merge_partials.restype = ci
         L.fa_fwd_window.argtypes = [vp, vp, vp, vp, vp, ci, ci, ci, ci, ci, ci, cf, ci, vp]
+        L.fa_fwd_window_f16.argtypes = [vp, vp, vp, vp, vp, ci, ci, ci, ci, ci, ci, cf, ci, vp]
+        L.fa_fwd_window_f16.restype = ci
+        L.fa_fwd_splitkv_f16.argtypes = [vp, vp, vp, vp, vp, ci, ci, ci, ci, ci, ci, cf, ci, ci, vp, ctypes.c_size_t, vp]
+        L.fa_fwd_splitkv_f16.restype = ci
         L.fa_fwd_window.restype = ci
         L.fa_fwd_splitkv.argtypes = [vp, vp, vp, vp, vp, ci, ci, ci, ci, ci, ci, cf, ci, ci, vp, ctypes.c_size_t, vp]
         L.fa_fwd_splitkv.restype = ci
@@ -169,24 +173,24 @@ def fa_fwd(q, k, v, *, causal: bool = False, scale: float | None = None, out=Non
     if not return_lse:
         lse = None
     lse_ptr = lse.data_ptr() if lse is not None else None
-    if dt == torch.float16:
-        if window is not None or (num_splits is not None and num_splits > 1):
-            raise ValueError("fp16 inputs take the causal or no mask, without split-KV")
-        rc = lib().fa_fwd_f16(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse_ptr,
-                              B, Hq, Hkv, Nq, Nk, d, float(scale), 1 if causal else 0, _stream_handle(stream))
-    elif num_splits is not None and num_splits > 1:
+    f16 = dt == torch.float16
+    if num_splits is not None and num_splits > 1:
         if window is not None:
             raise ValueError("split-KV takes the causal or no mask")
         need = splitkv_workspace_bytes(B, Hq, Nq, d, num_splits)
         if workspace is None:
             workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
-        rc = lib().fa_fwd_splitkv(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse_ptr,
-                                  B, Hq, Hkv, Nq, Nk, d, float(scale), 1 if causal else 0, int(num_splits),
-                                  workspace.data_ptr(), workspace.numel() * workspace.element_size(),
-                                  _stream_handle(stream))
+        entry = lib().fa_fwd_splitkv_f16 if f16 else lib().fa_fwd_splitkv
+        rc = entry(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse_ptr,
+                   B, Hq, Hkv, Nq, Nk, d, float(scale), 1 if causal else 0, int(num_splits),
+                   workspace.data_ptr(), workspace.numel() * workspace.element_size(), _stream_handle(stream))
     elif window is not None:
-        rc = lib().fa_fwd_window(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse_ptr,
-                                 B, Hq, Hkv, Nq, Nk, d, float(scale), int(window), _stream_handle(stream))
+        entry = lib().fa_fwd_window_f16 if f16 else lib().fa_fwd_window
+        rc = entry(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse_ptr,
+                   B, Hq, Hkv, Nq, Nk, d, float(scale), int(window), _stream_handle(stream))
+    elif f16:
+        rc = lib().fa_fwd_f16(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse_ptr,
+                              B, Hq, Hkv, Nq, Nk, d, float(scale), 1 if causal else 0, _stream_handle(stream))
     else:
         rc = fa_fwd_raw(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse_ptr,
                         B, Hq, Hkv, Nq, Nk, d, scale, 1 if causal else 0, _stream_handle(stream))

@@ -162,8 +162,12 @@ template <bool H> using Cfg96 = TileCfg<96, 128, 2, 4, 1, 1, false, 0, H>;
 template <bool H> using Cfg128 = TileCfg<128, 128, 2, 4, 1, 1, false, 0, H>;
 template <bool H> using Cfg192 = TileCfg<192, 64, 2, 4, 1, 1, false, 0, H>;
 template <bool H> using Cfg256 = TileCfg<256, 64, 1, 4, 1, 2, false, 0, H>;
-// FP8 (E4M3) inputs, d = 128: 16 KB tiles, so eight K/V slots
+// FP8 (E4M3) inputs.  d = 128: 16 KB tiles, so eight K/V slots; d = 64: 64-byte rows
+// (64-byte swizzle, 8 KB tiles); d = 256: one 128-row query tile with two S buffers (S 2 x 128
+// + O 256 TMEM columns), 32 KB tiles.  P is rounded to E4M3 over S (four per column).
 using Cfg128F8 = TileCfg<128, 128, 2, 8, 1, 1, false, 0, false, true>;
+using Cfg64F8 = TileCfg<64, 128, 2, 8, 1, 1, false, 0, false, true>;
+using Cfg256F8 = TileCfg<256, 128, 1, 4, 1, 2, false, 0, false, true>;
 // The d = 64 bf16 tiling built for the failure-path test (fa_test_withheld_load): wait limit
 // taken from the parameters, one K/V load left out by the producer.
 using Cfg64Fault = TileCfg<64, 128, 2, 8, 2, 1, true, 2, false, false, true>;
@@ -379,7 +383,7 @@ int forward(const void *q, const void *k, const void *v, void *out, float *lse, 
     if (num_splits < 1 || num_splits > kMaxSplits) return FA_ERR_INVALID_ARG;
     if (!std::isfinite(scale) || !(scale > 0.f)) return FA_ERR_INVALID_ARG;
     if (tile_config(d, nullptr, nullptr, nullptr, nullptr) != FA_OK) return FA_ERR_UNSUPPORTED_HEAD_DIM;
-    if (elem == 2 && d != 128) return FA_ERR_UNSUPPORTED_HEAD_DIM;
+    if (elem == 2 && d != 64 && d != 128 && d != 256) return FA_ERR_UNSUPPORTED_HEAD_DIM;
     if (!std::isfinite(o_scale) || !(o_scale > 0.f)) return FA_ERR_INVALID_ARG;
     const size_t es = elem == 2 ? 1 : 2;   // input element bytes; out is 2-byte
     const size_t q_bytes = size_t(B) * size_t(Nq) * size_t(Hq) * size_t(d) * es;
@@ -446,7 +450,11 @@ int forward(const void *q, const void *k, const void *v, void *out, float *lse, 
         pf.withheld_load = fault->withheld_load;
         return launch<Cfg64Fault>(pf, *dev, kFaultSlot, st);
     }
-    if (elem == 2) return launch<Cfg128F8>(pr, *dev, kFp8Slot, st);
+    if (elem == 2) {
+        if (d == 64) return launch<Cfg64F8>(pr, *dev, kFp8Slot64, st);
+        if (d == 256) return launch<Cfg256F8>(pr, *dev, kFp8Slot256, st);
+        return launch<Cfg128F8>(pr, *dev, kFp8Slot, st);
+    }
     return elem == 1 ? dispatch<true>(pr, *dev, st) : dispatch<false>(pr, *dev, st);
 }
 
@@ -565,6 +573,19 @@ int fa_fwd_window(const void *q, const void *k, const void *v, void *out, float 
                   int Hkv, int Nq, int Nk, int d, float scale, int window, void *stream) {
     if (window < 1) return FA_ERR_INVALID_ARG;
     return forward(q, k, v, out, lse, B, Hq, Hkv, Nq, Nk, d, scale, 1, window, 1, nullptr, 0, stream);
+}
+
+int fa_fwd_window_f16(const void *q, const void *k, const void *v, void *out, float *lse, int B, int Hq,
+                      int Hkv, int Nq, int Nk, int d, float scale, int window, void *stream) {
+    if (window < 1) return FA_ERR_INVALID_ARG;
+    return forward(q, k, v, out, lse, B, Hq, Hkv, Nq, Nk, d, scale, 1, window, 1, nullptr, 0, stream, false, 1);
+}
+
+int fa_fwd_splitkv_f16(const void *q, const void *k, const void *v, void *out, float *lse, int B, int Hq,
+                       int Hkv, int Nq, int Nk, int d, float scale, int causal, int num_splits, void *workspace,
+                       size_t workspace_bytes, void *stream) {
+    return forward(q, k, v, out, lse, B, Hq, Hkv, Nq, Nk, d, scale, causal, 0, num_splits, workspace,
+                   workspace_bytes, stream, false, 1);
 }
 
 int fa_test_withheld_load(const void *q, const void *k, const void *v, void *out, float *lse, int B, int Hq,

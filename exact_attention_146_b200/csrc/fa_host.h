@@ -12,11 +12,13 @@
 namespace fa_host {
 
 // Forward instantiations with per-device launch state: slots 0-6 bf16 and 8-14 fp16 (one per
-// head dim), 15 the FP8 one, 16 the failure-path test build.  (The backward keeps its own
-// state in fa_bwd.cu.)
-constexpr int kNumCfgSlots = 17;
+// head dim), 15, 17 and 18 the FP8 ones (d = 128, 64, 256), 16 the failure-path test build.
+// (The backward keeps its own state in fa_bwd.cu.)
+constexpr int kNumCfgSlots = 19;
 constexpr int kFp8Slot = 15;
 constexpr int kFaultSlot = 16;
+constexpr int kFp8Slot64 = 17;
+constexpr int kFp8Slot256 = 18;
 
 constexpr int kMaxDevices = 64;
 constexpr int kMaxSplits = 256;

@@ -102,7 +102,7 @@ int fa_fwd_f16(const void *q, const void *k, const void *v, void *out, float *ls
  * forward the datacanvas.csdn.net head-dim page attributes to FlashAttention-3.  The tensor
  * cores multiply E4M3 x E4M3 (kind::f8f6f4) with fp32 accumulation; P is rounded to E4M3
  * (relative error <= 2^-4) before P V; out is bf16 [B, Nq, Hq, d], lse fp32 as in fa_fwd
- * (the LSE of the dequantised logits).  d must be 128 (FA_ERR_UNSUPPORTED_HEAD_DIM
+ * (the LSE of the dequantised logits).  d must be 64, 128 or 256 (FA_ERR_UNSUPPORTED_HEAD_DIM
  * otherwise); the descales must be finite and > 0.  Layouts, ownership and the other
  * errors as fa_fwd (q, k, v one byte per element, 16-byte aligned).
  */
@@ -125,6 +125,12 @@ int fa_fwd_fp8(const void *q, const void *k, const void *v, void *out, float *ls
 int fa_fwd_window(const void *q, const void *k, const void *v, void *out, float *lse,
                   int B, int Hq, int Hkv, int Nq, int Nk, int d, float scale, int window,
                   void *stream);
+/* fa_fwd_window_f16: the same on IEEE fp16 q, k, v and out (P rounded to fp16), as fa_fwd_f16
+ * is to fa_fwd (the data-type option of the hwcomputing.csdn.net article's "performance
+ * tuning" is independent of the mask mode). */
+int fa_fwd_window_f16(const void *q, const void *k, const void *v, void *out, float *lse,
+                      int B, int Hq, int Hkv, int Nq, int Nk, int d, float scale, int window,
+                      void *stream);
 
 /*
  * Split-KV forward, for shapes with too few (batch, head, query block) units to fill the
@@ -156,6 +162,10 @@ int fa_splitkv_default_splits(int B, int Hq, int Hkv, int Nq, int Nk, int d, int
 int fa_fwd_splitkv(const void *q, const void *k, const void *v, void *out, float *lse,
                    int B, int Hq, int Hkv, int Nq, int Nk, int d, float scale, int causal,
                    int num_splits, void *workspace, size_t workspace_bytes, void *stream);
+/* fa_fwd_splitkv_f16: the same on fp16 q, k, v and out (the merge writes fp16). */
+int fa_fwd_splitkv_f16(const void *q, const void *k, const void *v, void *out, float *lse,
+                       int B, int Hq, int Hkv, int Nq, int Nk, int d, float scale, int causal,
+                       int num_splits, void *workspace, size_t workspace_bytes, void *stream);
 
 /*
  * fa_fwd_splitkv_static -- fa_fwd_splitkv without a caller workspace and without any

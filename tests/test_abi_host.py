@@ -172,7 +172,9 @@ def test_fp8_validation(L):
     def call(d=128, ds=(1.0, 1.0, 1.0)):
         return L.fa_fwd_fp8(FAKE, FAKE + (1 << 30), FAKE + (2 << 30), FAKE + (3 << 30), FAKE + (4 << 30),
                             1, 2, 1, 64, 64, d, 0.125, ds[0], ds[1], ds[2], 0, None)
-    assert call(d=64) == fa.FA_ERR_UNSUPPORTED_HEAD_DIM
+    assert call(d=80) == fa.FA_ERR_UNSUPPORTED_HEAD_DIM and call(d=96) == fa.FA_ERR_UNSUPPORTED_HEAD_DIM
+    assert call(d=64) in (fa.FA_ERR_UNSUPPORTED_DEVICE, fa.FA_ERR_NOT_DEVICE_MEMORY)
+    assert call(d=256) in (fa.FA_ERR_UNSUPPORTED_DEVICE, fa.FA_ERR_NOT_DEVICE_MEMORY)
     assert call(ds=(0.0, 1.0, 1.0)) == fa.FA_ERR_INVALID_ARG
     assert call(ds=(1.0, float("inf"), 1.0)) == fa.FA_ERR_INVALID_ARG
     assert call(ds=(1.0, 1.0, -2.0)) == fa.FA_ERR_INVALID_ARG

@@ -196,6 +196,25 @@ def test_fp8_small_shapes(orc, N, causal):
     check_full(orc, x, 1.0 / math.sqrt(128), causal, f"fp8 N={N} causal={causal}", dtype="e4m3")
 
 
+@pytest.mark.parametrize("d", [64, 256])
+@pytest.mark.parametrize("N", [1, 17, 129, 300, 600])
+@pytest.mark.parametrize("causal", [False, True])
+def test_fp8_head_dims(orc, d, N, causal):
+    """fa_fwd_fp8 at the other FP8 head dims (64-byte rows at d = 64; one query tile and two
+    S buffers at d = 256), several key tiles and a ragged tail, against the oracle."""
+    x = tiny(1, 2, 1, N, N, d, seed=N + d, dtype="e4m3")
+    check_full(orc, x, 1.0 / math.sqrt(d), causal, f"fp8 d={d} N={N} causal={causal}", dtype="e4m3")
+
+
+@pytest.mark.parametrize("d", [64, 256])
+def test_fp8_head_dims_gqa_descales(orc, d):
+    B, Hq, Hkv, Nq, Nk, causal, ds = 2, 8, 2, 200, 700, True, (0.5, 2.0, 0.25)
+    x = tiny(B, Hq, Hkv, Nq, Nk, d, seed=Nq + d, q_mult=4.0, dtype="e4m3")
+    scale = 1.0 / math.sqrt(d)
+    O, L = _parity.run_cuda_fp8(x, scale, causal, descale=ds)
+    _parity.compare_fp8(orc, x, O, L, scale, causal, descale=ds, what=f"fp8 d={d} gqa descales")
+
+
 @pytest.mark.parametrize("case", [(2, 8, 2, 200, 700, True, (0.5, 2.0, 0.25)), (1, 32, 8, 16, 3000, False, (1.0, 1.0, 4.0)),
                                   (2, 6, 3, 130, 129, True, (0.125, 0.75, 1.5)), (1, 4, 4, 1000, 1000, False, (2.0, 2.0, 0.5))])
 def test_fp8_gqa_descales(orc, case):
@@ -329,3 +348,23 @@ def test_workload_sampled_rows(orc, name):
     Ls = L[rows[:, 0], rows[:, 1], rows[:, 2]]
     res = _parity.compare(Os, Ls, Oref, Lref, name)
     print(name, len(rows), res)
+
+
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("window", [1, 77, 300])
+def test_f16_sliding_window(orc, d, window):
+    """fp16 inputs with the sliding-window mask (fa_fwd_window_f16), Nq != Nk, GQA."""
+    x = tiny(2, 4, 2, 333, 517, d, seed=window + d, dtype="f16")
+    O, L = _parity.run_cuda(x, 1.0 / math.sqrt(d), True, window=window, dtype="f16")
+    Oref, Lref = orc.forward(x["q"], x["k"], x["v"], 1.0 / math.sqrt(d), True, window=window, dtype="f16")
+    _parity.compare(O, L, Oref, Lref, f"f16 window={window} d={d}")
+
+
+@pytest.mark.parametrize("splits", [2, 7])
+@pytest.mark.parametrize("causal", [False, True])
+def test_f16_splitkv(orc, splits, causal):
+    """fp16 inputs through split-KV (fa_fwd_splitkv_f16): decode-shaped GQA rows, fp16 merge."""
+    x = tiny(2, 8, 2, 16, 2500, 128, seed=splits + 40, dtype="f16")
+    O, L = _parity.run_cuda(x, 0.09, causal, num_splits=splits, dtype="f16")
+    Oref, Lref = orc.forward(x["q"], x["k"], x["v"], 0.09, causal, dtype="f16")
+    _parity.compare(O, L, Oref, Lref, f"f16 splitkv S={splits} causal={causal}")
