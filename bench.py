@@ -48,11 +48,23 @@ def peaks():
     return dict(FALLBACK_PEAKS)
 
 
+def fp8_peak():
+    """Measured dense E4M3 GEMM throughput (TFLOP/s, burst) from profiles/fp8_gemm_peak.md, or None."""
+    f = ROOT / "profiles" / "fp8_gemm_peak.md"
+    if not f.exists():
+        return None
+    m = re.search(r"fp8_tflops_burst:\s*([0-9.]+)", f.read_text())
+    return float(m.group(1)) if m else None
+
+
 def tensor_peak(pk, w):
     """(TFLOP/s, source) of the tensor roofline for a workload's dtype: the measured bf16
-    figure (fp16 has the same nominal rate); E4M3 takes it x 2, the nominal dense fp8/bf16
-    ratio (4.5 / 2.25 PFLOP/s)."""
+    figure (fp16 has the same nominal rate); E4M3 takes the measured E4M3 GEMM figure, else
+    the bf16 one x 2 (the nominal dense fp8/bf16 ratio, 4.5 / 2.25 PFLOP/s)."""
     if w.dtype == "e4m3":
+        f8 = fp8_peak()
+        if f8 is not None:
+            return f8, "measured E4M3 GEMM 8192^3 (burst, profiles/fp8_gemm_peak.md)"
         return 2.0 * pk["bf16_tflops"], f"{pk['source']} bf16 dense (burst) x 2 (nominal fp8/bf16 ratio)"
     return pk["bf16_tflops"], f"{pk['source']} bf16 dense (burst)"
 
