@@ -33,6 +33,10 @@
  *  - Work is enqueued asynchronously on `stream`; no host synchronisation happens,
  *    except in fa_device_status.
  *  - A non-zero return means nothing was launched.
+ *  - Per device, the library looks up once (cudaGetSymbolAddress) and caches the addresses
+ *    of its device status word and of the static scratch of fa_fwd_splitkv_static.  A
+ *    cudaDeviceReset unloads the module behind them, so the library must not be called on a
+ *    device after cudaDeviceReset in the same process.
  */
 #ifndef EXACT_ATTENTION_FA_H
 #define EXACT_ATTENTION_FA_H
