@@ -527,6 +527,46 @@ def run_sweep(args):
     return 0
 
 
+def run_fp8_peak(args):
+    """Dense E4M3 GEMM throughput (cuBLASLt through torch._scaled_mm, 8192^3, bf16 out): the
+    best of 10 calls (burst) and back to back for 3 s (sustained).  One JSON line; the figures
+    committed in profiles/fp8_gemm_peak.md come from this mode."""
+    import torch
+    torch.cuda.set_device(0)
+    n = 8192
+    a = torch.randn(n, n, device="cuda").to(torch.float8_e4m3fn)
+    b = torch.randn(n, n, device="cuda").to(torch.float8_e4m3fn).t()
+    one = torch.tensor(1.0, device="cuda")
+
+    def mm():
+        return torch._scaled_mm(a, b, scale_a=one, scale_b=one, out_dtype=torch.bfloat16)
+
+    for _ in range(3):
+        mm()
+    torch.cuda.synchronize()
+    best = float("inf")
+    for _ in range(10):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        mm()
+        e1.record()
+        torch.cuda.synchronize()
+        best = min(best, e0.elapsed_time(e1))
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    calls, t0 = 0, time.time()
+    e0.record()
+    while time.time() - t0 < 3.0:
+        mm()
+        calls += 1
+    e1.record()
+    torch.cuda.synchronize()
+    flop = 2.0 * n ** 3
+    print(json.dumps({"fp8_tflops_burst": flop / best / 1e9,
+                      "fp8_tflops_sustained": flop / (e0.elapsed_time(e1) / calls) / 1e9,
+                      "n": n, "sustained_calls": calls}), flush=True)
+    return 0
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
@@ -543,6 +583,7 @@ def main(argv=None):
     ap.add_argument("--sweep", action="store_true", help="time every workload of the table (1 GPU)")
     ap.add_argument("--sweep-only", default="", help="comma-separated workload names for --sweep / --bwd-sweep")
     ap.add_argument("--bwd-sweep", action="store_true", help="time the backward pass on workloads of the table")
+    ap.add_argument("--fp8-peak", action="store_true", help="measure the dense E4M3 GEMM peak (1 GPU)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -550,6 +591,8 @@ def main(argv=None):
         return run_sweep(args)
     if args.bwd_sweep:
         return run_bwd_sweep(args)
+    if args.fp8_peak:
+        return run_fp8_peak(args)
     w = synth.WORKLOADS[args.workload]
     world, rank, local = dist_setup(args.gpus)
     if args.impl == "reference":
