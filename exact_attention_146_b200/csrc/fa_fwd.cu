@@ -258,13 +258,18 @@ int launch(const Problem &pr, DeviceState &dev, int cfg_slot, cudaStream_t strea
     p.causal = pr.causal;
     p.window = pr.window;
     p.pack = pack;
-    p.nqb = (pr.Nq * pack + C::NQT * kBlockQ - 1) / (C::NQT * kBlockQ);
+    // Causal / window masks with GQA: pair two query heads of a KV group in a unit (both tiles
+    // over the same rows, so they see the same key tiles and share every K/V load); otherwise
+    // a unit is NQT consecutive 128-row tiles of one head.
+    p.hpair = (C::NQT == 2 && pack == 1 && pr.causal && (pr.Hq / pr.Hkv) % 2 == 0) ? 1 : 0;
+    p.nqb = p.hpair ? (pr.Nq + kBlockQ - 1) / kBlockQ
+                    : (pr.Nq * pack + C::NQT * kBlockQ - 1) / (C::NQT * kBlockQ);
     const int nkv = (pr.Nk + C::BC - 1) / C::BC;
     p.num_splits = pr.num_splits > 1 ? pr.num_splits : 1;
     p.split_tiles = (nkv + p.num_splits - 1) / p.num_splits;
     p.o_part = pr.o_part;
     p.lse_part = pr.lse_part;
-    const long long units = (long long)pr.B * (pr.Hq / pack) * p.nqb * p.num_splits;
+    const long long units = (long long)pr.B * (pr.Hq / (p.hpair ? C::NQT : pack)) * p.nqb * p.num_splits;
     if (units > 0x7fffffffLL) return FA_ERR_INVALID_ARG;
     p.num_units = int(units);
     p.scale_log2 = pr.scale * 1.4426950408889634f;

@@ -80,6 +80,8 @@ struct FwdParams {
     unsigned long long wait_limit_ns;
     int withheld_load;
     int o_tma;            // 1: the epilogue writes O through shared memory and TMA stores (tm_o)
+    int hpair;            // 1: the two query tiles of a unit are two query heads of one KV group
+                          // over the same 128 query rows (same keys, so causal tiles end together)
 };
 
 // Compile-time tiling for one head dimension.
@@ -176,7 +178,8 @@ struct TileCfg {
                          B_PFULL = B_SFULL + NQT * SB,       // P_t written over buffer b
                          B_PHALF = B_PFULL + NQT * SB,       // its first 64 keys written (PSPLIT)
                          B_PVDONE = B_PHALF + NQT * SB,      // the P V MMA reading buffer b done
-                         B_ODONE = B_PVDONE + NQT * SB,      // a P V MMA of tile t done (rescale)
+                         B_ODONE = B_PVDONE + NQT * SB,      // a P V MMA of tile t done (rescale; with one S
+                                                             // buffer and P over S, PVDONE serves)
                          B_OFINAL = B_ODONE + NQT,           // the last P V of tile t in a unit done
                          B_OEMPTY = B_OFINAL + NQT,          // epilogue finished reading O_t
                          B_DRAIN = B_OEMPTY + NQT;
@@ -197,7 +200,8 @@ __device__ __forceinline__ UnitInfo decode_unit(int u, const FwdParams &p) {
     UnitInfo w;
     w.split = u % p.num_splits;
     u /= p.num_splits;
-    const int groups = p.Hq / p.pack;   // head groups (= Hq without packing)
+    const int hstep = p.hpair ? C::NQT : p.pack;   // query heads per unit
+    const int groups = p.Hq / hstep;               // head groups (= Hq without packing or pairing)
     const int bh = p.B * groups;
     int qb, r;
     if (p.causal) {
@@ -209,9 +213,9 @@ __device__ __forceinline__ UnitInfo decode_unit(int u, const FwdParams &p) {
         qb = u - r * p.nqb;
     }
     w.b = r / groups;
-    w.hq = (r - w.b * groups) * p.pack;
+    w.hq = (r - w.b * groups) * hstep;
     w.kvh = w.hq / p.n_rep;
-    w.q0 = qb * (C::NQT * kBlockQ);
+    w.q0 = qb * (p.hpair ? kBlockQ : C::NQT * kBlockQ);
     const int flat_rows = p.Nq * p.pack;
     const int nkv = (p.Nk + C::BC - 1) / C::BC;
     const int diag = p.diag;         // row i sees keys up to i + diag (causal / window)
@@ -220,7 +224,7 @@ __device__ __forceinline__ UnitInfo decode_unit(int u, const FwdParams &p) {
 #pragma unroll
     for (int t = 0; t < 2; ++t) {
         int js = 0, je = 0;
-        const int f_lo = w.q0 + t * kBlockQ;
+        const int f_lo = w.q0 + (p.hpair ? 0 : t * kBlockQ);
         if (t < C::NQT && f_lo < flat_rows) {
             const int q_lo = f_lo / p.pack;   // the tile's first and last query
             je = nkv;
@@ -338,8 +342,8 @@ __device__ void producer_role(const CUtensorMap *tm_q, const CUtensorMap *tm_k, 
             const uint32_t dst = sbase + C::SMEM_Q + (t * C::NQB + qb) * C::Q_TILE;
 #pragma unroll
             for (int c = 0; c < C::NCH; ++c)
-                sm100::tma_load_4d_elected(dst + c * C::Q_CHUNK, tm_q, fb, c * C::CW, w.hq,
-                                           (w.q0 + t * kBlockQ) / p.pack, w.b);
+                sm100::tma_load_4d_elected(dst + c * C::Q_CHUNK, tm_q, fb, c * C::CW, w.hq + (p.hpair ? t : 0),
+                                           (w.q0 + (p.hpair ? 0 : t * kBlockQ)) / p.pack, w.b);
         }
         for (int j = w.j_lo; ok && j < w.j_hi; ++j) {
 #pragma unroll
@@ -497,7 +501,7 @@ __device__ void mma_role(const FwdParams &p, uint32_t sbase, uint32_t tmem, cons
                 sm100::tc_fence_after_sync();
                 issue_pv<C>(sbase, tmem, t, slot, sb, j > w.js[t]);
             }
-            sm100::tc_commit_elected(bar(C::B_ODONE + t));
+            if (C::PSEP || C::SB != 1) sm100::tc_commit_elected(bar(C::B_ODONE + t));
             if (!C::PSEP) sm100::tc_commit_elected(bar(C::B_PVDONE + t * C::SB + sb));
             if (j == w.je[t] - 1) sm100::tc_commit_elected(bar(C::B_OFINAL + t));
             ++p_got[t];
@@ -677,7 +681,7 @@ __device__ void softmax_role(const FwdParams &p, const CUtensorMap *tm_o, uint32
     // the max held).
     auto rescale_o = [&](bool need, float alpha, uint32_t odone) -> bool {
         if (!__any_sync(0xffffffffu, need)) return true;
-        if (!warp_wait_bar(bar(C::B_ODONE + t), odone & 1u, ctl, kSiteODone)) return false;
+        if (!warp_wait_bar(bar((C::PSEP || C::SB != 1) ? C::B_ODONE + t : C::B_PVDONE + t * C::SB), odone & 1u, ctl, kSiteODone)) return false;
         sm100::tc_fence_after_sync();
 #pragma unroll
         for (int c = 0; c < C::O_CHUNKS; ++c) {
@@ -696,11 +700,11 @@ __device__ void softmax_role(const FwdParams &p, const CUtensorMap *tm_o, uint32
         const UnitInfo w = decode_unit<C>(u, p);
         const int js = w.js[t], je = w.je[t];
         const int nk = je - js;
-        const int f_lo = w.q0 + t * kBlockQ;       // flat row f = i * pack + (hq - w.hq)
+        const int f_lo = w.q0 + (p.hpair ? 0 : t * kBlockQ);   // flat row f = i * pack + (hq - w.hq)
         const int q_lo = f_lo / p.pack;            // the tile's first query
         const int f_row = f_lo + row_in_tile;
         const int row = f_row / p.pack;            // this thread's query i and head hq
-        const int hq = w.hq + (f_row - row * p.pack);
+        const int hq = w.hq + (p.hpair ? t : f_row - row * p.pack);
         const int diag = p.diag;                   // causal: key j visible to row i iff j <= i + diag
         const int row_lim = p.causal ? row + diag : 0x7fffffff;
         // sliding window: keys j > i + diag - W; the tile's first row has the lowest bound
@@ -820,7 +824,7 @@ __device__ void softmax_role(const FwdParams &p, const CUtensorMap *tm_o, uint32
                     sm100::fence_proxy_async_smem();
                     __syncwarp();
                     if (lane == 0 && row0 < p.Nq) {   // (a box wholly past Nq has nothing to write)
-                        sm100::tma_store_4d(tm_o, stage, 64 * c2, w.hq, row0, w.b);
+                        sm100::tma_store_4d(tm_o, stage, 64 * c2, w.hq + (p.hpair ? t : 0), row0, w.b);
                         sm100::bulk_commit_group();
                         sm100::bulk_wait_group_read0();   // the staging buffer may be rewritten
                     }
