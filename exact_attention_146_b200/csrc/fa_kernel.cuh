@@ -130,10 +130,10 @@ struct TileCfg {
     static constexpr int SMEM_BAR = SMEM_KV + NS * KV_TILE;
     static constexpr int NUM_BARS = 2 * NS + 2 * NQT * NQB + 4 * NQT * SB + 3 * NQT + 1;
     static constexpr int SMEM_MISC = SMEM_BAR + NUM_BARS * 8;
-    // Output staging (d = 64 .. 128): each softmax warp writes its 32 rows of O, 64 columns
-    // at a time, into 4 KB of its own (128-byte rows, 128-byte swizzle) and stores them with
-    // one TMA box, so the epilogue writes whole lines instead of one 16-byte piece per row.
-    static constexpr bool OSTAGE = (D >= 64 && D <= 128);
+    // Output staging (d >= 64): each softmax warp writes its 32 rows of O, 64 columns at a
+    // time, into 4 KB of its own (128-byte rows, 128-byte swizzle) and stores them with one
+    // TMA box, so the epilogue writes whole lines instead of one 16-byte piece per row.
+    static constexpr bool OSTAGE = (D >= 64);
     static constexpr int SMEM_OST = ((SMEM_MISC + 16 + 1023) / 1024) * 1024;
     static constexpr int OST_BYTES = OSTAGE ? 32 * 128 : 0;   // per warp
     // Each CTA holds all 512 TMEM columns, so ask for enough shared memory that a
