@@ -46,15 +46,15 @@ def _lse_merge(o_parts, l_parts):
 SHAPE = dict(B=2, Hq=4, Hkv=2, Nq=9, Nk=23, d=32)
 
 
-def _worker(rank, world, port, out):
+def _worker(rank, world, port, out, shape=None):
     import torch
     import torch.distributed as dist
     import oracle
     os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
     dist.init_process_group("gloo", rank=rank, world_size=world)
     try:
-        w = synth.Workload("kshard", 77, SHAPE["B"], SHAPE["Hq"], SHAPE["Hkv"], SHAPE["Nq"], SHAPE["Nk"], SHAPE["d"],
-                           False, seed=5)
+        sh = shape or SHAPE
+        w = synth.Workload("kshard", 77, sh["B"], sh["Hq"], sh["Hkv"], sh["Nq"], sh["Nk"], sh["d"], False, seed=5)
         x = synth.make_inputs(w)
         off, n = kshard.shard_range(w.Nk, rank, world)
         O, L = oracle.default().forward(x["q"], x["k"][:, off:off + n], x["v"][:, off:off + n], w.scale, False)
@@ -92,3 +92,25 @@ def test_exchange_by_rows_reproduces_full_attention(world):
         assert np.abs(o - Oref).max() < 1e-12 and np.abs(lse - Lref).max() < 1e-12
         assert received == world * n * w.Hq * w.d           # partial values this rank received
     assert sum(out[r][3] for r in range(world)) == rows
+
+
+def test_exchange_with_fewer_rows_than_ranks():
+    """Two query rows over three ranks: one rank owns no row; the exchange and the gather
+    still deliver every row, equal to the oracle over all keys."""
+    import oracle
+    shape = dict(B=1, Hq=2, Hkv=1, Nq=2, Nk=11, d=32)
+    ctx = mp.get_context("spawn")
+    out = ctx.Manager().dict()
+    port = _free_port()
+    procs = [ctx.Process(target=_worker, args=(r, 3, port, out, shape)) for r in range(3)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(120)
+        assert p.exitcode == 0
+    w = synth.Workload("kshard", 77, 1, 2, 1, 2, 11, 32, False, seed=5)
+    x = synth.make_inputs(w)
+    Oref, Lref = oracle.default().forward(x["q"], x["k"], x["v"], w.scale, False)
+    assert sorted(out[r][3] for r in range(3)) == [0, 1, 1]
+    for r in range(3):
+        assert np.abs(out[r][0] - Oref).max() < 1e-12 and np.abs(out[r][1] - Lref).max() < 1e-12
