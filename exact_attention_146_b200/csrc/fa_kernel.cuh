@@ -10,8 +10,10 @@
 //
 // How it maps onto a B200 SM (one CTA per SM, persistent over work units):
 //   * work unit = (batch b, query head hq, block of NQT x 128 query rows; with GQA
-//     packing the n_rep heads of one KV head share a unit, their rows stacked; with
-//     split-KV or a key-shard partial, also a slice of the key tiles);
+//     packing the n_rep heads of one KV head share a unit, their rows stacked; with a
+//     causal or window mask and GQA, the NQT tiles are NQT query heads of one KV head over
+//     the same 128 rows; with split-KV or a key-shard partial, also a slice of the key
+//     tiles); units are taken in a static snake order (sched_unit);
 //   * TMA warp (one thread): Q tiles once per unit, then K_j, V_j into an NS-slot
 //     shared-memory ring guarded by full/empty mbarriers;
 //   * MMA warp (one thread): S_t = Q_t K_j^T with tcgen05.mma into TMEM (fp32), and
@@ -25,8 +27,9 @@
 //     first half of P V overlaps the second half of the exponentials), keeps m and l in
 //     registers, rescales its O row in TMEM only when the max grew by more than
 //     2^8 (the final O / l is unchanged by the reference max used), and at the end
-//     writes O / l and LSE = (m + log2 l) ln 2 (split-KV / key shards: fp32 O / l and the
-//     slice's LSE to a workspace, combined by fa_splitkv_merge_kernel).
+//     writes O / l (d >= 64: through a per-warp shared-memory box and a TMA store) and
+//     LSE = (m + log2 l) ln 2 (split-KV / key shards: fp32 O / l and the slice's LSE to a
+//     workspace, combined by fa_splitkv_merge_kernel).
 // Every pipeline wait is bounded: after a time limit the kernel records
 // FA_ERR_DEVICE_TIMEOUT in a device status word, unwinds every role, waits for its own
 // in-flight copies and MMAs, frees TMEM and returns.
