@@ -159,13 +159,13 @@ template <bool H> using Cfg32 = TileCfg<32, 128, 2, 8, 2, 1, true, 2, H>;
 template <bool H> using Cfg64 = TileCfg<64, 128, 2, 8, 2, 1, true, 2, H>;
 template <bool H> using Cfg80 = TileCfg<80, 128, 2, 4, 1, 1, false, 0, H>;
 template <bool H> using Cfg96 = TileCfg<96, 128, 2, 4, 1, 1, false, 0, H>;
-template <bool H> using Cfg128 = TileCfg<128, 128, 2, 4, 1, 1, false, 0, H>;
+template <bool H> using Cfg128 = TileCfg<128, 128, 2, 4, 1, 1, true, 0, H, false, false, true>;
 template <bool H> using Cfg192 = TileCfg<192, 64, 2, 4, 1, 1, false, 0, H>;
 template <bool H> using Cfg256 = TileCfg<256, 64, 1, 4, 1, 2, false, 0, H>;
 // FP8 (E4M3) inputs.  d = 128: 16 KB tiles, so eight K/V slots; d = 64: 64-byte rows
 // (64-byte swizzle, 8 KB tiles); d = 256: one 128-row query tile with two S buffers (S 2 x 128
 // + O 256 TMEM columns), 32 KB tiles.  P is rounded to E4M3 over S (four per column).
-using Cfg128F8 = TileCfg<128, 128, 2, 8, 1, 1, false, 0, false, true>;
+using Cfg128F8 = TileCfg<128, 128, 2, 8, 1, 1, true, 0, false, true, false, true>;
 using Cfg64F8 = TileCfg<64, 128, 2, 8, 1, 1, false, 0, false, true>;
 using Cfg256F8 = TileCfg<256, 128, 1, 4, 1, 2, false, 0, false, true>;
 // The d = 64 bf16 tiling built for the failure-path test (fa_test_withheld_load): wait limit

@@ -18,9 +18,14 @@
 //     shared-memory ring guarded by full/empty mbarriers;
 //   * MMA warp (one thread): S_t = Q_t K_j^T with tcgen05.mma into TMEM (fp32), and
 //     O_t += P_t V_j with P read straight from TMEM (it overwrites S_t as bf16 / fp16 /
-//     E4M3, or has columns of its own for d <= 64);
+//     E4M3, or has columns of its own);
 //     the two query tiles are interleaved so that one tile's softmax runs while the
-//     tensor core works on the other tile;
+//     tensor core works on the other tile.  At d = 128 (bf16, fp16 and E4M3) the two
+//     tiles share ONE S buffer and P has columns of its own (S 128 + O 2 x 128 + P 2 x 64
+//     of the 512 TMEM columns): the next S, of either tile, is issued as soon as the
+//     softmax that owns the current one has loaded it into registers, so no tile's S
+//     waits for its own P V to finish reading P (the softmax instead waits for that P V
+//     before it stores the next P);
 //   * softmax warpgroup t (128 threads, thread r owns row r of tile t, which is TMEM
 //     lane r): loads its row of S_t, masks, takes the row max, p = 2^(s*scale*log2e - m)
 //     with one FFMA + ex2 per element, writes P back (in two halves for d <= 80, so the
@@ -52,7 +57,7 @@ constexpr int kStatusTimeout = 6;                     // = FA_ERR_DEVICE_TIMEOUT
 enum WaitSite : int {
     kSiteQEmpty = 1, kSiteKvEmpty = 2, kSiteKvFull = 3, kSiteQFull = 4, kSitePFull = 5,
     kSiteOEmpty = 6, kSiteSFull = 7, kSiteODone = 8, kSiteDrain = 9, kSiteProducerDrain = 10,
-    kSitePvDone = 11, kSiteOFinal = 12
+    kSitePvDone = 11, kSiteOFinal = 12, kSiteSEmpty = 13
 };
 
 struct FwdParams {
@@ -89,7 +94,7 @@ struct FwdParams {
 
 // Compile-time tiling for one head dimension.
 template <int D_, int BC_, int NQT_, int NS_, int NQB_ = 1, int SB_ = 1, bool PSEP_ = false, int SOFT_EXP_ = 0,
-          bool F16_ = false, bool FP8_ = false, bool FAULT_ = false>
+          bool F16_ = false, bool FP8_ = false, bool FAULT_ = false, bool SSHARE_ = false>
 struct TileCfg {
     static constexpr int D = D_;        // head dim
     static constexpr int BC = BC_;      // key/value rows per tile
@@ -103,6 +108,11 @@ struct TileCfg {
     static constexpr bool FP8 = FP8_;   // Q, K, V and P in OCP E4M3 (kind::f8f6f4); O stays bf16
     static constexpr bool FAULT = FAULT_;   // failure-path test build: wait limit from the
                                             // parameters, one K/V load withheld
+    // One S buffer for both query tiles (P in columns of its own): the next S, of either
+    // tile, is computed as soon as the softmax that owns the current one has read it into
+    // registers, so no tile's S waits for its own P V.  The two tiles' S tiles take turns
+    // in the buffer (S_0(j), S_1(j), S_0(j+1), ...).
+    static constexpr bool SSHARE = SSHARE_;
     static constexpr int ES = FP8 ? 1 : 2;                // bytes per Q/K/V/P element
     static constexpr int RB = (D * ES >= 128) ? 128 : 64; // bytes per swizzled smem row
     static constexpr int CW = RB / ES;                    // elements per swizzled smem row
@@ -112,7 +122,7 @@ struct TileCfg {
     // the softmax computes the second half of P.  Worth it where the exponentials dominate
     // (d <= 80: 6-10 % faster); at d >= 96 the extra register pressure costs more than the
     // overlap gains, so the hand-off stays whole there.
-    static constexpr bool PSPLIT = (BC == 128) && !FP8 && D <= 80;
+    static constexpr bool PSPLIT = (BC == 128) && !FP8 && D <= 80 && !SSHARE;
     static constexpr int NCH = (D + CW - 1) / CW;         // column chunks of a tile
     static constexpr int Q_CHUNK = kBlockQ * RB;
     static constexpr int KV_CHUNK = BC * RB;
@@ -120,10 +130,11 @@ struct TileCfg {
     static constexpr int KV_TILE = NCH * KV_CHUNK;
     static constexpr uint32_t LAYOUT = (RB == 128) ? 2u : 4u;   // UMMA 128B / 64B swizzle
     static constexpr int SBO = 8 * RB;                          // 8-row swizzle atom
-    // TMEM columns: S buffer b of tile t at (t*SB + b)*BC, O_t after all S buffers, and
-    // P_t either over the first BC/2 columns of its S buffer or (PSEP) after all O.
+    // TMEM columns: S buffer b of tile t at (t*SB + b)*BC (SSHARE: the one S buffer at 0),
+    // O_t after the S buffers, and P_t either over the first BC/2 columns of its S buffer
+    // or (PSEP) after all O.
     static constexpr int OST = (D == 256) ? 256 : ((D + 63) / 64) * 64;
-    static constexpr int O_COL0 = NQT * SB * BC;
+    static constexpr int O_COL0 = SSHARE ? BC : NQT * SB * BC;
     static constexpr int P_COL0 = O_COL0 + NQT * OST;
     static constexpr int TMEM_COLS = 512;
     static constexpr int O_CHUNKS = (D + 31) / 32;
@@ -131,7 +142,7 @@ struct TileCfg {
     static constexpr int SMEM_Q = 0;
     static constexpr int SMEM_KV = NQT * NQB * Q_TILE;
     static constexpr int SMEM_BAR = SMEM_KV + NS * KV_TILE;
-    static constexpr int NUM_BARS = 2 * NS + 2 * NQT * NQB + 4 * NQT * SB + 3 * NQT + 1;
+    static constexpr int NUM_BARS = 2 * NS + 2 * NQT * NQB + 4 * NQT * SB + 3 * NQT + 2;
     static constexpr int SMEM_MISC = SMEM_BAR + NUM_BARS * 8;
     // Output staging (d >= 64): each softmax warp writes its 32 rows of O, 64 columns at a
     // time, into 4 KB of its own (128-byte rows, 128-byte swizzle) and stores them with one
@@ -152,12 +163,13 @@ struct TileCfg {
     static constexpr int THREADS = 32 * (SOFTMAX_WARPS + 4);
     // Registers per thread: the launch budget (65536 / THREADS rounded down to 8) and,
     // for two query tiles, the split moved from the control warpgroup to the softmax
-    // warpgroups.  LAUNCH_REGS is checked against the compiled kernel on the host before
-    // the first launch.
+    // warpgroups.  The control share (88) keeps the MMA issuer's loop free of register
+    // spills; the softmax needs no more than 208.  LAUNCH_REGS is checked against the
+    // compiled kernel on the host before the first launch.
     static constexpr int LAUNCH_REGS = ((65536 / THREADS) / 8) * 8 > 255 ? 255 : ((65536 / THREADS) / 8) * 8;
     static constexpr bool REALLOC_REGS = (NQT == 2);
-    static constexpr int SOFTMAX_REGS = 216;
-    static constexpr int CONTROL_REGS = 72;
+    static constexpr int SOFTMAX_REGS = 208;
+    static constexpr int CONTROL_REGS = 88;
     static_assert(!REALLOC_REGS || (SOFTMAX_REGS * 32 * SOFTMAX_WARPS + CONTROL_REGS * 128 <= LAUNCH_REGS * THREADS),
                   "register split exceeds the launch budget");
     // format code 0 is F16 under kind::f16 and E4M3 under kind::f8f6f4
@@ -170,7 +182,8 @@ struct TileCfg {
     static_assert(D % 16 == 0 && D >= 32 && D <= 256, "MMA N and K granularity");
     static_assert(BC % 64 == 0 && BC <= 256, "key tile: whole 32-column TMEM chunks of P");
     static_assert(P_COL0 + (PSEP ? NQT * PCOLS : 0) <= TMEM_COLS, "TMEM budget");
-    static_assert(!FP8 || (!F16 && !PSEP && SOFT_EXP == 0 && BC % 128 == 0), "FP8 tiling");
+    static_assert(!FP8 || (!F16 && (!PSEP || SSHARE) && SOFT_EXP == 0 && BC % 128 == 0), "FP8 tiling");
+    static_assert(!SSHARE || (PSEP && SB == 1 && NQT == 2), "shared S tiling");
     static_assert(SMEM_BYTES <= 232448, "shared memory budget");
     // Barrier indices (Q barriers indexed t * NQB + buffer, S/P barriers t * SB + buffer).
     // Every barrier is waited on densely (each completion in order) by its waiter, except
@@ -185,7 +198,8 @@ struct TileCfg {
                                                              // buffer and P over S, PVDONE serves)
                          B_OFINAL = B_ODONE + NQT,           // the last P V of tile t in a unit done
                          B_OEMPTY = B_OFINAL + NQT,          // epilogue finished reading O_t
-                         B_DRAIN = B_OEMPTY + NQT;
+                         B_DRAIN = B_OEMPTY + NQT,
+                         B_SEMPTY = B_DRAIN + 1;             // SSHARE: the S buffer read into registers
 };
 
 struct UnitInfo {
@@ -397,7 +411,7 @@ __device__ __forceinline__ void issue_qk(uint32_t sbase, uint32_t tmem, int t, i
     // address stays below 256 KB, so the 14-bit field never carries).
     const uint64_t a0 = sm100::opaque(sm100::smem_desc(sbase + C::SMEM_Q + (t * C::NQB + qbuf) * C::Q_TILE, 16, C::SBO, C::LAYOUT));
     const uint64_t b0 = sm100::opaque(sm100::smem_desc(sbase + C::SMEM_KV + slot * C::KV_TILE, 16, C::SBO, C::LAYOUT));
-    const uint32_t d_tmem = tmem + uint32_t((t * C::SB + sbuf) * C::BC);
+    const uint32_t d_tmem = tmem + uint32_t(C::SSHARE ? 0 : (t * C::SB + sbuf) * C::BC);
 #pragma unroll
     for (int kk = 0; kk < C::D / C::KSTEP; ++kk) {
         constexpr int kCW = C::CW;
@@ -440,6 +454,7 @@ __device__ void mma_role(const FwdParams &p, uint32_t sbase, uint32_t tmem, cons
     uint32_t s_iss[2] = {0, 0};      // S tiles issued per query tile (S buffer = count % SB)
     uint32_t p_got[2] = {0, 0};      // P tiles consumed per query tile (= P V MMAs issued)
     uint32_t u_count = 0;            // units of this CTA so far (each releases O_EMPTY once)
+    uint32_t s_total = 0;            // SSHARE: S tiles issued into the shared buffer so far
     bool ok = true;
     auto wait_load = [&](uint32_t n, int &slot) -> bool {
         slot = int(n % C::NS);
@@ -471,6 +486,12 @@ __device__ void mma_role(const FwdParams &p, uint32_t sbase, uint32_t tmem, cons
         // S_t,j for query tile t, from the K tile in `slot`.
         auto issue_s = [&](int t, int j, int slot) -> bool {
             if (!wait_buffer_free(t)) return false;
+            if constexpr (C::SSHARE) {
+                // the shared buffer's previous S (of either tile) has been read by its softmax
+                if (s_total > 0 && !warp_wait_bar<kRoleControl>(bar(C::B_SEMPTY), (s_total - 1u) & 1u, ctl, kSiteSEmpty))
+                    return false;
+                ++s_total;
+            }
             sm100::tc_fence_after_sync();
             const int sb = int(s_iss[t] % C::SB);
             issue_qk<C>(sbase, tmem, t, qbuf[t], slot, sb);
@@ -554,6 +575,23 @@ __device__ void mma_role(const FwdParams &p, uint32_t sbase, uint32_t tmem, cons
                         if (ok && visits(t, jn) && !issue_s(t, jn, slot_k)) ok = false;
                     if (!ok) break;
                 }
+            } else if constexpr (C::SSHARE) {
+                // Per tile, the next S (as soon as the shared buffer is free) then this
+                // P V: S_0(j+1), P_0(j) V_j, S_1(j+1), P_1(j) V_j.
+#pragma unroll
+                for (int t = 0; t < C::NQT; ++t) {
+                    if (!ok) break;
+                    if (visits(t, jn)) {
+                        if (!k_ready) {
+                            if (!wait_load(kv_base + 2u * (jn - w.j_lo), slot_k)) { ok = false; break; }
+                            k_ready = true;
+                        }
+                        if (!issue_s(t, jn, slot_k)) { ok = false; break; }
+                    }
+                    if (visits(t, j) && !issue_o(t, j, slot_v)) { ok = false; break; }
+                }
+                if (!ok) break;
+                sm100::tc_commit_elected(bar(C::B_EMPTY + slot_v));
             } else {
                 // One S buffer: per tile, P V then (once it is done) the next S.
 #pragma unroll
@@ -591,9 +629,9 @@ __device__ void mma_role(const FwdParams &p, uint32_t sbase, uint32_t tmem, cons
 // hardware ex2 throughout.
 // FP8 P: four exponentials per 32-bit TMEM column (E4M3 bytes), 128 keys per store of
 // 32 columns; the row sum is taken over the unrounded fp32 values, like the LSE.
-template <int BC>
+template <int BC, bool DEFER = false>
 __device__ __forceinline__ float exp_pack_store_e4m3(const uint32_t (&s)[BC], float c_log2, float neg_m,
-                                                     uint32_t p_taddr) {
+                                                     uint32_t p_taddr, uint32_t (*pk_all)[32] = nullptr) {
     const uint64_t c2 = sm100::pack2(c_log2, c_log2);
     const uint64_t nm2 = sm100::pack2(neg_m, neg_m);
     uint64_t acc0 = sm100::pack2(0.f, 0.f), acc1 = acc0;
@@ -614,6 +652,11 @@ __device__ __forceinline__ float exp_pack_store_e4m3(const uint32_t (&s)[BC], fl
             acc1 = sm100::add2(acc1, sm100::pack2(p2, p3));
             pk[i] = sm100::pack_e4m3x4(p0, p1, p2, p3);
         }
+        if constexpr (DEFER) {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) pk_all[c][i] = pk[i];
+            continue;
+        }
         sm100::tmem_st32(p_taddr + uint32_t(32 * c), pk);
     }
     float a0, a1, b0, b1;
@@ -622,9 +665,12 @@ __device__ __forceinline__ float exp_pack_store_e4m3(const uint32_t (&s)[BC], fl
     return (a0 + a1) + (b0 + b1);
 }
 
-template <int BC, int SOFT_EXP, bool MIXED, bool F16, bool SPLIT = false>
+// DEFER: nothing is stored; the packed P is left in pk_all for the caller to store once the
+// P V MMA still reading this tile's P buffer has completed.
+template <int BC, int SOFT_EXP, bool MIXED, bool F16, bool SPLIT = false, bool DEFER = false>
 __device__ __forceinline__ float exp_pack_store(const uint32_t (&s)[BC], float c_log2, float neg_m,
-                                                uint32_t p_taddr, uint32_t half_bar = 0) {
+                                                uint32_t p_taddr, uint32_t half_bar = 0,
+                                                uint32_t (*pk_all)[32] = nullptr) {
     const uint64_t c2 = sm100::pack2(c_log2, c_log2);
     const uint64_t nm2 = sm100::pack2(neg_m, neg_m);
     uint64_t acc0 = sm100::pack2(0.f, 0.f), acc1 = acc0;
@@ -650,6 +696,11 @@ __device__ __forceinline__ float exp_pack_store(const uint32_t (&s)[BC], float c
             sm100::unpack2(p2, lo, hi);
             pk[i] = sm100::pack_x2<F16>(lo, hi);
         }
+        if constexpr (DEFER) {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) pk_all[c][i] = pk[i];
+            continue;
+        }
         sm100::tmem_st32(p_taddr + uint32_t(32 * c), pk);
         if constexpr (SPLIT) {
             if (c == 0) {   // first 64 keys of P (and any rescale of O before it) are in TMEM
@@ -674,7 +725,7 @@ __device__ void softmax_role(const FwdParams &p, const CUtensorMap *tm_o, uint32
     const int quarter = warp % 4;                  // TMEM lanes 32*quarter .. +31
     const int row_in_tile = quarter * 32 + lane;
     const uint32_t lane_off = uint32_t(quarter * 32) << 16;
-    const uint32_t s_taddr0 = tmem + lane_off + uint32_t(t * C::SB * BC);   // S buffer 0 of this tile
+    const uint32_t s_taddr0 = tmem + lane_off + uint32_t(C::SSHARE ? 0 : t * C::SB * BC);   // S buffer 0 of this tile
     const uint32_t p_taddr_sep = tmem + lane_off + uint32_t(C::P_COL0 + t * C::PCOLS);
     const uint32_t o_taddr = tmem + lane_off + uint32_t(C::O_COL0 + t * C::OST);
     const float c_log2 = p.scale_log2;
@@ -726,6 +777,11 @@ __device__ void softmax_role(const FwdParams &p, const CUtensorMap *tm_o, uint32
             uint32_t s[BC];
             if constexpr (BC == 128) sm100::tmem_ld128_sync(s_taddr, s);
             else sm100::tmem_ld64_sync(s_taddr, s);
+            if constexpr (C::SSHARE) {
+                // S is in registers: the shared buffer may take the next S (either tile's)
+                sm100::tc_fence_before_sync();
+                sm100::mbar_arrive(bar(C::B_SEMPTY));
+            }
 
             const int k_lo = j * BC;
             // boundary tiles: the key tail, the causal diagonal, the window's lower edge
@@ -766,7 +822,23 @@ __device__ void softmax_role(const FwdParams &p, const CUtensorMap *tm_o, uint32
                     if (!rescale_o(need_rescale, alpha, ocnt + uint32_t(j - js) - 1u)) goto unwind;
                 const float neg_m = (m_ref == -INFINITY) ? 0.f : -m_ref;
                 const uint32_t half_bar = bar(C::B_PHALF + t * C::SB + sb);
-                if constexpr (C::FP8)
+                if constexpr (C::SSHARE) {
+                    // P_t's columns are free once the previous P_t V has completed (the
+                    // first P of a unit: the epilogue's wait for the unit's last P V)
+                    constexpr int kChunks = C::PCOLS / 32;
+                    uint32_t pk_all[kChunks][32];
+                    if constexpr (C::FP8)
+                        row_sum = exp_pack_store_e4m3<BC, true>(s, c_log2, neg_m, p_taddr, pk_all);
+                    else
+                        row_sum = need_mask
+                                      ? exp_pack_store<BC, C::SOFT_EXP, false, C::F16, false, true>(s, c_log2, neg_m, p_taddr, 0, pk_all)
+                                      : exp_pack_store<BC, C::SOFT_EXP, true, C::F16, false, true>(s, c_log2, neg_m, p_taddr, 0, pk_all);
+                    if (j > js && !warp_wait_bar(bar(C::B_ODONE + t), (ocnt + uint32_t(j - js) - 1u) & 1u, ctl, kSiteODone))
+                        goto unwind;
+                    sm100::tc_fence_after_sync();
+#pragma unroll
+                    for (int c = 0; c < kChunks; ++c) sm100::tmem_st32(p_taddr + uint32_t(32 * c), pk_all[c]);
+                } else if constexpr (C::FP8)
                     row_sum = exp_pack_store_e4m3<BC>(s, c_log2, neg_m, p_taddr);
                 else
                     row_sum = need_mask
@@ -926,6 +998,7 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             sm100::mbar_init(bar(C::B_OEMPTY + t), 128);
         }
         sm100::mbar_init(bar(C::B_DRAIN), 1);
+        sm100::mbar_init(bar(C::B_SEMPTY), 128);
         *abort_flag = 0;
         sm100::fence_mbar_init();
     }
