@@ -152,21 +152,26 @@ using namespace fa_host;
 
 // Tiling per head dim: TileCfg<d, key rows per tile, query tiles per unit, K/V slots,
 // buffers per Q tile, S buffers per Q tile, P in TMEM columns of its own, exponential
-// pairs per 8 on the FMA pipe, fp16 elements (H) instead of bf16>.  d = 256 runs one 128-row query tile, so it has TMEM room
-// for a second S buffer (S_{j+1} computed while the softmax works on S_j); d <= 64 has
-// room to keep P apart from S, and is where the exponentials dominate.
+// pairs per 8 on the FMA pipe, fp16 elements (H) instead of bf16, E4M3, failure-path
+// build, one S buffer shared by the two query tiles>.  d = 80 ... 192: the two query tiles
+// take turns in one S buffer and P has columns of its own (S + O_0 + O_1 + P_0 + P_1 fit
+// the 512 TMEM columns), so no tile's next S waits for its own P V.  d = 256 runs one
+// 128-row query tile, so it has TMEM room for a second S buffer (S_{j+1} computed while the
+// softmax works on S_j); d <= 64 keeps an S buffer per tile with P apart from S (handed
+// over in two halves), and is where the exponentials dominate.
 template <bool H> using Cfg32 = TileCfg<32, 128, 2, 8, 2, 1, true, 2, H>;
 template <bool H> using Cfg64 = TileCfg<64, 128, 2, 8, 2, 1, true, 2, H>;
-template <bool H> using Cfg80 = TileCfg<80, 128, 2, 4, 1, 1, false, 0, H>;
-template <bool H> using Cfg96 = TileCfg<96, 128, 2, 4, 1, 1, false, 0, H>;
+template <bool H> using Cfg80 = TileCfg<80, 128, 2, 4, 1, 1, true, 0, H, false, false, true>;
+template <bool H> using Cfg96 = TileCfg<96, 128, 2, 4, 1, 1, true, 0, H, false, false, true>;
 template <bool H> using Cfg128 = TileCfg<128, 128, 2, 4, 1, 1, true, 0, H, false, false, true>;
-template <bool H> using Cfg192 = TileCfg<192, 64, 2, 4, 1, 1, false, 0, H>;
+template <bool H> using Cfg192 = TileCfg<192, 64, 2, 4, 1, 1, true, 0, H, false, false, true>;
 template <bool H> using Cfg256 = TileCfg<256, 64, 1, 4, 1, 2, false, 0, H>;
 // FP8 (E4M3) inputs.  d = 128: 16 KB tiles, so eight K/V slots; d = 64: 64-byte rows
-// (64-byte swizzle, 8 KB tiles); d = 256: one 128-row query tile with two S buffers (S 2 x 128
-// + O 256 TMEM columns), 32 KB tiles.  P is rounded to E4M3 over S (four per column).
+// (64-byte swizzle, 8 KB tiles); both with the shared S buffer and P (E4M3, four per
+// column) in columns of its own.  d = 256: one 128-row query tile with two S buffers
+// (S 2 x 128 + O 256 TMEM columns), 32 KB tiles, P rounded to E4M3 over S.
 using Cfg128F8 = TileCfg<128, 128, 2, 8, 1, 1, true, 0, false, true, false, true>;
-using Cfg64F8 = TileCfg<64, 128, 2, 8, 1, 1, false, 0, false, true>;
+using Cfg64F8 = TileCfg<64, 128, 2, 8, 1, 1, true, 0, false, true, false, true>;
 using Cfg256F8 = TileCfg<256, 128, 1, 4, 1, 2, false, 0, false, true>;
 // The d = 64 bf16 tiling built for the failure-path test (fa_test_withheld_load): wait limit
 // taken from the parameters, one K/V load left out by the producer.

@@ -20,9 +20,9 @@
 //     O_t += P_t V_j with P read straight from TMEM (it overwrites S_t as bf16 / fp16 /
 //     E4M3, or has columns of its own);
 //     the two query tiles are interleaved so that one tile's softmax runs while the
-//     tensor core works on the other tile.  At d = 128 (bf16, fp16 and E4M3) the two
-//     tiles share ONE S buffer and P has columns of its own (S 128 + O 2 x 128 + P 2 x 64
-//     of the 512 TMEM columns): the next S, of either tile, is issued as soon as the
+//     tensor core works on the other tile.  At d = 80 ... 192 (and E4M3 at d = 64, 128) the
+//     two tiles share ONE S buffer and P has columns of its own (d = 128: S 128 + O 2 x 128
+//     + P 2 x 64 of the 512 TMEM columns): the next S, of either tile, is issued as soon as the
 //     softmax that owns the current one has loaded it into registers, so no tile's S
 //     waits for its own P V to finish reading P (the softmax instead waits for that P V
 //     before it stores the next P);
