@@ -33,7 +33,8 @@ def cuda_ready():
 
 @pytest.mark.parametrize("R", [1, 2, 3, 5])
 @pytest.mark.parametrize("causal", [False, True])
-@pytest.mark.parametrize("shape", [(1, 4, 2, 300, 1000, 128), (2, 2, 2, 129, 129, 64), (1, 8, 8, 700, 450, 128)])
+@pytest.mark.parametrize("shape", [(1, 4, 2, 300, 1000, 128), (2, 2, 2, 129, 129, 64), (1, 8, 8, 700, 450, 128),
+                                   (1, 4, 4, 333, 700, 96)])
 def test_sharded_equals_full(orc, R, causal, shape):
     import torch
     import exact_attention_146_b200 as fa

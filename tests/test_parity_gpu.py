@@ -125,6 +125,48 @@ def test_splitkv(orc, d, Nq, Nk, splits, causal):
     _parity.compare(O, L, Oref, Lref, f"splitkv d={d} Nq={Nq} Nk={Nk} S={splits} causal={causal}")
 
 
+# The head dims whose two query tiles take turns in one TMEM S buffer (P in columns of its
+# own); d = 128 is covered by the tests above and the full-size workloads.
+SHARED_S_DIMS = (80, 96, 192)
+
+
+@pytest.mark.parametrize("d", SHARED_S_DIMS)
+@pytest.mark.parametrize("N,W", [(300, 1), (300, 129), (700, 250), (700, 1000)])
+def test_shared_s_sliding_window(orc, d, N, W):
+    x = tiny(1, 2, 1, N, N, d, seed=N + W + d + 1)
+    O, L = _parity.run_cuda(x, 1.0 / math.sqrt(d), True, window=W)
+    Oref, Lref = orc.forward(x["q"], x["k"], x["v"], 1.0 / math.sqrt(d), True, window=W)
+    _parity.compare(O, L, Oref, Lref, f"window d={d} N={N} W={W}")
+
+
+@pytest.mark.parametrize("d", SHARED_S_DIMS)
+@pytest.mark.parametrize("Nq,Nk,splits,causal", [(1, 1000, 3, False), (16, 2049, 7, True), (130, 700, 2, True),
+                                                 (130, 700, 40, False)])
+def test_shared_s_splitkv(orc, d, Nq, Nk, splits, causal):
+    x = tiny(1, 4, 2, Nq, Nk, d, seed=Nq + Nk + splits + d + 1)
+    O, L = _parity.run_cuda(x, 1.0 / math.sqrt(d), causal, num_splits=splits)
+    Oref, Lref = orc.forward(x["q"], x["k"], x["v"], 1.0 / math.sqrt(d), causal)
+    _parity.compare(O, L, Oref, Lref, f"splitkv d={d} Nq={Nq} Nk={Nk} S={splits} causal={causal}")
+
+
+@pytest.mark.parametrize("d", SHARED_S_DIMS)
+def test_shared_s_rescale_path(orc, d):
+    """Q x 8: the row maxima keep growing, so O is rescaled between P V products."""
+    x = tiny(2, 4, 4, 700, 700, d, seed=61 + d, q_mult=8.0)
+    check_full(orc, x, 1.0 / math.sqrt(d), False, f"qx8 d={d}")
+    check_full(orc, x, 1.0 / math.sqrt(d), True, f"qx8 causal d={d}")
+
+
+@pytest.mark.parametrize("d", SHARED_S_DIMS)
+@pytest.mark.parametrize("Hkv", [1, 4])
+def test_shared_s_causal_tile_ranges(orc, d, Hkv):
+    """Causal with Hq == Hkv: the unit's two query tiles see different numbers of key tiles
+    (the second one more), so the shared buffer's turns are uneven; Hkv = 1: the causal GQA
+    units pair two query heads over the same rows."""
+    x = tiny(1, 4, Hkv, 600, 600, d, seed=80 + d + Hkv)
+    check_full(orc, x, 1.0 / math.sqrt(d), True, f"causal d={d} Hkv={Hkv}")
+
+
 @pytest.mark.parametrize("n_rep", [2, 4, 8, 16, 32])
 @pytest.mark.parametrize("Nq", [1, 5, 16, 33, 127])
 @pytest.mark.parametrize("causal", [False, True])
