@@ -163,10 +163,10 @@ __device__ __forceinline__ Unit decode_unit(int u, const BwdParams &p) {
     return w;
 }
 
-// The static schedule: in round r the CTAs take units r * G .. r * G + G - 1 (G = gridDim.x),
-// CTA i unit r * G + i in even rounds and r * G + G - 1 - i in odd ones.  The causal order
+// The static schedule: in pass r the CTAs take units r * G .. r * G + G - 1 (G = gridDim.x),
+// CTA i unit r * G + i in even passes and r * G + G - 1 - i in odd ones.  The causal order
 // puts the key tiles with the most query tiles first, so alternating the direction pairs the
-// CTAs that drew the longest units of one round with the shortest of the next (the busiest
+// CTAs that drew the longest units of one pass with the shortest of the next (the busiest
 // CTA 1.6 % above the mean on the causal GQA 4K workload, where a plain stride left it 13.7 %
 // above).  Every role walks the same sequence; an index past the end is skipped by all.
 __device__ __forceinline__ int sched_unit(int r) {

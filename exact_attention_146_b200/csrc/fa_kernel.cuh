@@ -271,13 +271,13 @@ __device__ __forceinline__ UnitInfo decode_unit(int u, const FwdParams &p) {
     return w;
 }
 
-// The static schedule: in round r the CTAs take units r * G .. r * G + G - 1 (G = gridDim.x),
-// CTA i unit r * G + i in even rounds and r * G + G - 1 - i in odd ones (a snake order).
+// The static schedule: in pass r the CTAs take units r * G .. r * G + G - 1 (G = gridDim.x),
+// CTA i unit r * G + i in even passes and r * G + G - 1 - i in odd ones (a snake order).
 // The causal order sorts units longest first, so alternating the direction pairs the CTAs
-// that drew the longest units of one round with the shortest of the next: the busiest CTA
+// that drew the longest units of one pass with the shortest of the next: the busiest CTA
 // ends within about 1 % of the mean on the causal 4K and 16K workloads, where a plain
 // stride left it 6-7 % above.  Every role walks the same sequence; a unit index past the
-// end (only in the schedule's last round) is skipped by all of them.
+// end (only in the schedule's last pass) is skipped by all of them.
 __device__ __forceinline__ int sched_unit(int r) {
     const int g = int(gridDim.x), i = int(blockIdx.x);
     return r * g + ((r & 1) ? g - 1 - i : i);
